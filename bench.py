@@ -1,0 +1,401 @@
+"""Benchmark of the fused ZeRO-1/2 sharded optimizer step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl zr|reference]
+                    [--config NAME] [--no-cpu-baseline]
+
+One step = one zr_step() call on one rank's owned shard: the W-replica bf16
+gradient reduce, (the global-norm clip when the workload has it), AdamW on
+the fp32 master / m / v, and the bf16 write into the all-gather buffer.
+Inputs are seeded synthetic data resident in HBM before the timed region;
+each step's bytes exceed the 126 MB L2, so no flush is needed between steps.
+
+N > 1 (torchrun, one process per GPU): process i runs ZeRO rank i mod W of
+the same workload on its own GPU -- independent shards, no data-path
+collective (weak scaling); the step time is the max over processes.
+
+--impl reference times the oracle (plain single-threaded C on the host) on a
+bounded sample of the same workload and prints the same JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "owned Gparams/s of fused reduce+AdamW step; achieved HBM GB/s vs B200 peak"
+UNIT = "Gparams/s"
+DEFAULT_CONFIG = "gpt2_124m_w8"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCE = os.path.join(ROOT, "sharded_optimizer_step_zr_b200", "csrc", "zr_kernels.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="zr", choices=["zr", "reference"])
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def workload(name):
+    import synth
+    if name in synth.WORKLOADS:
+        return synth.WORKLOADS[name]
+    for wl in synth.sweep_workloads():
+        if wl.name == name:
+            return wl
+    raise SystemExit(f"unknown config {name}")
+
+
+def bytes_per_owned_param(W, clip):
+    """Algorithmic bytes: 2W gradient reads + 12 state reads + 12 state
+    writes + 2 bf16 writes (+ the clip pass: fp32 g scratch written and read
+    back when W > 4, the gradients read again when W <= 4)."""
+    b = 2 * W + 26
+    if clip:
+        b += 8 if W > 4 else 2 * W
+    return b
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    with open(KERNEL_SOURCE, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(workload_name):
+    """dram__bytes_read.sum + dram__bytes_write.sum per launch of the step's
+    dominant kernel from the committed ncu summary, if it was taken on the
+    current kernel source; else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+        e = d.get(workload_name)
+        if e and e.get("kernel_source_sha256_16") == kernel_source_hash():
+            return float(e["bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """NVML samples of SM clock and throttle reasons while the timed region runs."""
+
+    def __init__(self, device_index):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            self._ok = False
+
+    def _run(self):
+        nv = self._nv
+        names = {
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for k, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self._ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# CPU arm: the oracle on a bounded sample
+# ---------------------------------------------------------------------------
+
+def oracle_sample_rate(wl, rank, target_seconds, max_elems=1 << 21):
+    """Time the oracle's rank step (single thread) on the first owned
+    elements of `rank` for the workload's gradient statistics; repeat steps
+    until `target_seconds` of CPU work.  Returns (Gparams/s, description)."""
+    import numpy as np
+    import oracle
+    import synth
+    oplan = oracle.Plan(wl.shapes, wl.world_size, wl.mode, wl.bucket_cap_bytes)
+    n = min(int(oplan.owned_numel[rank]), max_elems)
+    # the sample: owned elements [0, n) of this rank, as their own small plan
+    # with the same W (flat, one tensor of n elements owned by every rank)
+    idx = oplan.owned_global_index(rank)[:n]
+    import torch
+    t_idx = torch.from_numpy(idx)
+    grads = [synth.grad_bf16(wl.seed, 1, w, t_idx, wl.grad_sigma, wl.outlier_frac,
+                             n_valid=oplan.total_numel).view(torch.int16).numpy().view(np.uint16).copy()
+             for w in range(wl.world_size)]
+    master = synth.master_f32(wl.seed, t_idx, n_valid=oplan.total_numel).numpy().copy()
+    m = np.zeros(n, np.float32)
+    v = np.zeros(n, np.float32)
+    sample_plan = oracle.Plan([(n * wl.world_size,)], wl.world_size, oracle.FLAT, 1 << 62)
+    out = np.zeros(sample_plan.padded_numel, np.uint16)
+    clip = 1.0 if wl.max_grad_norm > 0 else None
+    steps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.rank_step(sample_plan, 0, grads, master, m, v, out, wl.hp, steps + 1, clip=clip)
+        if clip is not None:
+            oracle.sumsq(oracle.reduce(grads))      # the clip's extra reduce pass
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= target_seconds:
+            break
+    rate = n * steps / el / 1e9
+    desc = (f"oracle rank_step on {n} of rank {rank}'s {int(oplan.owned_numel[rank])} owned params "
+            f"(W={wl.world_size}), {steps} steps, {el:.1f} s, 1 thread")
+    return rate, desc
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = workload(args.config)
+    K, Wm = args.steps, args.warmup
+    budget = max(0.05, min(2.0, 120.0 / max(1, K + Wm)))
+    rates = []
+    desc = ""
+    for i in range(Wm + K):
+        r, desc = oracle_sample_rate(wl, wl.ranks[0], budget, max_elems=1 << 18)
+        if i >= Wm:
+            rates.append(r)
+    value = statistics.median(rates)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": K, "warmup": Wm, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "param_set": wl.param_set, "W": wl.world_size,
+                   "rank": wl.ranks[0], "partition": "flat" if wl.mode == 0 else "whole_tensor",
+                   "bucket_cap_mb": wl.bucket_cap_mb},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_zr(args):
+    import torch
+    import synth
+    from sharded_optimizer_step_zr_b200.plan import ZrPlan
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    grank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    wl = workload(args.config)
+    W = wl.world_size
+    zr_rank = wl.ranks[0] if world == 1 else (wl.ranks[0] + grank) % W
+    clip = wl.max_grad_norm > 0
+    plan = ZrPlan(wl.shapes, W, zr_rank, wl.mode, wl.bucket_cap_bytes, *wl.hp, device=dev)
+    n = plan.owned_numel
+    runs = plan.runs()
+    stream = torch.cuda.current_stream()
+
+    grads = [torch.empty(n, dtype=torch.bfloat16, device=dev) for _ in range(W)]
+    for w in range(W):
+        synth.fill_owned_grad(grads[w], runs, wl.seed, 1, w, wl.grad_sigma, wl.outlier_frac,
+                              n_valid=plan.total_numel)
+    master = torch.empty(n, dtype=torch.float32, device=dev)
+    synth.fill_owned_master(master, runs, wl.seed, n_valid=plan.total_numel)
+    m = torch.zeros_like(master)
+    v = torch.zeros_like(master)
+    param_out = torch.zeros(plan.padded_numel, dtype=torch.bfloat16, device=dev)
+    if clip:
+        # other ranks' sums of squares: the emulated scalar all-gather
+        plan.grad_sumsq(grads, plan.partials[zr_rank:zr_rank + 1])
+    torch.cuda.synchronize()
+
+    step_no = 0
+
+    def one_step():
+        nonlocal step_no
+        step_no += 1
+        plan.step(grads, master, m, v, param_out, step_no, stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(dev.index)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(K):
+            ev[i][0].record(stream)
+            one_step()
+            ev[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    per_launch_ms = [a.elapsed_time(b) for a, b in ev]
+    owned_total = n * K
+    if dist:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        o = torch.tensor([owned_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(o, op=dist.ReduceOp.SUM)
+        owned_total = float(o.item())
+    value = owned_total / (total_ms * 1e-3) / 1e9
+    ms_per_step = total_ms / K
+
+    # roofline of the step's kernels (one launch per step without clipping)
+    bpp = bytes_per_owned_param(W, clip)
+    alg_bytes = n * bpp
+    avg_ms = statistics.mean(per_launch_ms)
+    achieved = alg_bytes / (avg_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peak()
+    traffic = recorded_traffic(wl.name)
+
+    # end to end through zr_step_host: pinned host gradients in, result out
+    e2e = None
+    if not args.no_e2e:
+        host_grads = [g.cpu().pin_memory() for g in grads]
+        host_out = torch.empty(plan.padded_numel, dtype=torch.bfloat16).pin_memory()
+        for _ in range(3):
+            step_no += 1
+            plan.step_host(host_grads, grads, master, m, v, param_out, host_out, step_no, stream)
+        torch.cuda.synchronize()
+        K2 = max(3, min(K, 50))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(K2):
+            step_no += 1
+            plan.step_host(host_grads, grads, master, m, v, param_out, host_out, step_no, stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b)
+        e2e_owned = n * K2
+        if dist:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+            o = torch.tensor([e2e_owned], dtype=torch.float64, device=dev)
+            dist.all_reduce(o, op=dist.ReduceOp.SUM)
+            e2e_owned = float(o.item())
+        e2e = {"value": e2e_owned / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
+               "h2d_bytes_per_step": 2 * W * n, "d2h_bytes_per_step": 2 * n,
+               "steps": K2, "api": "zr_step_host"}
+
+    cpu = None
+    if grank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, desc = oracle_sample_rate(wl, zr_rank, args.cpu_seconds)
+        cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if grank != 0:
+        return
+    launches_per_step = 3 if clip else 1
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "param_set": wl.param_set, "W": W, "rank": zr_rank,
+                   "partition": "flat" if wl.mode == 0 else "whole_tensor",
+                   "bucket_cap_mb": wl.bucket_cap_mb, "clip": clip, "owned_params": n,
+                   "bytes_per_owned_param": bpp,
+                   "l2": f"no flush: each step touches {alg_bytes / 1e6:.0f} MB > 126 MB L2"},
+        "hbm_gbs": achieved,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
+                     "kernel": "zr_tile_kernel" if not clip else "zr_step (3 kernels)"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * K,
+        "clocks": sampler.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_zr(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,204 @@
+/*
+ * zr.h -- C ABI of the fused ZeRO-1/2 sharded optimizer step for NVIDIA B200
+ * (sm_100a).
+ *
+ * One step of data-parallel training with sharded optimizer state, for the
+ * slice of parameters that one rank owns:
+ *
+ *   1. reduce   g = (g_0 + g_1 + ... + g_{W-1}) / W   -- the W replicas'
+ *               bf16 gradients for the owned elements, summed in fp32 in
+ *               rank order, then divided by W.  This is the reduce half of
+ *               the gradient reduce-scatter ("CS336 lecture 8, parallelism
+ *               basics", ZeRO level 1 and its code sketch; "Scaling training
+ *               to thousands of GPUs", 03:41 DP: gradients are summed and
+ *               averaged over replicas; 11:24 ZeRO: AllReduce is
+ *               reduce-scatter + all-gather);
+ *   2. clip     optional: g <- g * min(1, max_norm / (||g||_global + 1e-6))
+ *               (not on those pages; the usual global-norm convention);
+ *   3. AdamW    on the owned slice's fp32 master weights p and moments m, v
+ *               (the pages name AdamW with fp32 master / m / v -- "DDP -> ZeRO"
+ *               blog section 1.1, "CS336" 16 bytes/param ledger; the rule is
+ *               bias-corrected Adam with decoupled weight decay):
+ *                 m = b1*m + (1-b1)*g ;  v = b2*v + (1-b2)*(g*g)
+ *                 p = p*(1 - lr*wd)
+ *                 p = p - (lr/(1-b1^t)) * m / (sqrt(v)/sqrt(1-b2^t) + eps)
+ *   4. cast     param_out[global position] = bf16(p), round to nearest even:
+ *               this rank's contribution to the parameter all-gather buffer
+ *               ("CS336", ZeRO-1 sketch, update-then-gather).
+ *
+ * The four stages run as one fused, memory-bound GPU pass (two passes and a
+ * tiny combine kernel when clipping).  All W replicas' gradients live in the
+ * memory of the one GPU the call runs on; there is no collective.
+ *
+ * Partitioning ("Scaling training to thousands of GPUs", 11:24 ZeRO, FSDP1
+ * vs FSDP2):
+ *   ZR_PARTITION_FLAT          tensors concatenated in declaration order and
+ *                              zero padded to W equal chunks of
+ *                              C = ceil(N/W); rank r owns [r*C, (r+1)*C).
+ *   ZR_PARTITION_WHOLE_TENSOR  every tensor owned whole by one rank, greedy
+ *                              longest-processing-time balance by element
+ *                              count (largest first, ties by declaration
+ *                              index; to the least-loaded rank, ties by
+ *                              lowest rank).  No padding.
+ * Buckets ("Scaling training ...", 03:41 DP, bucket_cap_mb; "DDP -> ZeRO"
+ * blog section 2.1): whole tensors packed in reverse declaration order; a new
+ * bucket opens when the next tensor's bf16 gradient bytes would push a
+ * non-empty bucket past bucket_cap_bytes.  The flat zero pad closes bucket 0.
+ *
+ * Layouts
+ *   global layout  all tensors, declaration order, flat (plus the flat pad);
+ *                  param_out is a bf16 buffer of padded_numel elements in it.
+ *   owned order    the order of this rank's elements: flat -> [r*C, (r+1)*C)
+ *                  as is; whole-tensor -> this rank's tensors in declaration
+ *                  order, concatenated.  master, m, v and every grad_ptrs[w]
+ *                  hold owned_numel elements in owned order.
+ *
+ * Ownership and errors
+ *   The caller allocates and owns every device buffer, including the
+ *   workspace; a plan owns host memory only.  Device-side calls are
+ *   asynchronous on the given stream and return the launch status; a fault
+ *   inside a kernel surfaces at the caller's next synchronisation.  On any
+ *   error status nothing has been launched.  Buffers must not overlap; the
+ *   gradient buffers are read-only.  A plan may be used from one host thread
+ *   at a time.
+ */
+#ifndef ZR_H_
+#define ZR_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; 0 is the legacy default stream. */
+typedef struct CUstream_st* zr_stream_t;
+
+typedef enum {
+    ZR_OK = 0,
+    ZR_ERR_INVALID_ARG = 1,   /* bad size, rank, mode, step, NULL pointer    */
+    ZR_ERR_ALIGNMENT = 2,     /* a device pointer not 16-byte aligned        */
+    ZR_ERR_NO_WORKSPACE = 3,  /* zr_plan_set_workspace not called / too small */
+    ZR_ERR_CUDA = 4,          /* a CUDA runtime call failed                  */
+    ZR_ERR_UNSUPPORTED = 5,   /* W above ZR_MAX_WORLD_SIZE, no sm_100 device */
+    ZR_ERR_BUFFER_TOO_SMALL = 6
+} zr_status;
+
+typedef enum { ZR_PARTITION_FLAT = 0, ZR_PARTITION_WHOLE_TENSOR = 1 } zr_partition;
+
+/* Largest W: the W gradient pointers travel by value in the kernel's
+ * parameter block. */
+#define ZR_MAX_WORLD_SIZE 512
+
+/* AdamW hyperparameters (fp32, as a training script holds them).
+ * max_grad_norm <= 0 disables clipping. */
+typedef struct {
+    float lr, beta1, beta2, eps, weight_decay, max_grad_norm;
+} zr_adamw;
+
+/* One piece of the partition: a run of `length` consecutive elements of
+ * tensor `tensor` (-1: the flat zero pad), starting at element
+ * `offset_in_tensor`, placed in bucket `bucket`, owned by rank `owner`, at
+ * `global_offset` in the global layout and `owned_offset` in the owner's
+ * owned order.  Segments are ordered by bucket, then by tensor in packing
+ * (reverse declaration) order, then by offset; the pad comes last in
+ * bucket 0. */
+typedef struct {
+    int32_t bucket, tensor, owner, reserved;
+    int64_t offset_in_tensor, length, global_offset, owned_offset;
+} zr_segment;
+
+typedef struct zr_plan zr_plan;
+
+/* Build the partition, bucket and segment tables for one rank (host only,
+ * no CUDA call).  n_tensors >= 0; ndims[t] >= 0; shapes[t] points to
+ * ndims[t] non-negative extents (a tensor of ndims 0 is a scalar).
+ * 1 <= world_size <= ZR_MAX_WORLD_SIZE, 0 <= rank < world_size.
+ * bucket_cap_bytes counts bf16 gradient bytes (2 per element).  *hp is
+ * copied.  On success *out receives a plan to release with zr_plan_destroy.
+ * Errors: ZR_ERR_INVALID_ARG (NULL pointers, negative extents, bad mode or
+ * rank, element counts overflowing int64), ZR_ERR_UNSUPPORTED (W too large). */
+zr_status zr_plan_create(int32_t n_tensors, const int32_t* ndims, const int64_t* const* shapes,
+                         int32_t world_size, int32_t rank, zr_partition mode,
+                         uint64_t bucket_cap_bytes, const zr_adamw* hp, zr_plan** out);
+
+/* Sizes of the plan.  Any output pointer may be NULL.  owned_numel is this
+ * rank's element count; n_segments counts all ranks' segments. */
+zr_status zr_plan_query(const zr_plan* plan, int64_t* total_numel, int64_t* padded_numel,
+                        int64_t* owned_numel, int32_t* n_buckets, int64_t* n_segments);
+
+/* Copy all ranks' segments (see zr_segment) into out[0..cap).  *n receives
+ * the total count; if it exceeds cap, nothing is written and
+ * ZR_ERR_BUFFER_TOO_SMALL is returned (call with cap 0 to size). */
+zr_status zr_plan_segments(const zr_plan* plan, zr_segment* out, int64_t cap, int64_t* n);
+
+/* Device workspace the plan needs: the tile table, the clip partial sums and
+ * (when clipping with W > 4) an fp32 scratch copy of the reduced gradient. */
+zr_status zr_plan_workspace_bytes(const zr_plan* plan, uint64_t* bytes);
+
+/* Bind a device workspace (>= zr_plan_workspace_bytes, 256-byte aligned,
+ * owned by the caller, kept alive while the plan is used) and upload the
+ * tile table into it with an asynchronous copy on `stream`.  Selects the
+ * current CUDA device as the plan's device.  Errors: ZR_ERR_NO_WORKSPACE
+ * (too small), ZR_ERR_ALIGNMENT, ZR_ERR_UNSUPPORTED (the current device is
+ * not compute capability 10.x), ZR_ERR_CUDA. */
+zr_status zr_plan_set_workspace(zr_plan* plan, void* d_workspace, uint64_t bytes,
+                                zr_stream_t stream);
+
+/* Clipping only.  d_partials: device array of world_size doubles, entry w =
+ * rank w's sum of squares S_w of its averaged owned gradient.  zr_step
+ * writes this rank's entry itself; the other entries must hold the other
+ * ranks' S_w (from zr_grad_sumsq, or from a scalar all-gather across GPUs)
+ * before zr_step runs on the stream.  The clip norm is
+ * sqrt(S_0 + S_1 + ... + S_{W-1}), summed in rank order in fp64, so every
+ * rank derives the same coefficient. */
+zr_status zr_plan_set_sumsq_partials(zr_plan* plan, double* d_partials);
+
+/* The optimizer step for this rank (stages 1-4 above).
+ * grad_ptrs: host array of world_size device pointers, replica w's bf16
+ *            gradient for this rank's owned elements in owned order.
+ * master, m, v: fp32 device arrays of owned_numel, updated in place.
+ * param_out: bf16 device array of padded_numel (global layout); only this
+ *            rank's positions are written.
+ * step: 1-based AdamW step count t (bias corrections use it).
+ * Every device pointer must be 16-byte aligned.  With owned_numel == 0 it
+ * returns ZR_OK and launches nothing.
+ * Errors: ZR_ERR_INVALID_ARG, ZR_ERR_ALIGNMENT, ZR_ERR_NO_WORKSPACE (also:
+ * clipping enabled and no partials array bound), ZR_ERR_CUDA. */
+zr_status zr_step(const zr_plan* plan, const void* const* grad_ptrs, float* master, float* m,
+                  float* v, void* param_out, int64_t step, zr_stream_t stream);
+
+/* zr_step with host-resident gradients and a host copy of the result, for
+ * callers whose gradients arrive in host memory.  On `stream`: copies
+ * host_grad_ptrs[w] (owned_numel bf16, pinned host memory for an
+ * asynchronous copy) into dev_grad_ptrs[w], runs zr_step, then copies this
+ * rank's positions of param_out into host_param_out (a host buffer in the
+ * global layout, padded_numel bf16).  Asynchronous: the host buffers must
+ * stay untouched until the stream is synchronised. */
+zr_status zr_step_host(const zr_plan* plan, const void* const* host_grad_ptrs,
+                       void* const* dev_grad_ptrs, float* master, float* m, float* v,
+                       void* param_out, void* host_param_out, int64_t step, zr_stream_t stream);
+
+/* Clipping building block: writes this rank's S_r = sum over owned elements
+ * of g*g (g the averaged gradient, each square exact in fp64, fp64
+ * accumulation in a fixed order) to the device double *d_out.  zr_step's
+ * own pass computes bit-identical values, so other ranks' entries of the
+ * partials array may come from this call. */
+zr_status zr_grad_sumsq(const zr_plan* plan, const void* const* grad_ptrs, double* d_out,
+                        zr_stream_t stream);
+
+/* Test hook: write the averaged fp32 gradient g (stage 1 only, before any
+ * clipping) for the owned elements, in owned order, to g_out (owned_numel
+ * floats, 16-byte aligned). */
+zr_status zr_debug_reduce(const zr_plan* plan, const void* const* grad_ptrs, float* g_out,
+                          zr_stream_t stream);
+
+void zr_plan_destroy(zr_plan* plan);
+
+const char* zr_status_string(zr_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZR_H_ */

@@ -1,0 +1,265 @@
+// C ABI of the fused sharded optimizer step (declared in include/zr.h).
+//
+// This layer validates arguments, holds the host-side plan, binds the
+// caller's device workspace and enqueues the kernels; it never allocates
+// device memory and never synchronises.
+#include <cuda_runtime.h>
+
+#include <cstring>
+#include <new>
+
+#include "zr_internal.hpp"
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+zr_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ZR_OK : ZR_ERR_CUDA; }
+
+zr_status check_grads(const zr_plan* p, const void* const* grad_ptrs) {
+    if (!grad_ptrs) return ZR_ERR_INVALID_ARG;
+    for (int32_t w = 0; w < p->world_size; ++w) {
+        if (!grad_ptrs[w]) return ZR_ERR_INVALID_ARG;
+        if (!aligned16(grad_ptrs[w])) return ZR_ERR_ALIGNMENT;
+    }
+    return ZR_OK;
+}
+
+zr::LaunchArgs base_args(const zr_plan* p) {
+    zr::LaunchArgs a{};
+    a.tiles = p->d_tiles;
+    a.n_tiles = static_cast<int32_t>(p->tiles.size());
+    a.world_size = p->world_size;
+    const bool pow2 = (p->world_size & (p->world_size - 1)) == 0;
+    a.w_is_pow2 = pow2 ? 1 : 0;
+    a.inv_w = pow2 ? 1.0f / static_cast<float>(p->world_size) : 0.0f;
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* zr_status_string(zr_status s) {
+    switch (s) {
+        case ZR_OK: return "ZR_OK";
+        case ZR_ERR_INVALID_ARG: return "ZR_ERR_INVALID_ARG: invalid argument";
+        case ZR_ERR_ALIGNMENT: return "ZR_ERR_ALIGNMENT: device pointer not 16-byte aligned";
+        case ZR_ERR_NO_WORKSPACE: return "ZR_ERR_NO_WORKSPACE: workspace (or clip partials) not bound or too small";
+        case ZR_ERR_CUDA: return "ZR_ERR_CUDA: a CUDA runtime call failed";
+        case ZR_ERR_UNSUPPORTED: return "ZR_ERR_UNSUPPORTED: unsupported configuration or device";
+        case ZR_ERR_BUFFER_TOO_SMALL: return "ZR_ERR_BUFFER_TOO_SMALL: output array too small";
+    }
+    return "unknown zr_status";
+}
+
+zr_status zr_plan_create(int32_t n_tensors, const int32_t* ndims, const int64_t* const* shapes,
+                         int32_t world_size, int32_t rank, zr_partition mode,
+                         uint64_t bucket_cap_bytes, const zr_adamw* hp, zr_plan** out) {
+    if (!out) return ZR_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (n_tensors < 0 || (n_tensors > 0 && (!ndims || !shapes)) || !hp) return ZR_ERR_INVALID_ARG;
+    if (world_size < 1 || rank < 0 || rank >= world_size) return ZR_ERR_INVALID_ARG;
+    if (world_size > ZR_MAX_WORLD_SIZE) return ZR_ERR_UNSUPPORTED;
+    if (mode != ZR_PARTITION_FLAT && mode != ZR_PARTITION_WHOLE_TENSOR) return ZR_ERR_INVALID_ARG;
+    zr_plan* p = new (std::nothrow) zr_plan();
+    if (!p) return ZR_ERR_INVALID_ARG;
+    p->world_size = world_size;
+    p->rank = rank;
+    p->mode = mode;
+    p->cap_bytes = bucket_cap_bytes;
+    p->hp = *hp;
+    zr_status st;
+    try {
+        st = zr::build_plan(*p, n_tensors, ndims, shapes);
+    } catch (...) {
+        st = ZR_ERR_INVALID_ARG;
+    }
+    if (st != ZR_OK) {
+        delete p;
+        return st;
+    }
+    // A tile index must fit the grid's x dimension.
+    if (p->tiles.size() > 0x7FFFFFFFull) {
+        delete p;
+        return ZR_ERR_UNSUPPORTED;
+    }
+    *out = p;
+    return ZR_OK;
+}
+
+void zr_plan_destroy(zr_plan* plan) { delete plan; }
+
+zr_status zr_plan_query(const zr_plan* p, int64_t* total_numel, int64_t* padded_numel,
+                        int64_t* owned_numel, int32_t* n_buckets, int64_t* n_segments) {
+    if (!p) return ZR_ERR_INVALID_ARG;
+    if (total_numel) *total_numel = p->total_numel;
+    if (padded_numel) *padded_numel = p->padded_numel;
+    if (owned_numel) *owned_numel = p->owned_numel();
+    if (n_buckets) *n_buckets = p->n_buckets;
+    if (n_segments) *n_segments = static_cast<int64_t>(p->segments.size());
+    return ZR_OK;
+}
+
+zr_status zr_plan_segments(const zr_plan* p, zr_segment* out, int64_t cap, int64_t* n) {
+    if (!p || !n || cap < 0 || (cap > 0 && !out)) return ZR_ERR_INVALID_ARG;
+    *n = static_cast<int64_t>(p->segments.size());
+    if (*n > cap) return ZR_ERR_BUFFER_TOO_SMALL;
+    if (*n) std::memcpy(out, p->segments.data(), sizeof(zr_segment) * p->segments.size());
+    return ZR_OK;
+}
+
+zr_status zr_plan_workspace_bytes(const zr_plan* p, uint64_t* bytes) {
+    if (!p || !bytes) return ZR_ERR_INVALID_ARG;
+    *bytes = zr::workspace_layout(*p).total;
+    return ZR_OK;
+}
+
+zr_status zr_plan_set_workspace(zr_plan* p, void* d_ws, uint64_t bytes, zr_stream_t stream) {
+    if (!p || !d_ws) return ZR_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(d_ws) & 255u) != 0) return ZR_ERR_ALIGNMENT;
+    const zr::WorkspaceLayout L = zr::workspace_layout(*p);
+    if (bytes < L.total) return ZR_ERR_NO_WORKSPACE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ZR_ERR_CUDA;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+        return ZR_ERR_CUDA;
+    if (major != 10) return ZR_ERR_UNSUPPORTED;
+    char* base = static_cast<char*>(d_ws);
+    p->device = dev;
+    p->d_workspace = d_ws;
+    p->workspace_bytes = bytes;
+    p->d_tiles = reinterpret_cast<zr::Tile*>(base + L.tiles);
+    p->d_tile_partials = p->clip_enabled() ? reinterpret_cast<double*>(base + L.tile_partials) : nullptr;
+    p->d_clip_coef = reinterpret_cast<float*>(base + L.clip_coef);
+    p->d_own_sumsq = reinterpret_cast<double*>(base + L.own_sumsq);
+    p->d_g_scratch = p->clip_uses_scratch() ? reinterpret_cast<float*>(base + L.g_scratch) : nullptr;
+    if (!p->tiles.empty()) {
+        const cudaError_t e = cudaMemcpyAsync(p->d_tiles, p->tiles.data(), sizeof(zr::Tile) * p->tiles.size(),
+                                              cudaMemcpyHostToDevice, reinterpret_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return ZR_ERR_CUDA;
+    }
+    return ZR_OK;
+}
+
+zr_status zr_plan_set_sumsq_partials(zr_plan* p, double* d_partials) {
+    if (!p || !d_partials) return ZR_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(d_partials) & 7u) != 0) return ZR_ERR_ALIGNMENT;
+    p->d_sumsq_partials = d_partials;
+    return ZR_OK;
+}
+
+zr_status zr_step(const zr_plan* p, const void* const* grad_ptrs, float* master, float* m, float* v,
+                  void* param_out, int64_t step, zr_stream_t stream) {
+    if (!p || step < 1) return ZR_ERR_INVALID_ARG;
+    if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
+    if (p->owned_numel() == 0) return ZR_OK;
+    zr_status st = check_grads(p, grad_ptrs);
+    if (st != ZR_OK) return st;
+    if (!master || !m || !v || !param_out) return ZR_ERR_INVALID_ARG;
+    if (!aligned16(master) || !aligned16(m) || !aligned16(v) || !aligned16(param_out)) return ZR_ERR_ALIGNMENT;
+    if (p->clip_enabled() && !p->d_sumsq_partials) return ZR_ERR_NO_WORKSPACE;
+
+    zr::LaunchArgs a = base_args(p);
+    a.master = master;
+    a.m = m;
+    a.v = v;
+    a.param_out = static_cast<uint16_t*>(param_out);
+    a.s = zr::adam_scalars(p->hp, step);
+    void* s = stream;
+    if (!p->clip_enabled())
+        return cuda_status(static_cast<cudaError_t>(zr::launch_tiles(zr::Pass::kStep, a, grad_ptrs, false, false, s)));
+
+    // Pass 1: reduce, per-tile sums of squares (and the fp32 g scratch for W > 4).
+    const bool scratch = p->clip_uses_scratch();
+    a.g_buf = p->d_g_scratch;
+    a.tile_partials = p->d_tile_partials;
+    int e = zr::launch_tiles(zr::Pass::kSumsq, a, grad_ptrs, false, scratch, s);
+    if (e != cudaSuccess) return ZR_ERR_CUDA;
+    // Combine: this rank's S_r, all ranks' S in rank order, the coefficient.
+    e = zr::launch_clip_combine(p->d_tile_partials, a.n_tiles, p->d_sumsq_partials, p->world_size, p->rank,
+                                p->hp.max_grad_norm, p->d_clip_coef, p->d_own_sumsq, s);
+    if (e != cudaSuccess) return ZR_ERR_CUDA;
+    // Pass 2: scale by the coefficient, AdamW, cast.
+    a.clip_coef = p->d_clip_coef;
+    e = zr::launch_tiles(zr::Pass::kStepClip, a, grad_ptrs, scratch, false, s);
+    return cuda_status(static_cast<cudaError_t>(e));
+}
+
+zr_status zr_grad_sumsq(const zr_plan* p, const void* const* grad_ptrs, double* d_out, zr_stream_t stream) {
+    if (!p || !d_out) return ZR_ERR_INVALID_ARG;
+    if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
+    if (!p->clip_enabled()) return ZR_ERR_INVALID_ARG;   // tile partials live in the clip workspace
+    if ((reinterpret_cast<uintptr_t>(d_out) & 7u) != 0) return ZR_ERR_ALIGNMENT;
+    void* s = stream;
+    if (p->owned_numel() == 0) {
+        return cuda_status(cudaMemsetAsync(d_out, 0, sizeof(double), static_cast<cudaStream_t>(s)));
+    }
+    zr_status st = check_grads(p, grad_ptrs);
+    if (st != ZR_OK) return st;
+    zr::LaunchArgs a = base_args(p);
+    a.tile_partials = p->d_tile_partials;
+    int e = zr::launch_tiles(zr::Pass::kSumsq, a, grad_ptrs, false, false, s);
+    if (e != cudaSuccess) return ZR_ERR_CUDA;
+    e = zr::launch_clip_combine(p->d_tile_partials, a.n_tiles, nullptr, p->world_size, p->rank,
+                                p->hp.max_grad_norm, nullptr, d_out, s);
+    return cuda_status(static_cast<cudaError_t>(e));
+}
+
+zr_status zr_debug_reduce(const zr_plan* p, const void* const* grad_ptrs, float* g_out, zr_stream_t stream) {
+    if (!p || !g_out) return ZR_ERR_INVALID_ARG;
+    if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
+    if (p->owned_numel() == 0) return ZR_OK;
+    zr_status st = check_grads(p, grad_ptrs);
+    if (st != ZR_OK) return st;
+    if (!aligned16(g_out)) return ZR_ERR_ALIGNMENT;
+    zr::LaunchArgs a = base_args(p);
+    a.g_buf = g_out;
+    return cuda_status(static_cast<cudaError_t>(
+        zr::launch_tiles(zr::Pass::kReduceOnly, a, grad_ptrs, false, false, stream)));
+}
+
+zr_status zr_step_host(const zr_plan* p, const void* const* host_grad_ptrs, void* const* dev_grad_ptrs,
+                       float* master, float* m, float* v, void* param_out, void* host_param_out,
+                       int64_t step, zr_stream_t stream) {
+    if (!p || !host_grad_ptrs || !dev_grad_ptrs || !host_param_out || step < 1) return ZR_ERR_INVALID_ARG;
+    if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
+    const int64_t n = p->owned_numel();
+    if (n == 0) return ZR_OK;
+    for (int32_t w = 0; w < p->world_size; ++w)
+        if (!host_grad_ptrs[w]) return ZR_ERR_INVALID_ARG;
+    zr_status st = check_grads(p, const_cast<const void* const*>(dev_grad_ptrs));
+    if (st != ZR_OK) return st;
+    if (!param_out || !aligned16(param_out)) return param_out ? ZR_ERR_ALIGNMENT : ZR_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    for (int32_t w = 0; w < p->world_size; ++w) {
+        if (cudaMemcpyAsync(dev_grad_ptrs[w], host_grad_ptrs[w], sizeof(uint16_t) * static_cast<size_t>(n),
+                            cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return ZR_ERR_CUDA;
+    }
+    st = zr_step(p, const_cast<const void* const*>(dev_grad_ptrs), master, m, v, param_out, step, stream);
+    if (st != ZR_OK) return st;
+    // This rank's positions of the parameter buffer: one copy per merged run.
+    const uint16_t* src = static_cast<const uint16_t*>(param_out);
+    uint16_t* dst = static_cast<uint16_t*>(host_param_out);
+    int64_t run_start = -1, run_len = 0;
+    auto flush = [&]() -> bool {
+        if (run_len == 0) return true;
+        return cudaMemcpyAsync(dst + run_start, src + run_start, sizeof(uint16_t) * static_cast<size_t>(run_len),
+                               cudaMemcpyDeviceToHost, s) == cudaSuccess;
+    };
+    for (const zr::Tile& t : p->tiles) {
+        if (run_len > 0 && run_start + run_len == t.global) {
+            run_len += t.len;
+        } else {
+            if (!flush()) return ZR_ERR_CUDA;
+            run_start = t.global;
+            run_len = t.len;
+        }
+    }
+    if (!flush()) return ZR_ERR_CUDA;
+    return ZR_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,121 @@
+// Internal types shared by the planner, the C ABI layer and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <vector>
+
+#include "zr.h"
+
+namespace zr {
+
+// A unit of GPU work: a run of consecutive owned elements that is also
+// consecutive in the global layout and lies inside one bucket.
+struct Tile {
+    int64_t owned;     // first element in owned order
+    int64_t global;    // first element in the global layout
+    int32_t len;       // element count, 1..kTileElems
+    int32_t flags;     // kTileVector | kTileStoreVector
+    int32_t bucket;
+    int32_t reserved;
+};
+static_assert(sizeof(Tile) == 32, "Tile is 32 bytes");
+
+constexpr int32_t kTileVector = 1;       // owned % 8 == 0 and len % 8 == 0
+constexpr int32_t kTileStoreVector = 2;  // global % 8 == 0 as well: 16-byte bf16 stores
+
+constexpr int kThreads = 256;                  // threads per CTA
+constexpr int kElemsPerThreadIter = 8;         // one 16-byte bf16 vector
+constexpr int kTileElems = kThreads * kElemsPerThreadIter * 2;  // 4096
+
+// AdamW scalars for one step, fp64 on the host rounded once to fp32.
+struct AdamScalars {
+    float beta1, beta2, one_minus_beta1, one_minus_beta2;
+    float step_size;   // lr / (1 - beta1^t)
+    float bc2_sqrt;    // sqrt(1 - beta2^t)
+    float decay;       // 1 - lr * weight_decay
+    float eps;
+};
+
+enum class Pass : int {
+    kStep = 0,         // reduce -> AdamW -> cast (no clipping)
+    kReduceOnly = 1,   // reduce -> fp32 g to an output buffer
+    kSumsq = 2,        // reduce -> per-tile fp64 sum of squares (+ optional g scratch)
+    kStepClip = 3,     // (reduce | read g scratch) -> * clip coef -> AdamW -> cast
+};
+
+struct LaunchArgs {
+    const Tile* tiles;
+    int32_t n_tiles;
+    int32_t world_size;
+    int32_t w_is_pow2;
+    float inv_w;               // 1/W when W is a power of two (exact)
+    float* master;
+    float* m;
+    float* v;
+    uint16_t* param_out;
+    float* g_buf;              // kReduceOnly: output; kSumsq/kStepClip: scratch (may be null)
+    double* tile_partials;     // kSumsq: one double per tile
+    const float* clip_coef;    // kStepClip: device scalar
+    AdamScalars s;
+};
+
+// Kernel launchers (zr_kernels.cu).  grad_ptrs: host array of W device
+// pointers.  Return cudaError_t as int.
+int launch_tiles(Pass pass, const LaunchArgs& a, const void* const* grad_ptrs, bool g_from_scratch,
+                 bool write_g_scratch, void* stream);
+int launch_clip_combine(const double* tile_partials, int32_t n_tiles, double* partials_all,
+                        int32_t world_size, int32_t rank, float max_norm, float* clip_coef_out,
+                        double* sumsq_out, void* stream);
+
+}  // namespace zr
+
+// The opaque plan.
+struct zr_plan {
+    int32_t n_tensors = 0;
+    int32_t world_size = 1;
+    int32_t rank = 0;
+    int32_t mode = 0;
+    uint64_t cap_bytes = 0;
+    zr_adamw hp{};
+
+    std::vector<int64_t> numel;          // per tensor
+    std::vector<int64_t> goff;           // per tensor, global layout
+    std::vector<int32_t> tensor_owner;   // whole-tensor mode
+    std::vector<int32_t> tensor_bucket;
+    std::vector<int64_t> rank_numel;     // owned element count per rank
+    int64_t total_numel = 0;
+    int64_t padded_numel = 0;
+    int64_t chunk = 0;
+    int32_t n_buckets = 0;
+
+    std::vector<zr_segment> segments;    // all ranks
+    std::vector<zr::Tile> tiles;         // this rank, bucket by bucket
+    std::vector<int32_t> bucket_first_tile;  // n_buckets + 1 entries
+
+    // device binding
+    int device = -1;
+    void* d_workspace = nullptr;
+    uint64_t workspace_bytes = 0;
+    zr::Tile* d_tiles = nullptr;
+    double* d_tile_partials = nullptr;
+    float* d_clip_coef = nullptr;
+    double* d_own_sumsq = nullptr;
+    float* d_g_scratch = nullptr;
+    double* d_sumsq_partials = nullptr;   // caller-owned, world_size doubles
+
+    bool clip_enabled() const { return hp.max_grad_norm > 0.0f; }
+    bool clip_uses_scratch() const { return clip_enabled() && world_size > 4; }
+    int64_t owned_numel() const { return rank_numel[rank]; }
+};
+
+namespace zr {
+// planner.cpp
+zr_status build_plan(zr_plan& p, int32_t n_tensors, const int32_t* ndims,
+                     const int64_t* const* shapes);
+// Workspace layout: offsets of each region, total bytes.
+struct WorkspaceLayout {
+    uint64_t tiles, tile_partials, clip_coef, own_sumsq, g_scratch, total;
+};
+WorkspaceLayout workspace_layout(const zr_plan& p);
+AdamScalars adam_scalars(const zr_adamw& hp, int64_t step);
+}  // namespace zr

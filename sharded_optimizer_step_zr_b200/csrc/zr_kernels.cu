@@ -1,0 +1,347 @@
+// Fused sharded optimizer step kernels for B200 (sm_100a).
+//
+// The step is a pure stream over the owned slice: per owned element it reads
+// W bf16 gradients (2W bytes), fp32 master, m and v (12 bytes), writes them
+// back (12 bytes) and writes one bf16 parameter (2 bytes).  Nothing here is
+// a contraction, so there is no tensor-core work; the roofline is HBM
+// bandwidth and the design goal is keeping enough bytes in flight:
+//   * one CTA per tile of up to 4096 owned elements (tiles never cross a
+//     bucket; the hardware block scheduler balances them across the 148 SMs);
+//   * each thread owns 8 consecutive elements per iteration and issues the W
+//     16-byte gradient loads of a group (up to 16 replicas) back to back,
+//     plus the 32-byte master / m / v loads, before consuming any of them;
+//   * the fold is a strict left fold in rank order in fp32, exactly the
+//     reduce of the definition; the AdamW arithmetic uses round-to-nearest
+//     intrinsics without contraction, so results equal the definition's
+//     fp32 evaluation order bit for bit.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "zr_internal.hpp"
+
+namespace zr {
+namespace {
+
+template <int CAP>
+struct GradPtrs {
+    const uint16_t* p[CAP];
+};
+
+// ---------------------------------------------------------------------------
+// memory helpers
+// ---------------------------------------------------------------------------
+
+// Read-only streaming 16-byte load (gradients are never written by the step).
+__device__ __forceinline__ uint4 ld_grad16(const uint16_t* p) {
+    uint4 r;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ uint16_t ld_grad2(const uint16_t* p) {
+    unsigned short r;
+    asm("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(r) : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ float4 ld_state16(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ void st_state16(float* p, float4 x) { __stcs(reinterpret_cast<float4*>(p), x); }
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ float bf16_1(uint16_t h) { return __uint_as_float(static_cast<uint32_t>(h) << 16); }
+
+__device__ __forceinline__ void unpack8(const uint4 q, float s[8]) {
+    s[0] = bf16_lo(q.x); s[1] = bf16_hi(q.x);
+    s[2] = bf16_lo(q.y); s[3] = bf16_hi(q.y);
+    s[4] = bf16_lo(q.z); s[5] = bf16_hi(q.z);
+    s[6] = bf16_lo(q.w); s[7] = bf16_hi(q.w);
+}
+
+__device__ __forceinline__ void add8(const uint4 q, float s[8]) {
+    s[0] = __fadd_rn(s[0], bf16_lo(q.x)); s[1] = __fadd_rn(s[1], bf16_hi(q.x));
+    s[2] = __fadd_rn(s[2], bf16_lo(q.y)); s[3] = __fadd_rn(s[3], bf16_hi(q.y));
+    s[4] = __fadd_rn(s[4], bf16_lo(q.z)); s[5] = __fadd_rn(s[5], bf16_hi(q.z));
+    s[6] = __fadd_rn(s[6], bf16_lo(q.w)); s[7] = __fadd_rn(s[7], bf16_hi(q.w));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);   // RNE on both halves
+    uint32_t u;
+    memcpy(&u, &h, 4);
+    return u;
+}
+
+// ---------------------------------------------------------------------------
+// element arithmetic
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float average(float s, const LaunchArgs& a) {
+    // Division by a power of two is exact scaling: multiplying by 1/W gives
+    // the same correctly rounded value as the division.
+    return a.w_is_pow2 ? __fmul_rn(s, a.inv_w) : __fdiv_rn(s, static_cast<float>(a.world_size));
+}
+
+// Decoupled weight decay on the pre-update weight, then the bias-corrected
+// Adam step; one rounding per operation, no fused multiply-add.
+__device__ __forceinline__ void adamw(const AdamScalars& c, float g, float& p, float& m, float& v) {
+    const float m_new = __fadd_rn(__fmul_rn(c.beta1, m), __fmul_rn(c.one_minus_beta1, g));
+    const float v_new = __fadd_rn(__fmul_rn(c.beta2, v), __fmul_rn(c.one_minus_beta2, __fmul_rn(g, g)));
+    const float p_dec = __fmul_rn(p, c.decay);
+    const float denom = __fadd_rn(__fdiv_rn(__fsqrt_rn(v_new), c.bc2_sqrt), c.eps);
+    const float update = __fdiv_rn(__fmul_rn(c.step_size, m_new), denom);
+    p = __fsub_rn(p_dec, update);
+    m = m_new;
+    v = v_new;
+}
+
+// Left fold of W replicas for 8 consecutive owned elements at `off`.  The
+// loads of one group of G replicas are all issued before the first add.
+template <int CAP, int G>
+__device__ __forceinline__ void fold8(const GradPtrs<CAP>& gp, int W, int64_t off, float s[8]) {
+    uint4 q[G];
+#pragma unroll
+    for (int j = 0; j < G; ++j)
+        if (j < W) q[j] = ld_grad16(gp.p[j] + off);
+    unpack8(q[0], s);
+#pragma unroll
+    for (int j = 1; j < G; ++j)
+        if (j < W) add8(q[j], s);
+    if constexpr (CAP > G) {
+        for (int w0 = G; w0 < W; w0 += G) {
+#pragma unroll
+            for (int j = 0; j < G; ++j)
+                if (w0 + j < W) q[j] = ld_grad16(gp.p[w0 + j] + off);
+#pragma unroll
+            for (int j = 0; j < G; ++j)
+                if (w0 + j < W) add8(q[j], s);
+        }
+    }
+}
+
+template <int CAP>
+__device__ __forceinline__ float fold1(const GradPtrs<CAP>& gp, int W, int64_t off) {
+    float s = bf16_1(ld_grad2(gp.p[0] + off));
+    if constexpr (CAP <= 16) {
+#pragma unroll
+        for (int w = 1; w < CAP; ++w)
+            if (w < W) s = __fadd_rn(s, bf16_1(ld_grad2(gp.p[w] + off)));
+    } else {
+        for (int w = 1; w < W; ++w) s = __fadd_rn(s, bf16_1(ld_grad2(gp.p[w] + off)));
+    }
+    return s;
+}
+
+// Deterministic block sum of one double per thread (fixed shuffle tree, then
+// warp partials in order).
+__device__ double block_sum(double x) {
+    __shared__ double warp_part[kThreads / 32];
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1) x += __shfl_down_sync(0xFFFFFFFFu, x, d);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) warp_part[warp] = x;
+    __syncthreads();
+    double total = 0.0;
+    if (threadIdx.x == 0) {
+        for (int w = 0; w < kThreads / 32; ++w) total += warp_part[w];
+    }
+    return total;   // valid in thread 0
+}
+
+// ---------------------------------------------------------------------------
+// the tile kernel
+// ---------------------------------------------------------------------------
+
+template <int CAP, int G, Pass PASS, bool G_FROM_SCRATCH, bool WRITE_G>
+__global__ void __launch_bounds__(kThreads)
+zr_tile_kernel(const GradPtrs<CAP> gp, const LaunchArgs a) {
+    const Tile tile = a.tiles[blockIdx.x];
+    const int W = a.world_size;
+    float coef = 1.0f;
+    if constexpr (PASS == Pass::kStepClip) coef = *a.clip_coef;
+    double sq = 0.0;
+
+    if (tile.flags & kTileVector) {
+        for (int e = threadIdx.x * 8; e < tile.len; e += kThreads * 8) {
+            const int64_t o = tile.owned + e;
+            float g[8];
+            float4 p0, p1, m0, m1, v0, v1;
+            constexpr bool kUpdate = PASS == Pass::kStep || PASS == Pass::kStepClip;
+            // Small W: state loads go out with the gradient loads.  Large W:
+            // the fold alone keeps enough bytes in flight, and deferring the
+            // state loads frees 24 registers across it.
+            constexpr bool kEarlyState = kUpdate && (CAP <= 16 || G_FROM_SCRATCH);
+            if constexpr (kEarlyState) {
+                p0 = ld_state16(a.master + o); p1 = ld_state16(a.master + o + 4);
+                m0 = ld_state16(a.m + o);      m1 = ld_state16(a.m + o + 4);
+                v0 = ld_state16(a.v + o);      v1 = ld_state16(a.v + o + 4);
+            }
+            if constexpr (G_FROM_SCRATCH) {
+                const float4 g0 = ld_state16(a.g_buf + o), g1 = ld_state16(a.g_buf + o + 4);
+                g[0] = g0.x; g[1] = g0.y; g[2] = g0.z; g[3] = g0.w;
+                g[4] = g1.x; g[5] = g1.y; g[6] = g1.z; g[7] = g1.w;
+            } else {
+                fold8<CAP, G>(gp, W, o, g);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) g[k] = average(g[k], a);
+            }
+            if constexpr (PASS == Pass::kReduceOnly || WRITE_G) {
+                st_state16(a.g_buf + o, make_float4(g[0], g[1], g[2], g[3]));
+                st_state16(a.g_buf + o + 4, make_float4(g[4], g[5], g[6], g[7]));
+            }
+            if constexpr (PASS == Pass::kSumsq) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) sq += static_cast<double>(g[k]) * static_cast<double>(g[k]);
+            }
+            if constexpr (kUpdate) {
+                if constexpr (!kEarlyState) {
+                    p0 = ld_state16(a.master + o); p1 = ld_state16(a.master + o + 4);
+                    m0 = ld_state16(a.m + o);      m1 = ld_state16(a.m + o + 4);
+                    v0 = ld_state16(a.v + o);      v1 = ld_state16(a.v + o + 4);
+                }
+                if constexpr (PASS == Pass::kStepClip) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) g[k] = __fmul_rn(g[k], coef);
+                }
+                float p[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+                float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+                float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+                for (int k = 0; k < 8; ++k) adamw(a.s, g[k], p[k], mm[k], vv[k]);
+                st_state16(a.master + o, make_float4(p[0], p[1], p[2], p[3]));
+                st_state16(a.master + o + 4, make_float4(p[4], p[5], p[6], p[7]));
+                st_state16(a.m + o, make_float4(mm[0], mm[1], mm[2], mm[3]));
+                st_state16(a.m + o + 4, make_float4(mm[4], mm[5], mm[6], mm[7]));
+                st_state16(a.v + o, make_float4(vv[0], vv[1], vv[2], vv[3]));
+                st_state16(a.v + o + 4, make_float4(vv[4], vv[5], vv[6], vv[7]));
+                const int64_t go = tile.global + e;
+                if (tile.flags & kTileStoreVector) {
+                    uint4 q;
+                    q.x = pack_bf16x2(p[0], p[1]);
+                    q.y = pack_bf16x2(p[2], p[3]);
+                    q.z = pack_bf16x2(p[4], p[5]);
+                    q.w = pack_bf16x2(p[6], p[7]);
+                    __stcs(reinterpret_cast<uint4*>(a.param_out + go), q);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        __nv_bfloat16 h = __float2bfloat16_rn(p[k]);
+                        uint16_t u;
+                        memcpy(&u, &h, 2);
+                        a.param_out[go + k] = u;
+                    }
+                }
+            }
+        }
+    } else {
+        // Ragged tile: one element per thread.
+        for (int e = threadIdx.x; e < tile.len; e += kThreads) {
+            const int64_t o = tile.owned + e;
+            float g;
+            if constexpr (G_FROM_SCRATCH) g = a.g_buf[o];
+            else g = average(fold1<CAP>(gp, W, o), a);
+            if constexpr (PASS == Pass::kReduceOnly || WRITE_G) a.g_buf[o] = g;
+            if constexpr (PASS == Pass::kSumsq) sq += static_cast<double>(g) * static_cast<double>(g);
+            if constexpr (PASS == Pass::kStep || PASS == Pass::kStepClip) {
+                if constexpr (PASS == Pass::kStepClip) g = __fmul_rn(g, coef);
+                float p = a.master[o], mm = a.m[o], vv = a.v[o];
+                adamw(a.s, g, p, mm, vv);
+                a.master[o] = p;
+                a.m[o] = mm;
+                a.v[o] = vv;
+                __nv_bfloat16 h = __float2bfloat16_rn(p);
+                uint16_t u;
+                memcpy(&u, &h, 2);
+                a.param_out[tile.global + e] = u;
+            }
+        }
+    }
+    if constexpr (PASS == Pass::kSumsq) {
+        const double total = block_sum(sq);
+        if (threadIdx.x == 0) a.tile_partials[blockIdx.x] = total;
+    }
+}
+
+// One block: S_r = sum of the per-tile partials in a fixed order, stored as
+// this rank's entry of the partials array (or to sumsq_out alone); then the
+// clip coefficient from all ranks' entries, summed in rank order.
+__global__ void __launch_bounds__(1024)
+zr_clip_combine_kernel(const double* __restrict__ tile_partials, int32_t n_tiles,
+                       double* partials_all, int32_t world_size, int32_t rank, float max_norm,
+                       float* clip_coef_out, double* sumsq_out) {
+    __shared__ double part[1024];
+    double x = 0.0;
+    for (int32_t i = threadIdx.x; i < n_tiles; i += blockDim.x) x += tile_partials[i];
+    part[threadIdx.x] = x;
+    __syncthreads();
+    for (int stride = blockDim.x / 2; stride >= 1; stride >>= 1) {
+        if (threadIdx.x < stride) part[threadIdx.x] += part[threadIdx.x + stride];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        const double own = part[0];
+        if (sumsq_out) *sumsq_out = own;
+        if (partials_all) {
+            partials_all[rank] = own;
+            double S = partials_all[0];
+            for (int32_t w = 1; w < world_size; ++w) S += partials_all[w];
+            const double c = static_cast<double>(max_norm) / (sqrt(S) + 1e-6);
+            *clip_coef_out = static_cast<float>(c < 1.0 ? c : 1.0);
+        }
+    }
+}
+
+template <int CAP, int G, Pass PASS, bool FROM, bool WRITE>
+cudaError_t launch_one(const LaunchArgs& a, const void* const* grad_ptrs, cudaStream_t stream) {
+    GradPtrs<CAP> gp;
+    for (int w = 0; w < CAP; ++w)
+        gp.p[w] = w < a.world_size ? static_cast<const uint16_t*>(grad_ptrs[w]) : nullptr;
+    zr_tile_kernel<CAP, G, PASS, FROM, WRITE><<<a.n_tiles, kThreads, 0, stream>>>(gp, a);
+    return cudaGetLastError();
+}
+
+template <Pass PASS, bool FROM, bool WRITE>
+cudaError_t dispatch_w(const LaunchArgs& a, const void* const* grad_ptrs, cudaStream_t stream) {
+    const int W = a.world_size;
+    if (FROM) return launch_one<1, 1, PASS, FROM, WRITE>(a, grad_ptrs, stream);
+    if (W <= 2) return launch_one<2, 2, PASS, FROM, WRITE>(a, grad_ptrs, stream);
+    if (W <= 4) return launch_one<4, 4, PASS, FROM, WRITE>(a, grad_ptrs, stream);
+    if (W <= 8) return launch_one<8, 8, PASS, FROM, WRITE>(a, grad_ptrs, stream);
+    if (W <= 16) return launch_one<16, 16, PASS, FROM, WRITE>(a, grad_ptrs, stream);
+    if (W <= 64) return launch_one<64, 8, PASS, FROM, WRITE>(a, grad_ptrs, stream);
+    return launch_one<ZR_MAX_WORLD_SIZE, 8, PASS, FROM, WRITE>(a, grad_ptrs, stream);
+}
+
+}  // namespace
+
+int launch_tiles(Pass pass, const LaunchArgs& a, const void* const* grad_ptrs, bool g_from_scratch,
+                 bool write_g_scratch, void* stream_v) {
+    if (a.n_tiles == 0) return cudaSuccess;
+    cudaStream_t s = static_cast<cudaStream_t>(stream_v);
+    switch (pass) {
+        case Pass::kStep: return dispatch_w<Pass::kStep, false, false>(a, grad_ptrs, s);
+        case Pass::kReduceOnly: return dispatch_w<Pass::kReduceOnly, false, false>(a, grad_ptrs, s);
+        case Pass::kSumsq:
+            return write_g_scratch ? dispatch_w<Pass::kSumsq, false, true>(a, grad_ptrs, s)
+                                   : dispatch_w<Pass::kSumsq, false, false>(a, grad_ptrs, s);
+        case Pass::kStepClip:
+            return g_from_scratch ? dispatch_w<Pass::kStepClip, true, false>(a, grad_ptrs, s)
+                                  : dispatch_w<Pass::kStepClip, false, false>(a, grad_ptrs, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+int launch_clip_combine(const double* tile_partials, int32_t n_tiles, double* partials_all,
+                        int32_t world_size, int32_t rank, float max_norm, float* clip_coef_out,
+                        double* sumsq_out, void* stream_v) {
+    zr_clip_combine_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream_v)>>>(
+        tile_partials, n_tiles, partials_all, world_size, rank, max_norm, clip_coef_out, sumsq_out);
+    return cudaGetLastError();
+}
+
+}  // namespace zr

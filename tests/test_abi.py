@@ -1,0 +1,180 @@
+"""C ABI of libzr.so without a GPU: the library loads, exports every function
+include/zr.h declares, rejects bad arguments with the documented status
+codes, and its planner's tables equal the oracle's bit for bit.
+
+The planner runs on the host only, so table parity (the "bucket/owner tables
+bit-exact" requirement) is checked here; kernels are checked in test_gpu_*.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+import sharded_optimizer_step_zr_b200 as zr
+from conftest import ROOT
+from golden_plans import all_golden_plans
+
+FIELDS = ("bucket", "tensor", "owner", "offset_in_tensor", "length", "global_offset", "owned_offset")
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "zr.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(zr_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_function():
+    declared = header_functions()
+    assert set(declared) == set(zr.EXPORTED)
+    lib = zr.lib_handle()
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_only_zr_symbols_exported():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", zr.LIB_PATH], capture_output=True, text=True).stdout
+    syms = [l.split()[-1] for l in out.splitlines() if " T " in l]
+    assert syms and all(s.startswith("zr_") for s in syms), syms
+
+
+def test_status_strings():
+    for s in range(7):
+        assert zr.zr_status_string(s).startswith("ZR_")
+    assert "unknown" in zr.zr_status_string(99)
+
+
+def lib_plan_table(shapes, W, rank, mode, cap):
+    h = zr.zr_plan_create(shapes, W, rank, mode, cap)
+    try:
+        segs = zr.zr_plan_segments(h)
+        info = zr.zr_plan_query(h)
+    finally:
+        zr.zr_plan_destroy(h)
+    return [tuple(s[f] for f in FIELDS) for s in segs], info
+
+
+def oracle_table(shapes, W, mode, cap):
+    p = oracle.Plan(shapes, W, mode, cap)
+    return [tuple(int(s[f]) for f in FIELDS) for s in p.segments], p
+
+
+def assert_tables_equal(shapes, W, mode, cap):
+    want, p = oracle_table(shapes, W, mode, cap)
+    for rank in sorted({0, W - 1, W // 2}):
+        got, info = lib_plan_table(shapes, W, rank, mode, cap)
+        assert got == want
+        assert info["total_numel"] == p.total_numel
+        assert info["padded_numel"] == p.padded_numel
+        assert info["owned_numel"] == int(p.owned_numel[rank])
+        assert info["n_buckets"] == p.n_buckets
+        assert info["n_segments"] == len(want)
+
+
+@pytest.mark.parametrize("g", all_golden_plans(), ids=lambda g: g["name"])
+def test_tables_match_hand_derived(g):
+    got, info = lib_plan_table(g["shapes"], g["world_size"], 0, g["mode"], g["cap_bytes"])
+    assert got == g["segments"]
+    assert (info["total_numel"], info["padded_numel"], info["n_buckets"]) == (g["N"], g["padded"], g["n_buckets"])
+
+
+@pytest.mark.parametrize("name", list(synth.WORKLOADS))
+def test_tables_match_oracle_workloads(name):
+    wl = synth.WORKLOADS[name]
+    assert_tables_equal(wl.shapes, wl.world_size, wl.mode, wl.bucket_cap_bytes)
+
+
+def test_tables_match_oracle_sweep():
+    for wl in synth.sweep_workloads():
+        assert_tables_equal(wl.shapes, wl.world_size, wl.mode, wl.bucket_cap_bytes)
+
+
+def test_tables_match_oracle_random():
+    rng = np.random.default_rng(21)
+    for _ in range(400):
+        shapes = [tuple(int(x) for x in rng.integers(0, 30, size=int(rng.integers(0, 3))))
+                  for _ in range(int(rng.integers(0, 10)))]
+        W = int(rng.integers(1, 12))
+        mode = int(rng.integers(0, 2))
+        cap = int(rng.integers(0, 300))
+        assert_tables_equal(shapes, W, mode, cap)
+
+
+def test_empty_parameter_set():
+    h = zr.zr_plan_create([], 4, 1, 0, 1 << 20)
+    info = zr.zr_plan_query(h)
+    zr.zr_plan_destroy(h)
+    assert info == {"total_numel": 0, "padded_numel": 0, "owned_numel": 0, "n_buckets": 0, "n_segments": 0}
+
+
+@pytest.mark.parametrize("args, status", [
+    (([(4,)], 0, 0, 0, 16), zr.ZR_ERR_INVALID_ARG),          # W = 0
+    (([(4,)], 2, 2, 0, 16), zr.ZR_ERR_INVALID_ARG),          # rank = W
+    (([(4,)], 2, -1, 0, 16), zr.ZR_ERR_INVALID_ARG),         # negative rank
+    (([(4,)], 2, 0, 3, 16), zr.ZR_ERR_INVALID_ARG),          # unknown mode
+    (([(-4,)], 2, 0, 0, 16), zr.ZR_ERR_INVALID_ARG),         # negative extent
+    (([(1 << 40, 1 << 40)], 2, 0, 0, 16), zr.ZR_ERR_INVALID_ARG),  # numel overflow
+    (([(4,)], 513, 0, 0, 16), zr.ZR_ERR_UNSUPPORTED),        # W above the limit
+])
+def test_plan_create_rejects(args, status):
+    with pytest.raises(zr.ZrError) as e:
+        zr.zr_plan_create(*args)
+    assert e.value.status == status
+
+
+def test_null_arguments():
+    assert zr.raw_call("zr_plan_create", 0, None, None, 1, 0, 0, 0, None, None) == zr.ZR_ERR_INVALID_ARG
+    n = ctypes.c_int64()
+    assert zr.raw_call("zr_plan_query", None, None, None, None, None, None) == zr.ZR_ERR_INVALID_ARG
+    assert zr.raw_call("zr_plan_segments", None, None, 0, ctypes.byref(n)) == zr.ZR_ERR_INVALID_ARG
+    assert zr.raw_call("zr_plan_workspace_bytes", None, None) == zr.ZR_ERR_INVALID_ARG
+
+
+def test_step_checks_before_touching_the_device():
+    """Without a bound workspace or with a bad step the call returns an
+    error and launches nothing (no GPU needed to check this)."""
+    h = zr.zr_plan_create([(64,)], 2, 0, 0, 1 << 20)
+    try:
+        grads = (ctypes.c_void_p * 2)(16, 32)
+        assert zr.raw_call("zr_step", h, grads, 16, 16, 16, 16, 0, None) == zr.ZR_ERR_INVALID_ARG
+        assert zr.raw_call("zr_step", h, grads, 16, 16, 16, 16, 1, None) == zr.ZR_ERR_NO_WORKSPACE
+        assert zr.raw_call("zr_debug_reduce", h, grads, 16, None) == zr.ZR_ERR_NO_WORKSPACE
+        assert zr.raw_call("zr_grad_sumsq", h, grads, 16, None) == zr.ZR_ERR_NO_WORKSPACE
+        assert zr.raw_call("zr_plan_set_workspace", h, None, 0, None) == zr.ZR_ERR_INVALID_ARG
+        assert zr.raw_call("zr_plan_set_workspace", h, 8, 1 << 20, None) == zr.ZR_ERR_ALIGNMENT
+        assert zr.raw_call("zr_plan_set_sumsq_partials", h, 12) == zr.ZR_ERR_ALIGNMENT
+        # workspace too small is detected before any CUDA call
+        need = zr.zr_plan_workspace_bytes(h)
+        assert zr.raw_call("zr_plan_set_workspace", h, 256, need - 1, None) == zr.ZR_ERR_NO_WORKSPACE
+    finally:
+        zr.zr_plan_destroy(h)
+
+
+def test_segments_buffer_too_small():
+    h = zr.zr_plan_create(synth.tiny_shapes(), 2, 0, 0, 1 << 20)
+    try:
+        n = ctypes.c_int64()
+        arr = (zr.zr_segment * 2)()
+        assert zr.raw_call("zr_plan_segments", h, arr, 2, ctypes.byref(n)) == zr.ZR_ERR_BUFFER_TOO_SMALL
+        assert n.value == 5
+    finally:
+        zr.zr_plan_destroy(h)
+
+
+def test_workspace_grows_with_clip_scratch():
+    shapes = [(1024, 1024)]
+    plain = zr.zr_plan_create(shapes, 8, 0, 0, 1 << 20)
+    clip8 = zr.zr_plan_create(shapes, 8, 0, 0, 1 << 20, max_grad_norm=1.0)
+    clip4 = zr.zr_plan_create(shapes, 4, 0, 0, 1 << 20, max_grad_norm=1.0)
+    try:
+        b_plain, b8, b4 = (zr.zr_plan_workspace_bytes(h) for h in (plain, clip8, clip4))
+        owned8 = (1024 * 1024) // 8
+        assert b8 - b_plain >= 4 * owned8          # fp32 g scratch for W > 4
+        assert b4 - b_plain < 4 * (1024 * 1024) // 4  # W <= 4 re-reads the gradients instead
+    finally:
+        for h in (plain, clip8, clip4):
+            zr.zr_plan_destroy(h)

@@ -1,0 +1,217 @@
+"""GPU parity: libzr.so's kernels against the oracle on the same seeded inputs.
+
+Bars (element by element):
+  * averaged fp32 gradient (zr_debug_reduce): bit-exact (fixed rank-order
+    fold);
+  * master / m / v after the steps: |x - y| <= 1e-9 + 2e-6 |y|;
+  * bf16 parameters: within 1 ulp;
+  * and, since the kernels evaluate the definition's fp32 operations in the
+    same order with round-to-nearest intrinsics, bit-exactness is checked too.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_harness import (DEV, GpuRank, OracleRank, assert_state_close, bf16_ulp_distance, bits32, u16)
+
+pytestmark = pytest.mark.gpu
+
+HP = (3e-4, 0.9, 0.999, 1e-8, 0.1, 0.0)
+
+
+def run_all_ranks(shapes, W, mode, cap, steps, sigma, outlier, seed=2024, hp=HP, ranks=None,
+                  exact=True):
+    """Step every rank (or `ranks`) on the GPU and in the oracle, writing into
+    one parameter buffer each (the emulated all-gather), and compare."""
+    oplan = oracle.Plan(shapes, W, mode, cap)
+    ranks = list(range(W)) if ranks is None else ranks
+    gpu = {r: GpuRank(shapes, W, r, mode, cap, hp, seed) for r in ranks}
+    orc = {r: OracleRank(oplan, r, seed) for r in ranks}
+    P = max(oplan.padded_numel, 8)
+    out_gpu = torch.full((P,), -1, dtype=torch.int16, device=DEV).view(torch.bfloat16)
+    out_orc = np.full(P, 0xFFFF, dtype=np.uint16)
+    for t in range(1, steps + 1):
+        for r in ranks:
+            gpu[r].fill_grads(t, sigma, outlier)
+            orc[r].make_grads(t, sigma, outlier)
+            # inputs agree bit for bit
+            n = oplan.owned_numel[r]
+            for w in range(W):
+                assert np.array_equal(u16(gpu[r].grads[w][:n]), orc[r].grads[w])
+            g = gpu[r].reduce()
+            torch.cuda.synchronize()
+            assert np.array_equal(bits32(g), bits32(oracle.reduce(orc[r].grads))), f"reduce rank {r} step {t}"
+            gpu[r].step(out_gpu, t)
+            orc[r].step(out_orc, hp, t)
+        torch.cuda.synchronize()
+        for r in ranks:
+            gm, gmm, gv = gpu[r].state()
+            assert_state_close(gm, orc[r].master, f"master rank {r} step {t}")
+            assert_state_close(gmm, orc[r].m, f"m rank {r} step {t}")
+            assert_state_close(gv, orc[r].v, f"v rank {r} step {t}")
+            if exact:
+                assert np.array_equal(bits32(gm), bits32(orc[r].master))
+                assert np.array_equal(bits32(gmm), bits32(orc[r].m))
+                assert np.array_equal(bits32(gv), bits32(orc[r].v))
+        got = u16(out_gpu)
+        assert bf16_ulp_distance(got, out_orc).max() <= 1
+        if exact:
+            assert np.array_equal(got, out_orc)
+    return gpu, orc, oplan
+
+
+def test_generator_identical_on_cpu_and_gpu():
+    idx = torch.arange(0, 1 << 20, dtype=torch.int64)
+    for sigma, out in ((1e-2, 0.0), (1e-3, 0.01)):
+        a = synth.grad_bf16(5, 2, 3, idx, sigma, out)
+        b = synth.grad_bf16(5, 2, 3, idx.to(DEV), sigma, out).cpu()
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    a = synth.master_f32(5, idx)
+    b = synth.master_f32(5, idx.to(DEV)).cpu()
+    assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+
+
+def test_tiny_both_ranks_three_steps():
+    """The tiny workload: 4 tensors, W = 2, both ranks, flat, 1 MB buckets,
+    N(0, 1e-2) gradients, 3 steps; both ranks fill one parameter buffer."""
+    wl = synth.WORKLOADS["tiny"]
+    _, _, oplan = run_all_ranks(wl.shapes, 2, 0, wl.bucket_cap_bytes, 3, 1e-2, 0.0, seed=wl.seed,
+                                hp=wl.hp)
+    assert oplan.total_numel == 1_441_792
+
+
+@pytest.mark.parametrize("shapes, W, mode, cap", [
+    ([(3, 5), (7,), (2, 2, 2)], 4, 0, 16),                 # pad > 0, tiny segments
+    ([(4096 * 3 + 5,), (17,), (1,)], 1, 0, 1 << 20),       # W = 1, ragged tail, length 1
+    ([(1000, 3), (8191,), (9, 9)], 3, 0, 4096),            # W = 3 (non power of two), pad 2
+    ([(12345,), (8,), (777,), (64, 65)], 5, 0, 20000),     # W = 5
+    ([(10,), (4, 5), (7,), (3, 3), (20,)], 3, 1, 40),      # whole-tensor, odd sizes
+    ([(4097,), (33, 31), (5000,), (3,), (8, 8, 8)], 2, 1, 9000),  # whole-tensor, misaligned stores
+    ([(16384,), (2048,), (4099,)], 8, 0, 1 << 20),         # W = 8, multi-tile
+    ([(7, 1024), (100,)], 16, 0, 1 << 20),                 # W = 16
+    ([(5000,), (300,)], 33, 0, 1 << 20),                   # W = 33: a partial second load group
+    ([(4096,), (512,)], 64, 1, 1 << 20),                   # W = 64, whole-tensor, empty ranks
+])
+def test_edge_shapes(shapes, W, mode, cap):
+    run_all_ranks(shapes, W, mode, cap, 2, 1e-3, 0.01)
+
+
+def test_special_values():
+    """±0, subnormals, huge values, inf and NaN in the replicas."""
+    shapes = [(4096 + 24,)]
+    W = 4
+    rng = np.random.default_rng(0)
+    n = 4096 + 24
+    vals = (rng.standard_normal((W, n)) * 1e-3).astype(np.float32)
+    vals[:, 0] = -0.0                           # all -0: the fold keeps the sign
+    vals[0, 1], vals[1:, 1] = 0.0, -0.0
+    vals[:, 2] = 1e-39                           # bf16 subnormals
+    vals[:, 3] = np.float32(-3e38)               # fp32 overflow to -inf in the fold
+    vals[0, 4] = np.inf
+    vals[1, 5] = np.nan
+    vals[:, 6] = np.float32(1e30) * np.array([1, -1, 1, -1])   # exact cancellation
+    vals[:, 7] = np.float32(2.0 ** -130)
+    vals[:, 8:16] = np.float32(1e-3) * np.arange(8)
+    grads = [oracle.f32_to_bf16_array(vals[w]) for w in range(W)]
+    oplan = oracle.Plan(shapes, W, 0, 1 << 20)
+    P = oplan.padded_numel
+    out_gpu = torch.zeros(P, dtype=torch.bfloat16, device=DEV)
+    out_orc = np.zeros(P, dtype=np.uint16)
+    for r in range(W):
+        gr = GpuRank(shapes, W, r, 0, 1 << 20, HP, seed=1)
+        orr = OracleRank(oplan, r, seed=1)
+        idx = oplan.owned_global_index(r)
+        sl = [g[idx] for g in grads]
+        gr.set_grads(sl)
+        orr.grads = sl
+        g = gr.reduce()
+        torch.cuda.synchronize()
+        ref = oracle.reduce(sl)
+        same = (bits32(g) == bits32(ref)) | (np.isnan(g.cpu().numpy()) & np.isnan(ref))
+        assert same.all()
+        gr.step(out_gpu, 1)
+        orr.step(out_orc, HP, 1)
+        torch.cuda.synchronize()
+        for got, want, what in zip(gr.state(), (orr.master, orr.m, orr.v), ("master", "m", "v")):
+            assert_state_close(got, want, what)
+    assert bf16_ulp_distance(u16(out_gpu), out_orc).max() <= 1
+
+
+@pytest.mark.parametrize("W, mode", [(8, 0), (3, 0), (8, 1), (4, 1)])
+def test_clip_all_ranks(W, mode):
+    """Global-norm clip (max_norm small enough to bite): other ranks' sums of
+    squares come from zr_grad_sumsq, this rank's from zr_step itself."""
+    shapes = [(3000, 7), (5001,), (64, 64), (129,), (17, 5)]
+    hp = (3e-4, 0.9, 0.999, 1e-8, 0.1, 0.05)
+    seed = 99
+    oplan = oracle.Plan(shapes, W, mode, 8192)
+    gpu = [GpuRank(shapes, W, r, mode, 8192, hp, seed) for r in range(W)]
+    orc = [OracleRank(oplan, r, seed) for r in range(W)]
+    partials = torch.zeros(W, dtype=torch.float64, device=DEV)
+    P = oplan.padded_numel
+    out_gpu = torch.zeros(P, dtype=torch.bfloat16, device=DEV)
+    out_orc = np.zeros(P, dtype=np.uint16)
+    for t in (1, 2):
+        for r in range(W):
+            gpu[r].fill_grads(t, 1e-2, 0.01)
+            orc[r].make_grads(t, 1e-2, 0.01)
+        # the oracle's global S in rank order of per-rank partials
+        S_parts = [oracle.sumsq(oracle.reduce(o.grads)) for o in orc]
+        S = 0.0
+        for x in S_parts:
+            S += x
+        c = oracle.clip_coef(S, hp[5])
+        assert c < 1.0
+        for r in range(W):
+            gpu[r].plan.grad_sumsq(gpu[r].grads, partials[r:r + 1])
+        torch.cuda.synchronize()
+        got_parts = partials.cpu().numpy()
+        for r in range(W):
+            assert abs(got_parts[r] - S_parts[r]) <= 1e-12 * S_parts[r]
+        for r in range(W):
+            gpu[r].plan.partials.copy_(partials)
+            before = partials[r].item()
+            gpu[r].step(out_gpu, t)
+            torch.cuda.synchronize()
+            # zr_step's own pass reproduces zr_grad_sumsq's value bit for bit
+            assert gpu[r].plan.partials[r].item() == before
+            orc[r].step(out_orc, hp, t, clip=c)
+        torch.cuda.synchronize()
+        for r in range(W):
+            for got, want, what in zip(gpu[r].state(), (orc[r].master, orc[r].m, orc[r].v),
+                                       ("master", "m", "v")):
+                assert_state_close(got, want, f"{what} rank {r} step {t}")
+        assert bf16_ulp_distance(u16(out_gpu), out_orc).max() <= 1
+
+
+def test_unwritten_positions_untouched():
+    """A rank writes exactly its own positions of the parameter buffer."""
+    shapes = [(1000,), (333,), (4100,)]
+    for mode in (0, 1):
+        oplan = oracle.Plan(shapes, 3, mode, 2048)
+        for r in range(3):
+            gr = GpuRank(shapes, 3, r, mode, 2048, HP, seed=4)
+            gr.fill_grads(1, 1e-3, 0.0)
+            out = torch.full((oplan.padded_numel,), 0x7FC1, dtype=torch.int16, device=DEV)
+            gr.step(out.view(torch.bfloat16), 1)
+            torch.cuda.synchronize()
+            got = out.cpu().numpy().view(np.uint16)
+            mine = np.zeros(oplan.padded_numel, dtype=bool)
+            mine[oplan.owned_global_index(r)] = True
+            assert np.all(got[~mine] == 0x7FC1)
+            assert not np.any(got[mine] == 0x7FC1)
+
+
+def test_bad_alignment_rejected_on_device():
+    import sharded_optimizer_step_zr_b200 as zr
+    gr = GpuRank([(4096,)], 2, 0, 0, 1 << 20, HP, seed=1)
+    out = torch.zeros(4096 + 8, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(zr.ZrError) as e:
+        zr.zr_step(gr.plan.handle, [gr.grads[0].data_ptr() + 2, gr.grads[1]], gr.master, gr.m, gr.v,
+                   out, 1)
+    assert e.value.status == zr.ZR_ERR_ALIGNMENT
+    with pytest.raises(zr.ZrError) as e:
+        zr.zr_step(gr.plan.handle, gr.grads, gr.master.data_ptr() + 4, gr.m, gr.v, out, 1)
+    assert e.value.status == zr.ZR_ERR_ALIGNMENT
