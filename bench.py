@@ -73,6 +73,27 @@ def bytes_per_owned_param(W, clip):
     return b
 
 
+def shard_rank(wl, process_rank, n_processes):
+    """ZeRO rank emulated by process `process_rank`: the workload's rank on a
+    single process; consecutive ranks (mod W) across processes."""
+    if n_processes == 1:
+        return wl.ranks[0]
+    return (wl.ranks[0] + process_rank) % wl.world_size
+
+
+def reduce_timing(dist, elapsed_ms, owned_done, device):
+    """Max of the elapsed times and sum of the owned parameters processed over
+    all processes (identity without a process group)."""
+    if dist is None:
+        return elapsed_ms, owned_done
+    import torch
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    o = torch.tensor([owned_done], dtype=torch.float64, device=device)
+    dist.all_reduce(o, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(o.item())
+
+
 def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -253,7 +274,7 @@ def run_zr(args):
 
     wl = workload(args.config)
     W = wl.world_size
-    zr_rank = wl.ranks[0] if world == 1 else (wl.ranks[0] + grank) % W
+    zr_rank = shard_rank(wl, grank, world)
     clip = wl.max_grad_norm > 0
     plan = ZrPlan(wl.shapes, W, zr_rank, wl.mode, wl.bucket_cap_bytes, *wl.hp, device=dev)
     n = plan.owned_numel
@@ -305,14 +326,7 @@ def run_zr(args):
         dist.barrier()
     total_ms = t_start.elapsed_time(t_end)
     per_launch_ms = [a.elapsed_time(b) for a, b in ev]
-    owned_total = n * K
-    if dist:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-        o = torch.tensor([owned_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(o, op=dist.ReduceOp.SUM)
-        owned_total = float(o.item())
+    total_ms, owned_total = reduce_timing(dist, total_ms, n * K, dev)
     value = owned_total / (total_ms * 1e-3) / 1e9
     ms_per_step = total_ms / K
 
@@ -344,15 +358,7 @@ def run_zr(args):
             plan.step_host(host_grads, grads, master, m, v, param_out, host_out, step_no, stream)
         b.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = a.elapsed_time(b)
-        e2e_owned = n * K2
-        if dist:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-            o = torch.tensor([e2e_owned], dtype=torch.float64, device=dev)
-            dist.all_reduce(o, op=dist.ReduceOp.SUM)
-            e2e_owned = float(o.item())
+        e2e_ms, e2e_owned = reduce_timing(dist, a.elapsed_time(b), n * K2, dev)
         e2e = {"value": e2e_owned / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
                "h2d_bytes_per_step": 2 * W * n, "d2h_bytes_per_step": 2 * n,
                "steps": K2, "api": "zr_step_host"}
