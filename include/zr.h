@@ -193,6 +193,46 @@ zr_status zr_grad_sumsq(const zr_plan* plan, const void* const* grad_ptrs, doubl
 zr_status zr_debug_reduce(const zr_plan* plan, const void* const* grad_ptrs, float* g_out,
                           zr_stream_t stream);
 
+/* Size of the library-owned scratch array used by zr_step_no_alloc. */
+#define ZR_NO_ALLOC_SCRATCH_BYTES (4u << 20)
+
+/* zr_step for callers that cannot allocate device memory.  The pages have no
+ * counterpart to this call; it exists for callers such as a plug-in inside a
+ * host framework whose allocator owns all of the GPU's memory (a caching
+ * allocator that has reserved it, or a framework that forbids outside
+ * cudaMalloc), or a latency-critical loop that must not call cudaMalloc
+ * because it can synchronise the device.  Such callers have their inputs
+ * and outputs but cannot give the plan a workspace.
+ *
+ * Same arguments and results as zr_step, plus d_sumsq_partials (clipping
+ * only; otherwise may be NULL): the device array of world_size doubles that
+ * zr_plan_set_sumsq_partials would bind -- other ranks' S_w in, this rank's
+ * entry written.  No workspace needs to be bound; the call makes no
+ * cudaMalloc or cudaFree and calls no allocating routine.
+ *
+ * Scratch (the tile table and, with clipping, one double per tile) lives in a
+ * file-scope device array of ZR_NO_ALLOC_SCRATCH_BYTES (4 MiB) that every GPU
+ * that loads the library holds until the process exits.  The plan needs
+ * 32 bytes per tile, plus 8 more per tile with clipping, plus about 1 KB:
+ * up to about 131,000 tiles (about 104,800 with clipping).  A tile covers up
+ * to 4096 owned elements, so a shard of up to about 536 M owned elements
+ * fits (about 429 M with clipping).  A larger plan gets ZR_ERR_UNSUPPORTED before
+ * anything is launched: use zr_step with a workspace instead.  With clipping,
+ * the second pass reads the gradients again instead of keeping an fp32 copy
+ * of the averaged gradient, so results are bit-identical to zr_step's.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it: make that first call before any
+ * stream capture.  Every call, on every plan, uses the same array and leaves
+ * its contents behind; nothing in it needs to start at zero (each call writes
+ * what it reads).  Calls whose work overlaps on the GPU (different streams
+ * without ordering between them) race on the array and give wrong results.
+ * Errors: as zr_step, plus ZR_ERR_UNSUPPORTED (plan too large for the array,
+ * or the current device is not compute capability 10.x). */
+zr_status zr_step_no_alloc(const zr_plan* plan, const void* const* grad_ptrs, float* master, float* m,
+                           float* v, void* param_out, double* d_sumsq_partials, int64_t step,
+                           zr_stream_t stream);
+
 void zr_plan_destroy(zr_plan* plan);
 
 const char* zr_status_string(zr_status status);

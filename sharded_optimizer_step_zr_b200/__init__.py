@@ -39,8 +39,9 @@ ZR_MAX_WORLD_SIZE = 512
 EXPORTED = [
     "zr_plan_create", "zr_plan_query", "zr_plan_segments", "zr_plan_workspace_bytes",
     "zr_plan_set_workspace", "zr_plan_set_sumsq_partials", "zr_step", "zr_step_host",
-    "zr_grad_sumsq", "zr_debug_reduce", "zr_plan_destroy", "zr_status_string",
+    "zr_grad_sumsq", "zr_debug_reduce", "zr_step_no_alloc", "zr_plan_destroy", "zr_status_string",
 ]
+ZR_NO_ALLOC_SCRATCH_BYTES = 4 << 20
 
 
 class zr_adamw(ctypes.Structure):
@@ -67,6 +68,7 @@ _lib.zr_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_step_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_grad_sumsq.argtypes = [_vp, _vp, _vp, _vp]
 _lib.zr_debug_reduce.argtypes = [_vp, _vp, _vp, _vp]
+_lib.zr_step_no_alloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_plan_destroy.argtypes = [_vp]
 _lib.zr_plan_destroy.restype = None
 _lib.zr_status_string.argtypes = [ctypes.c_int]
@@ -192,6 +194,20 @@ def zr_grad_sumsq(plan: int, grads, out, stream=None) -> None:
 def zr_debug_reduce(plan: int, grads, g_out, stream=None) -> None:
     _check(_lib.zr_debug_reduce(plan, _ptr_array(grads), _addr(g_out), _stream(stream)),
            "zr_debug_reduce")
+
+
+def zr_step_no_alloc(plan: int, grads, master, m, v, param_out, sumsq_partials, step: int,
+                     stream=None) -> None:
+    """zr_step without a workspace: for callers that cannot allocate device
+    memory.  Scratch lives in the library's fixed 4 MiB device array (see
+    include/zr.h); plans too large for it raise ZR_ERR_UNSUPPORTED."""
+    st = _lib.zr_step_no_alloc(plan, _ptr_array(grads), _addr(master), _addr(m), _addr(v),
+                               _addr(param_out), _addr(sumsq_partials), int(step), _stream(stream))
+    if st == ZR_ERR_UNSUPPORTED:
+        raise ZrError(st, "zr_step_no_alloc (the plan's tile table, and clip partials, must fit "
+                          f"the library's {ZR_NO_ALLOC_SCRATCH_BYTES} byte static scratch on a "
+                          "compute capability 10.x device; use zr_step with a workspace)")
+    _check(st, "zr_step_no_alloc")
 
 
 def raw_call(name: str, *args) -> int:
