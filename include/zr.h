@@ -215,8 +215,8 @@ zr_status zr_debug_reduce(const zr_plan* plan, const void* const* grad_ptrs, flo
  * that loads the library holds until the process exits.  The plan needs
  * 32 bytes per tile, plus 8 more per tile with clipping, plus about 1 KB:
  * up to about 131,000 tiles (about 104,800 with clipping).  A tile covers up
- * to 4096 owned elements, so a shard of up to about 536 M owned elements
- * fits (about 429 M with clipping).  A larger plan gets ZR_ERR_UNSUPPORTED before
+ * to 2048 owned elements, so a shard of up to about 268 M owned elements
+ * fits (about 214 M with clipping).  A larger plan gets ZR_ERR_UNSUPPORTED before
  * anything is launched: use zr_step with a workspace instead.  With clipping,
  * the second pass reads the gradients again instead of keeping an fp32 copy
  * of the averaged gradient, so results are bit-identical to zr_step's.

@@ -5,8 +5,9 @@
 // back (12 bytes) and writes one bf16 parameter (2 bytes).  Nothing here is
 // a contraction, so there is no tensor-core work; the roofline is HBM
 // bandwidth and the design goal is keeping enough bytes in flight:
-//   * one CTA per tile of up to 4096 owned elements (tiles never cross a
-//     bucket; the hardware block scheduler balances them across the 148 SMs);
+//   * one 128-thread CTA per tile of up to 2048 owned elements (tiles never
+//     cross a bucket; the hardware block scheduler balances them across the
+//     148 SMs, five CTAs per SM);
 //   * each thread owns 8 consecutive elements per iteration and issues the W
 //     16-byte gradient loads of a group (up to 16 replicas) back to back,
 //     plus the 32-byte master / m / v loads, before consuming any of them;

@@ -53,6 +53,22 @@ class ZrPlan:
     def step(self, grads, master, m, v, param_out, step, stream=None):
         zr_step(self.handle, grads, master, m, v, param_out, step, stream)
 
+    def bound_step(self, grads, master, m, v, param_out, stream=None):
+        """A callable f(step) that runs zr_step on fixed buffers with the
+        arguments marshalled once (for tight loops)."""
+        from . import _addr, _check, _lib, _ptr_array, _stream
+        arr = _ptr_array(grads)
+        args = (self.handle, arr, _addr(master), _addr(m), _addr(v), _addr(param_out))
+        s = _stream(stream)
+        fn = _lib.zr_step
+
+        def step_fn(step):
+            st = fn(*args, step, s)
+            if st:
+                _check(st, "zr_step")
+        step_fn._keepalive = (arr, grads, master, m, v, param_out)
+        return step_fn
+
     def step_host(self, host_grads, dev_grads, master, m, v, param_out, host_param_out, step,
                   stream=None):
         zr_step_host(self.handle, host_grads, dev_grads, master, m, v, param_out, host_param_out,
