@@ -28,8 +28,10 @@
  *    written in oracle_adamw_element(), no fused multiply-add (built with
  *    -ffp-contract=off);
  *  - clip coefficient c = min(1, max_norm / (sqrt(S) + 1e-6)) in fp64,
- *    rounded to fp32, S the fp64 sum of exact squares of the averaged
- *    gradient over all N parameters; g <- g * c in fp32 before m and v;
+ *    rounded to fp32, S the sum of the exact fp64 squares of the averaged
+ *    gradient over all N parameters, accumulated with compensated summation
+ *    so that the sum is accurate to a few ulps at any length; g <- g * c in
+ *    fp32 before m and v;
  *  - bf16 conversion: round to nearest, ties to even; NaN stays a quiet NaN.
  *
  * Parity of every function here is pinned by tests/test_oracle_*.py against
@@ -312,11 +314,23 @@ void oracle_adamw(const oracle_scalars* s, const float* g, int64_t n, float* p, 
 /* Global-norm clip                                                         */
 /* ------------------------------------------------------------------------ */
 
-/* Sum of squares in fp64; each square of an fp32 value is exact in fp64. */
+/* Sum of squares in fp64.  Each square of an fp32 value is exact in fp64
+ * (24-bit significand squared fits in 53 bits).  The additions use
+ * Neumaier's compensated summation: alongside the running sum, a running
+ * correction collects the low-order bits every addition rounds away, so the
+ * result is within about two units in the last place of the exact sum
+ * however many terms there are (a plain running sum of 1e8 terms can drift
+ * by ~1e-11 relative). */
 double oracle_sumsq(const float* g, int64_t n) {
-    double acc = 0.0;
-    for (int64_t i = 0; i < n; ++i) acc += (double)g[i] * (double)g[i];
-    return acc;
+    double sum = 0.0, correction = 0.0;
+    for (int64_t i = 0; i < n; ++i) {
+        double x = (double)g[i] * (double)g[i];
+        double t = sum + x;
+        if (fabs(sum) >= fabs(x)) correction += (sum - t) + x;
+        else correction += (x - t) + sum;
+        sum = t;
+    }
+    return sum + correction;
 }
 
 float oracle_clip_coef(double sumsq, float max_norm) {

@@ -63,6 +63,21 @@ def test_squares_are_exact_in_fp64():
     assert oracle.sumsq(np.array([x], np.float32)) == (1.0 + 2.0 ** -23) ** 2
 
 
+def test_sumsq_is_accurate_over_many_terms():
+    """1 followed by 2**20 copies of 2**-27: the exact sum of squares is
+    1 + 2**20 * 2**-54 = 1 + 2**-34.  A plain running sum drops every
+    2**-54 against the 1 and returns 1.0; the oracle must not."""
+    g = np.full(1 + (1 << 20), 2.0 ** -27, np.float32)
+    g[0] = 1.0
+    assert oracle.sumsq(g) == 1.0 + 2.0 ** -34
+    # and a long random sum agrees with an exactly rounded reference
+    import math
+    rng = np.random.default_rng(13)
+    h = (rng.standard_normal(200_000) * 10.0 ** rng.integers(-6, 3, 200_000)).astype(np.float32)
+    exact = math.fsum(float(x) * float(x) for x in h.astype(np.float64))
+    assert abs(oracle.sumsq(h) - exact) <= 4 * 2.0 ** -53 * exact
+
+
 def test_rank_partials_sum_to_global():
     """Per-rank S_r (owned order) summed in rank order equal the global S
     (global order) within 1e-12 relative."""
