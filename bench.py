@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--sweep", action="store_true",
+                    help="1.3B set: bucket cap x W x partition; one JSON record per point")
     return ap.parse_args()
 
 
@@ -391,8 +393,69 @@ def run_zr(args):
     print(json.dumps(line), flush=True)
 
 
+def run_sweep(args):
+    """Every point of the 1.3B sweep (bucket cap {1,5,25,100,400} MB x W
+    {2,8,32,64} x {flat, whole-tensor}); rank 0, plus the most-loaded rank
+    for whole-tensor points.  Prints one JSON record per point."""
+    import torch
+    import synth
+    from sharded_optimizer_step_zr_b200.plan import ZrPlan
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    peak, peak_kind = measured_peak()
+    for wl in synth.sweep_workloads():
+        probe = ZrPlan(wl.shapes, wl.world_size, 0, wl.mode, wl.bucket_cap_bytes, *wl.hp, bind=False)
+        loads = {}
+        for s in probe.segments():
+            loads[s["owner"]] = loads.get(s["owner"], 0) + s["length"]
+        probe.close()
+        ranks = [0]
+        if wl.mode == 1:
+            heavy = max(loads, key=lambda r: (loads[r], -r))
+            if heavy != 0:
+                ranks.append(heavy)
+        for rank in ranks:
+            plan = ZrPlan(wl.shapes, wl.world_size, rank, wl.mode, wl.bucket_cap_bytes, *wl.hp, device=dev)
+            n, W = plan.owned_numel, wl.world_size
+            runs = plan.runs()
+            grads = [torch.empty(n, dtype=torch.bfloat16, device=dev) for _ in range(W)]
+            for w in range(W):
+                synth.fill_owned_grad(grads[w], runs, wl.seed, 1, w, wl.grad_sigma, wl.outlier_frac,
+                                      n_valid=plan.total_numel)
+            master = torch.empty(n, dtype=torch.float32, device=dev)
+            synth.fill_owned_master(master, runs, wl.seed, n_valid=plan.total_numel)
+            m, v = torch.zeros_like(master), torch.zeros_like(master)
+            out = torch.zeros(plan.padded_numel, dtype=torch.bfloat16, device=dev)
+            run_step = plan.bound_step(grads, master, m, v, out, stream)
+            for t in range(args.warmup):
+                run_step(t + 1)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for t in range(args.steps):
+                run_step(args.warmup + t + 1)
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / args.steps
+            bpp = bytes_per_owned_param(W, False)
+            gbs = n * bpp / (ms * 1e-3) / 1e9
+            print(json.dumps({"point": wl.name, "W": W, "rank": rank,
+                              "partition": "flat" if wl.mode == 0 else "whole_tensor",
+                              "bucket_cap_mb": wl.bucket_cap_mb, "n_buckets": plan.n_buckets,
+                              "owned_params": n, "ms_per_step": ms,
+                              "gparams_per_s": n / (ms * 1e-3) / 1e9, "hbm_gbs": gbs,
+                              "frac_of_peak": gbs / peak, "peak_source": peak_kind}), flush=True)
+            plan.close()
+            del grads, master, m, v, out, run_step
+            torch.cuda.empty_cache()
+
+
 def main():
     args = parse()
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:
