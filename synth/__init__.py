@@ -239,6 +239,11 @@ WORKLOADS = {
                                        1e-3, 0.01, max_grad_norm=1.0),
     # Llama-7B, W=64, rank 0, flat, 25 MB buckets, N(0, 1e-3).
     "llama_7b_w64": Workload("llama_7b_w64", "llama_7b", 64, (0,), 0, 25, 1e-3, 0.0),
+    # Small cases of the same kernels, for profiler captures of a few hundred MB:
+    # the W = 64 flat step and the whole-tensor clip step on the GPT-2 set.
+    "gpt2_124m_w64": Workload("gpt2_124m_w64", "gpt2_124m", 64, (0,), 0, 25, 1e-3, 0.0),
+    "gpt2_124m_w8_whole_clip": Workload("gpt2_124m_w8_whole_clip", "gpt2_124m", 8, (3,), 1, 25,
+                                        1e-3, 0.01, max_grad_norm=1.0),
 }
 
 
