@@ -181,8 +181,11 @@ zr_status zr_step(const zr_plan* p, const void* const* grad_ptrs, float* master,
     e = zr::launch_clip_combine(p->d_tile_partials, a.n_tiles, p->d_sumsq_partials, p->world_size, p->rank,
                                 p->hp.max_grad_norm, p->d_clip_coef, p->d_own_sumsq, s);
     if (e != cudaSuccess) return ZR_ERR_CUDA;
-    // Pass 2: scale by the coefficient, AdamW, cast.
+    // Pass 2: scale by the coefficient, AdamW, cast.  Tiles in reverse
+    // order: the first CTAs then read the g scratch that pass 1's last CTAs
+    // wrote, while it is still in L2.
     a.clip_coef = p->d_clip_coef;
+    a.reverse = 1;
     e = zr::launch_tiles(zr::Pass::kStepClip, a, grad_ptrs, scratch, false, s);
     return cuda_status(static_cast<cudaError_t>(e));
 }

@@ -52,6 +52,7 @@ struct LaunchArgs {
     int32_t world_size;
     int32_t w_is_pow2;
     float inv_w;               // 1/W when W is a power of two (exact)
+    int32_t reverse;           // CTA b takes tile n_tiles - 1 - b (see the clip pass 2)
     float* master;
     float* m;
     float* v;

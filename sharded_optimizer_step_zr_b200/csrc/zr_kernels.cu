@@ -161,7 +161,9 @@ __device__ double block_sum(double x) {
 template <int CAP, int G, Pass PASS, bool G_FROM_SCRATCH, bool WRITE_G>
 __global__ void __launch_bounds__(kThreads)
 zr_tile_kernel(const GradPtrs<CAP> gp, const LaunchArgs a) {
-    const Tile tile = a.tiles[blockIdx.x];
+    const int32_t tix = a.reverse ? a.n_tiles - 1 - static_cast<int32_t>(blockIdx.x)
+                                  : static_cast<int32_t>(blockIdx.x);
+    const Tile tile = a.tiles[tix];
     const int W = a.world_size;
     float coef = 1.0f;
     if constexpr (PASS == Pass::kStepClip) coef = *a.clip_coef;
@@ -264,7 +266,7 @@ zr_tile_kernel(const GradPtrs<CAP> gp, const LaunchArgs a) {
     }
     if constexpr (PASS == Pass::kSumsq) {
         const double total = block_sum(sq);
-        if (threadIdx.x == 0) a.tile_partials[blockIdx.x] = total;
+        if (threadIdx.x == 0) a.tile_partials[tix] = total;
     }
 }
 
@@ -276,8 +278,21 @@ zr_clip_combine_kernel(const double* __restrict__ tile_partials, int32_t n_tiles
                        double* partials_all, int32_t world_size, int32_t rank, float max_norm,
                        float* clip_coef_out, double* sumsq_out) {
     __shared__ double part[1024];
+    // Thread t adds partials t, t + B, t + 2B, ... in that order (B = block
+    // size); the loads of 16 of them are issued before their additions so
+    // the block is not bound by one memory round trip per partial.
+    constexpr int kBatch = 16;
+    const int32_t B = static_cast<int32_t>(blockDim.x);
     double x = 0.0;
-    for (int32_t i = threadIdx.x; i < n_tiles; i += blockDim.x) x += tile_partials[i];
+    int32_t i = threadIdx.x;
+    for (; i + (kBatch - 1) * B < n_tiles; i += kBatch * B) {
+        double v[kBatch];
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) v[k] = tile_partials[i + k * B];
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) x += v[k];
+    }
+    for (; i < n_tiles; i += B) x += tile_partials[i];
     part[threadIdx.x] = x;
     __syncthreads();
     for (int stride = blockDim.x / 2; stride >= 1; stride >>= 1) {
