@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--per-bucket", action="store_true",
+                    help="step bucket by bucket (zr_step_bucket per bucket, then zr_step_finish)")
     ap.add_argument("--sweep", action="store_true",
                     help="1.3B set: bucket cap x W x partition; one JSON record per point")
     return ap.parse_args()
@@ -256,6 +258,27 @@ def run_reference(args):
 # GPU arm
 # ---------------------------------------------------------------------------
 
+def bound_bucket_steps(plan, buckets, grads, master, m, v, param_out, stream):
+    """f(step): zr_step_bucket for every bucket this rank owns part of, in
+    backward (bucket) order, then zr_step_finish; arguments marshalled once."""
+    from sharded_optimizer_step_zr_b200 import _addr, _check, _lib, _ptr_array, _stream
+    arr = _ptr_array(grads)
+    ptrs = (_addr(master), _addr(m), _addr(v), _addr(param_out))
+    s = _stream(stream)
+    h = plan.handle
+
+    def step_fn(step):
+        for b in buckets:
+            st = _lib.zr_step_bucket(h, b, arr, *ptrs, step, s)
+            if st:
+                _check(st, "zr_step_bucket")
+        st = _lib.zr_step_finish(h, arr, *ptrs, step, s)
+        if st:
+            _check(st, "zr_step_finish")
+    step_fn._keepalive = (arr, grads, master, m, v, param_out)
+    return step_fn
+
+
 def run_zr(args):
     import torch
     import synth
@@ -299,6 +322,9 @@ def run_zr(args):
 
     step_no = 0
     run_step = plan.bound_step(grads, master, m, v, param_out, stream)   # arguments marshalled once
+    my_buckets = sorted({s["bucket"] for s in plan.segments() if s["owner"] == zr_rank})
+    if args.per_bucket:
+        run_step = bound_bucket_steps(plan, my_buckets, grads, master, m, v, param_out, stream)
 
     for _ in range(args.warmup):
         step_no += 1
@@ -372,6 +398,8 @@ def run_zr(args):
     if grank != 0:
         return
     launches_per_step = 3 if clip else 1
+    if args.per_bucket:
+        launches_per_step = len(my_buckets) + (2 if clip else 0)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -379,6 +407,7 @@ def run_zr(args):
         "config": {"workload": wl.name, "param_set": wl.param_set, "W": W, "rank": zr_rank,
                    "partition": "flat" if wl.mode == 0 else "whole_tensor",
                    "bucket_cap_mb": wl.bucket_cap_mb, "clip": clip, "owned_params": n,
+                   "per_bucket": bool(args.per_bucket), "buckets_stepped": len(my_buckets),
                    "bytes_per_owned_param": bpp,
                    "l2": f"no flush: each step touches {alg_bytes / 1e6:.0f} MB > 126 MB L2"},
         "hbm_gbs": achieved,

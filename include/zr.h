@@ -168,6 +168,39 @@ zr_status zr_plan_set_sumsq_partials(zr_plan* plan, double* d_partials);
 zr_status zr_step(const zr_plan* plan, const void* const* grad_ptrs, float* master, float* m,
                   float* v, void* param_out, int64_t step, zr_stream_t stream);
 
+/* One bucket of the step, for overlapping the optimizer with the backward
+ * pass ("Scaling training to thousands of GPUs", 03:41 DP: a bucket's
+ * collective starts as soon as backward has produced its gradients;
+ * "CS336 lecture 8", ZeRO level 2: a gradient is released as soon as it has
+ * been reduced).  Enqueue it on a stream that waits for the bucket's
+ * gradients (e.g. cudaStreamWaitEvent).  Arguments as zr_step, plus
+ * 0 <= bucket < n_buckets; only this rank's elements of that bucket are read
+ * and written, and a bucket this rank owns nothing of is a no-op.
+ *   Without clipping: the fused step on the bucket's elements.  Calling it
+ *   once per bucket, in any order, gives exactly zr_step's result (the step
+ *   is elementwise).
+ *   With clipping: the coefficient needs every bucket's sum of squares, so
+ *   this runs the reduce and the sums of squares for the bucket (writing the
+ *   fp32 averaged gradient to the workspace when W > 4; master, m, v and
+ *   param_out are not touched and may be NULL); after every bucket,
+ *   zr_step_finish updates all elements.  For W > 4 the bucket's gradient
+ *   buffers may be released as soon as this call's work is done.
+ * Errors: as zr_step; ZR_ERR_INVALID_ARG for a bucket out of range. */
+zr_status zr_step_bucket(const zr_plan* plan, int32_t bucket, const void* const* grad_ptrs,
+                         float* master, float* m, float* v, void* param_out, int64_t step,
+                         zr_stream_t stream);
+
+/* Completes a bucket-by-bucket step of a plan with clipping: the norm from
+ * all buckets' sums of squares (and the other ranks' entries of the
+ * partials array, as for zr_step), then the scaled AdamW update and bf16
+ * cast of every owned element.  For W > 4 it reads the averaged gradient
+ * that zr_step_bucket stored and grad_ptrs may be NULL; for W <= 4 it reads
+ * the gradients again, so grad_ptrs must still hold every bucket's values.
+ * For plans without clipping it does nothing and returns ZR_OK.  The result
+ * equals zr_step's bit for bit. */
+zr_status zr_step_finish(const zr_plan* plan, const void* const* grad_ptrs, float* master, float* m,
+                         float* v, void* param_out, int64_t step, zr_stream_t stream);
+
 /* zr_step with host-resident gradients and a host copy of the result, for
  * callers whose gradients arrive in host memory.  On `stream`: copies
  * host_grad_ptrs[w] (owned_numel bf16, pinned host memory for an

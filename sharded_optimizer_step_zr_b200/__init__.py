@@ -38,7 +38,8 @@ ZR_MAX_WORLD_SIZE = 512
 
 EXPORTED = [
     "zr_plan_create", "zr_plan_query", "zr_plan_segments", "zr_plan_workspace_bytes",
-    "zr_plan_set_workspace", "zr_plan_set_sumsq_partials", "zr_step", "zr_step_host",
+    "zr_plan_set_workspace", "zr_plan_set_sumsq_partials", "zr_step", "zr_step_bucket",
+    "zr_step_finish", "zr_step_host",
     "zr_grad_sumsq", "zr_debug_reduce", "zr_step_no_alloc", "zr_plan_destroy", "zr_status_string",
 ]
 ZR_NO_ALLOC_SCRATCH_BYTES = 4 << 20
@@ -65,6 +66,8 @@ _lib.zr_plan_workspace_bytes.argtypes = [_vp, _P(_u64)]
 _lib.zr_plan_set_workspace.argtypes = [_vp, _vp, _u64, _vp]
 _lib.zr_plan_set_sumsq_partials.argtypes = [_vp, _vp]
 _lib.zr_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
+_lib.zr_step_bucket.argtypes = [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
+_lib.zr_step_finish.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_step_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_grad_sumsq.argtypes = [_vp, _vp, _vp, _vp]
 _lib.zr_debug_reduce.argtypes = [_vp, _vp, _vp, _vp]
@@ -178,6 +181,19 @@ def zr_plan_set_sumsq_partials(plan: int, partials) -> None:
 def zr_step(plan: int, grads, master, m, v, param_out, step: int, stream=None) -> None:
     _check(_lib.zr_step(plan, _ptr_array(grads), _addr(master), _addr(m), _addr(v),
                         _addr(param_out), int(step), _stream(stream)), "zr_step")
+
+
+def zr_step_bucket(plan: int, bucket: int, grads, master, m, v, param_out, step: int,
+                   stream=None) -> None:
+    _check(_lib.zr_step_bucket(plan, int(bucket), _ptr_array(grads), _addr(master), _addr(m),
+                               _addr(v), _addr(param_out), int(step), _stream(stream)),
+           "zr_step_bucket")
+
+
+def zr_step_finish(plan: int, grads, master, m, v, param_out, step: int, stream=None) -> None:
+    _check(_lib.zr_step_finish(plan, _ptr_array(grads) if grads is not None else None, _addr(master),
+                               _addr(m), _addr(v), _addr(param_out), int(step), _stream(stream)),
+           "zr_step_finish")
 
 
 def zr_step_host(plan: int, host_grads, dev_grads, master, m, v, param_out, host_param_out,

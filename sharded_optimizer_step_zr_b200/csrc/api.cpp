@@ -190,6 +190,71 @@ zr_status zr_step(const zr_plan* p, const void* const* grad_ptrs, float* master,
     return cuda_status(static_cast<cudaError_t>(e));
 }
 
+zr_status zr_step_bucket(const zr_plan* p, int32_t bucket, const void* const* grad_ptrs, float* master, float* m,
+                         float* v, void* param_out, int64_t step, zr_stream_t stream) {
+    if (!p || step < 1) return ZR_ERR_INVALID_ARG;
+    if (bucket < 0 || bucket >= p->n_buckets) return ZR_ERR_INVALID_ARG;
+    if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
+    const int32_t first = p->bucket_first_tile[bucket];
+    const int32_t count = p->bucket_first_tile[bucket + 1] - first;
+    if (count == 0) return ZR_OK;   // this rank owns nothing in the bucket
+    zr_status st = check_grads(p, grad_ptrs);
+    if (st != ZR_OK) return st;
+    zr::LaunchArgs a = base_args(p);
+    a.tiles = p->d_tiles + first;
+    a.n_tiles = count;
+    a.tile_base = first;
+    void* s = stream;
+    if (!p->clip_enabled()) {
+        if (!master || !m || !v || !param_out) return ZR_ERR_INVALID_ARG;
+        if (!aligned16(master) || !aligned16(m) || !aligned16(v) || !aligned16(param_out)) return ZR_ERR_ALIGNMENT;
+        a.master = master;
+        a.m = m;
+        a.v = v;
+        a.param_out = static_cast<uint16_t*>(param_out);
+        a.s = zr::adam_scalars(p->hp, step);
+        return cuda_status(static_cast<cudaError_t>(zr::launch_tiles(zr::Pass::kStep, a, grad_ptrs, false, false, s)));
+    }
+    // Clipping: the bucket's share of pass 1 (reduce, per-tile sums of
+    // squares, the fp32 g scratch when W > 4); zr_step_finish does the rest.
+    const bool scratch = p->clip_uses_scratch();
+    a.g_buf = p->d_g_scratch;
+    a.tile_partials = p->d_tile_partials;
+    return cuda_status(static_cast<cudaError_t>(zr::launch_tiles(zr::Pass::kSumsq, a, grad_ptrs, false, scratch, s)));
+}
+
+zr_status zr_step_finish(const zr_plan* p, const void* const* grad_ptrs, float* master, float* m, float* v,
+                         void* param_out, int64_t step, zr_stream_t stream) {
+    if (!p || step < 1) return ZR_ERR_INVALID_ARG;
+    if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
+    if (!p->clip_enabled() || p->owned_numel() == 0) return ZR_OK;
+    if (!p->d_sumsq_partials) return ZR_ERR_NO_WORKSPACE;
+    const bool scratch = p->clip_uses_scratch();
+    if (!scratch) {
+        zr_status st = check_grads(p, grad_ptrs);   // pass 2 reads the gradients again
+        if (st != ZR_OK) return st;
+    } else {
+        grad_ptrs = nullptr;                         // pass 2 reads the g scratch only
+    }
+    if (!master || !m || !v || !param_out) return ZR_ERR_INVALID_ARG;
+    if (!aligned16(master) || !aligned16(m) || !aligned16(v) || !aligned16(param_out)) return ZR_ERR_ALIGNMENT;
+    zr::LaunchArgs a = base_args(p);
+    a.master = master;
+    a.m = m;
+    a.v = v;
+    a.param_out = static_cast<uint16_t*>(param_out);
+    a.s = zr::adam_scalars(p->hp, step);
+    a.g_buf = p->d_g_scratch;
+    void* s = stream;
+    int e = zr::launch_clip_combine(p->d_tile_partials, a.n_tiles, p->d_sumsq_partials, p->world_size, p->rank,
+                                    p->hp.max_grad_norm, p->d_clip_coef, p->d_own_sumsq, s);
+    if (e != cudaSuccess) return ZR_ERR_CUDA;
+    a.clip_coef = p->d_clip_coef;
+    a.reverse = 1;
+    e = zr::launch_tiles(zr::Pass::kStepClip, a, grad_ptrs, scratch, false, s);
+    return cuda_status(static_cast<cudaError_t>(e));
+}
+
 zr_status zr_grad_sumsq(const zr_plan* p, const void* const* grad_ptrs, double* d_out, zr_stream_t stream) {
     if (!p || !d_out) return ZR_ERR_INVALID_ARG;
     if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;

@@ -53,6 +53,8 @@ struct LaunchArgs {
     int32_t w_is_pow2;
     float inv_w;               // 1/W when W is a power of two (exact)
     int32_t reverse;           // CTA b takes tile n_tiles - 1 - b (see the clip pass 2)
+    int32_t tile_base;         // index of tiles[0] in the plan's whole tile list
+                               // (per-tile partials are stored at that index)
     float* master;
     float* m;
     float* v;

@@ -266,7 +266,7 @@ zr_tile_kernel(const GradPtrs<CAP> gp, const LaunchArgs a) {
     }
     if constexpr (PASS == Pass::kSumsq) {
         const double total = block_sum(sq);
-        if (threadIdx.x == 0) a.tile_partials[tix] = total;
+        if (threadIdx.x == 0) a.tile_partials[a.tile_base + tix] = total;
     }
 }
 
@@ -314,9 +314,10 @@ zr_clip_combine_kernel(const double* __restrict__ tile_partials, int32_t n_tiles
 
 template <int CAP, int G, Pass PASS, bool FROM, bool WRITE>
 cudaError_t launch_one(const LaunchArgs& a, const void* const* grad_ptrs, cudaStream_t stream) {
+    // grad_ptrs may be NULL for the pass that reads the g scratch instead.
     GradPtrs<CAP> gp;
     for (int w = 0; w < CAP; ++w)
-        gp.p[w] = w < a.world_size ? static_cast<const uint16_t*>(grad_ptrs[w]) : nullptr;
+        gp.p[w] = (grad_ptrs != nullptr && w < a.world_size) ? static_cast<const uint16_t*>(grad_ptrs[w]) : nullptr;
     zr_tile_kernel<CAP, G, PASS, FROM, WRITE><<<a.n_tiles, kThreads, 0, stream>>>(gp, a);
     return cudaGetLastError();
 }

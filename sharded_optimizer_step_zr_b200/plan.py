@@ -7,7 +7,7 @@ from __future__ import annotations
 
 from . import (ZR_PARTITION_FLAT, zr_debug_reduce, zr_grad_sumsq, zr_plan_create, zr_plan_destroy,
                zr_plan_query, zr_plan_segments, zr_plan_set_sumsq_partials, zr_plan_set_workspace,
-               zr_plan_workspace_bytes, zr_step, zr_step_host)
+               zr_plan_workspace_bytes, zr_step, zr_step_bucket, zr_step_finish, zr_step_host)
 
 
 class ZrPlan:
@@ -52,6 +52,12 @@ class ZrPlan:
 
     def step(self, grads, master, m, v, param_out, step, stream=None):
         zr_step(self.handle, grads, master, m, v, param_out, step, stream)
+
+    def step_bucket(self, bucket, grads, master, m, v, param_out, step, stream=None):
+        zr_step_bucket(self.handle, bucket, grads, master, m, v, param_out, step, stream)
+
+    def step_finish(self, grads, master, m, v, param_out, step, stream=None):
+        zr_step_finish(self.handle, grads, master, m, v, param_out, step, stream)
 
     def bound_step(self, grads, master, m, v, param_out, stream=None):
         """A callable f(step) that runs zr_step on fixed buffers with the
