@@ -166,6 +166,39 @@ void build_tiles(zr_plan& p) {
     p.bucket_first_tile[p.n_buckets] = static_cast<int32_t>(p.tiles.size());
 }
 
+// Self-check of the tile list before anything reaches a kernel: the tiles
+// cover this rank's owned range [0, owned) exactly once, each maps owned
+// offsets to the same global offsets as the segment it came from, stays
+// inside [0, padded), and carries vector flags only where the 8-element
+// alignment holds.
+bool tiles_are_consistent(const zr_plan& p) {
+    const int64_t owned = p.rank_numel[p.rank];
+    std::vector<std::pair<int64_t, int64_t>> span;   // (owned start, global start - owned start)
+    for (const zr_segment& s : p.segments)
+        if (s.owner == p.rank) span.push_back({s.owned_offset, s.global_offset - s.owned_offset});
+    std::sort(span.begin(), span.end());
+    std::vector<std::pair<int64_t, int64_t>> cover;
+    for (const Tile& t : p.tiles) {
+        if (t.len <= 0 || t.len > kTileElems || t.owned < 0 || t.owned + t.len > owned) return false;
+        if (t.global < 0 || t.global + t.len > p.padded_numel) return false;
+        auto it = std::upper_bound(span.begin(), span.end(), std::make_pair(t.owned, std::numeric_limits<int64_t>::max()));
+        if (it == span.begin()) return false;
+        --it;
+        if (t.global - t.owned != it->second) return false;
+        const bool vec = (t.owned % 8 == 0) && (t.len % 8 == 0);
+        if ((t.flags & kTileVector) && !vec) return false;
+        if ((t.flags & kTileStoreVector) && !(vec && t.global % 8 == 0)) return false;
+        cover.push_back({t.owned, t.len});
+    }
+    std::sort(cover.begin(), cover.end());
+    int64_t next = 0;
+    for (const auto& c : cover) {
+        if (c.first != next) return false;
+        next += c.second;
+    }
+    return next == owned;
+}
+
 }  // namespace
 
 zr_status build_plan(zr_plan& p, int32_t n_tensors, const int32_t* ndims,
@@ -204,6 +237,7 @@ zr_status build_plan(zr_plan& p, int32_t n_tensors, const int32_t* ndims,
     pack_buckets(p);
     cut_segments(p);
     build_tiles(p);
+    if (!tiles_are_consistent(p)) return ZR_ERR_INVALID_ARG;
     return ZR_OK;
 }
 

@@ -1,0 +1,44 @@
+"""bench.py's output contract, checked on the CPU through its reference arm
+(the oracle timed on a bounded sample) and its helpers."""
+import json
+import os
+import subprocess
+import sys
+
+import bench
+import synth
+from conftest import ROOT
+
+
+def test_reference_arm_prints_one_json_line():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--steps", "2", "--warmup", "1"], capture_output=True, text=True,
+                         timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e", "impl"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "Gparams/s"
+    assert d["config"]["workload"] == bench.DEFAULT_CONFIG
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    assert d["value"] > 0
+
+
+def test_algorithmic_bytes_per_param():
+    # 2W gradient reads + 12 state reads + 12 state writes + 2 bf16 writes
+    assert bench.bytes_per_owned_param(8, False) == 42
+    assert bench.bytes_per_owned_param(64, False) == 154
+    assert bench.bytes_per_owned_param(8, True) == 50     # + fp32 g scratch write and read
+    assert bench.bytes_per_owned_param(2, True) == 34     # + gradients read again
+
+
+def test_shard_rank_and_workloads():
+    wl = synth.WORKLOADS["gpt_1p3b_w8_whole_clip"]
+    assert bench.shard_rank(wl, 0, 1) == 3
+    assert [bench.shard_rank(wl, i, 8) for i in range(8)] == [3, 4, 5, 6, 7, 0, 1, 2]
+    assert bench.workload("gpt2_124m_w8").world_size == 8
+    assert len(synth.sweep_workloads()) == 40
