@@ -202,12 +202,18 @@ zr_status zr_step_finish(const zr_plan* plan, const void* const* grad_ptrs, floa
                          float* v, void* param_out, int64_t step, zr_stream_t stream);
 
 /* zr_step with host-resident gradients and a host copy of the result, for
- * callers whose gradients arrive in host memory.  On `stream`: copies
- * host_grad_ptrs[w] (owned_numel bf16, pinned host memory for an
- * asynchronous copy) into dev_grad_ptrs[w], runs zr_step, then copies this
- * rank's positions of param_out into host_param_out (a host buffer in the
- * global layout, padded_numel bf16).  Asynchronous: the host buffers must
- * stay untouched until the stream is synchronised. */
+ * callers whose gradients arrive in host memory.  Copies host_grad_ptrs[w]
+ * (owned_numel bf16, owned order; pinned host memory for asynchronous
+ * copies) into dev_grad_ptrs[w], runs the step, and copies this rank's
+ * positions of param_out into host_param_out (a host buffer in the global
+ * layout, padded_numel bf16).  The owned range is cut into up to 4 chunks
+ * (1/2, 1/4, 1/8, 1/8 of it): while one chunk's gradients cross PCIe,
+ * earlier chunks are stepped and their parameters copied back, on two
+ * internal copy streams of the plan
+ * (created by the plan's first zr_step_host call, released by
+ * zr_plan_destroy) joined to `stream` by events.  Results equal zr_step's.
+ * Asynchronous: `stream` reaches the end of the call only when every copy is
+ * done; the host buffers must stay untouched until then. */
 zr_status zr_step_host(const zr_plan* plan, const void* const* host_grad_ptrs,
                        void* const* dev_grad_ptrs, float* master, float* m, float* v,
                        void* param_out, void* host_param_out, int64_t step, zr_stream_t stream);

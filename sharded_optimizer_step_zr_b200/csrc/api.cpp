@@ -5,6 +5,7 @@
 // device memory and never synchronises.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstring>
 #include <new>
 
@@ -36,7 +37,24 @@ zr::LaunchArgs base_args(const zr_plan* p) {
     return a;
 }
 
+zr_status ensure_host_pipeline(const zr_plan* p) {
+    if (p->host_pipeline_ready) return ZR_OK;
+    if (cudaStreamCreateWithFlags(&p->h2d_stream, cudaStreamNonBlocking) != cudaSuccess) return ZR_ERR_CUDA;
+    if (cudaStreamCreateWithFlags(&p->d2h_stream, cudaStreamNonBlocking) != cudaSuccess) return ZR_ERR_CUDA;
+    for (cudaEvent_t& e : p->host_events)
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return ZR_ERR_CUDA;
+    p->host_pipeline_ready = true;
+    return ZR_OK;
+}
+
 }  // namespace
+
+zr_plan::~zr_plan() {
+    for (cudaEvent_t e : host_events)
+        if (e) cudaEventDestroy(e);
+    if (h2d_stream) cudaStreamDestroy(h2d_stream);
+    if (d2h_stream) cudaStreamDestroy(d2h_stream);
+}
 
 extern "C" {
 
@@ -131,14 +149,18 @@ zr_status zr_plan_set_workspace(zr_plan* p, void* d_ws, uint64_t bytes, zr_strea
     p->d_workspace = d_ws;
     p->workspace_bytes = bytes;
     p->d_tiles = reinterpret_cast<zr::Tile*>(base + L.tiles);
+    p->d_tiles_by_owned = reinterpret_cast<zr::Tile*>(base + L.tiles_by_owned);
     p->d_tile_partials = p->clip_enabled() ? reinterpret_cast<double*>(base + L.tile_partials) : nullptr;
     p->d_clip_coef = reinterpret_cast<float*>(base + L.clip_coef);
     p->d_own_sumsq = reinterpret_cast<double*>(base + L.own_sumsq);
     p->d_g_scratch = p->clip_uses_scratch() ? reinterpret_cast<float*>(base + L.g_scratch) : nullptr;
     if (!p->tiles.empty()) {
-        const cudaError_t e = cudaMemcpyAsync(p->d_tiles, p->tiles.data(), sizeof(zr::Tile) * p->tiles.size(),
-                                              cudaMemcpyHostToDevice, reinterpret_cast<cudaStream_t>(stream));
-        if (e != cudaSuccess) return ZR_ERR_CUDA;
+        const size_t bytes_tiles = sizeof(zr::Tile) * p->tiles.size();
+        cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+        if (cudaMemcpyAsync(p->d_tiles, p->tiles.data(), bytes_tiles, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(p->d_tiles_by_owned, p->tiles_by_owned.data(), bytes_tiles, cudaMemcpyHostToDevice, s) !=
+                cudaSuccess)
+            return ZR_ERR_CUDA;
     }
     return ZR_OK;
 }
@@ -203,7 +225,6 @@ zr_status zr_step_bucket(const zr_plan* p, int32_t bucket, const void* const* gr
     zr::LaunchArgs a = base_args(p);
     a.tiles = p->d_tiles + first;
     a.n_tiles = count;
-    a.tile_base = first;
     void* s = stream;
     if (!p->clip_enabled()) {
         if (!master || !m || !v || !param_out) return ZR_ERR_INVALID_ARG;
@@ -297,36 +318,123 @@ zr_status zr_step_host(const zr_plan* p, const void* const* host_grad_ptrs, void
     if (n == 0) return ZR_OK;
     for (int32_t w = 0; w < p->world_size; ++w)
         if (!host_grad_ptrs[w]) return ZR_ERR_INVALID_ARG;
-    zr_status st = check_grads(p, const_cast<const void* const*>(dev_grad_ptrs));
+    const void* const* dev_grads = const_cast<const void* const*>(dev_grad_ptrs);
+    zr_status st = check_grads(p, dev_grads);
     if (st != ZR_OK) return st;
-    if (!param_out || !aligned16(param_out)) return param_out ? ZR_ERR_ALIGNMENT : ZR_ERR_INVALID_ARG;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    for (int32_t w = 0; w < p->world_size; ++w) {
-        if (cudaMemcpyAsync(dev_grad_ptrs[w], host_grad_ptrs[w], sizeof(uint16_t) * static_cast<size_t>(n),
-                            cudaMemcpyHostToDevice, s) != cudaSuccess)
-            return ZR_ERR_CUDA;
+    if (!master || !m || !v || !param_out) return ZR_ERR_INVALID_ARG;
+    if (!aligned16(master) || !aligned16(m) || !aligned16(v) || !aligned16(param_out)) return ZR_ERR_ALIGNMENT;
+    const bool clip = p->clip_enabled();
+    if (clip && !p->d_sumsq_partials) return ZR_ERR_NO_WORKSPACE;
+    st = ensure_host_pipeline(p);
+    if (st != ZR_OK) return st;
+
+    // Chunks of the owned range, cut at tile boundaries (tiles in owned
+    // order), halving in size: 1/2, 1/4, 1/8, 1/8.  Each chunk's copy-back
+    // overlaps the next chunk's copy-in, so only the last eighth of the
+    // copy-back is exposed, and the copy-in stays in few large transfers
+    // (small host-to-device copies lose PCIe throughput).
+    const int32_t n_tiles = static_cast<int32_t>(p->tiles_by_owned.size());
+    const int K = static_cast<int>(std::min<int32_t>(zr_plan::kHostChunks, n_tiles));
+    int32_t bounds[zr_plan::kHostChunks + 1];
+    bounds[0] = 0;
+    {
+        int64_t seen = 0;
+        int k = 1;
+        for (int32_t i = 0; i < n_tiles && k < K; ++i) {
+            seen += p->tiles_by_owned[i].len;
+            const int64_t target = n - (n >> k);   // n/2, 3n/4, 7n/8, ...
+            if (seen >= target) bounds[k++] = i + 1;
+        }
+        for (; k <= K; ++k) bounds[k] = n_tiles;
     }
-    st = zr_step(p, const_cast<const void* const*>(dev_grad_ptrs), master, m, v, param_out, step, stream);
-    if (st != ZR_OK) return st;
-    // This rank's positions of the parameter buffer: one copy per merged run.
-    const uint16_t* src = static_cast<const uint16_t*>(param_out);
-    uint16_t* dst = static_cast<uint16_t*>(host_param_out);
-    int64_t run_start = -1, run_len = 0;
-    auto flush = [&]() -> bool {
-        if (run_len == 0) return true;
-        return cudaMemcpyAsync(dst + run_start, src + run_start, sizeof(uint16_t) * static_cast<size_t>(run_len),
-                               cudaMemcpyDeviceToHost, s) == cudaSuccess;
+    cudaStream_t S = reinterpret_cast<cudaStream_t>(stream);
+    cudaStream_t C = p->h2d_stream, D = p->d2h_stream;
+    cudaEvent_t* ev_in = p->host_events;                       // K: chunk k's gradients on the device
+    cudaEvent_t* ev_done = p->host_events + zr_plan::kHostChunks;   // K: chunk k's parameters written
+    cudaEvent_t ev_start = p->host_events[2 * zr_plan::kHostChunks];
+    cudaEvent_t ev_end = p->host_events[2 * zr_plan::kHostChunks + 1];
+    // The copies may overwrite the device gradient buffers only after the
+    // work already queued on the caller's stream.
+    if (cudaEventRecord(ev_start, S) != cudaSuccess || cudaStreamWaitEvent(C, ev_start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(D, ev_start, 0) != cudaSuccess)
+        return ZR_ERR_CUDA;
+
+    zr::LaunchArgs a = base_args(p);
+    a.master = master;
+    a.m = m;
+    a.v = v;
+    a.param_out = static_cast<uint16_t*>(param_out);
+    a.s = zr::adam_scalars(p->hp, step);
+    const bool scratch = p->clip_uses_scratch();
+    a.g_buf = p->d_g_scratch;
+    a.tile_partials = p->d_tile_partials;
+    const uint16_t* out_dev = static_cast<const uint16_t*>(param_out);
+    uint16_t* out_host = static_cast<uint16_t*>(host_param_out);
+
+    auto chunk_args = [&](int k) {
+        zr::LaunchArgs c = a;
+        c.tiles = p->d_tiles_by_owned + bounds[k];
+        c.n_tiles = bounds[k + 1] - bounds[k];
+        return c;
     };
-    for (const zr::Tile& t : p->tiles) {
-        if (run_len > 0 && run_start + run_len == t.global) {
-            run_len += t.len;
-        } else {
-            if (!flush()) return ZR_ERR_CUDA;
-            run_start = t.global;
-            run_len = t.len;
+    auto copy_out = [&](int k) -> bool {
+        if (cudaStreamWaitEvent(D, ev_done[k], 0) != cudaSuccess) return false;
+        int64_t run_start = -1, run_len = 0;
+        for (int32_t i = bounds[k]; i <= bounds[k + 1]; ++i) {
+            const bool more = i < bounds[k + 1];
+            if (more && run_len > 0 && run_start + run_len == p->tiles_by_owned[i].global) {
+                run_len += p->tiles_by_owned[i].len;
+                continue;
+            }
+            if (run_len > 0 &&
+                cudaMemcpyAsync(out_host + run_start, out_dev + run_start, sizeof(uint16_t) * run_len,
+                                cudaMemcpyDeviceToHost, D) != cudaSuccess)
+                return false;
+            if (more) {
+                run_start = p->tiles_by_owned[i].global;
+                run_len = p->tiles_by_owned[i].len;
+            }
+        }
+        return true;
+    };
+
+    for (int k = 0; k < K; ++k) {
+        if (bounds[k + 1] == bounds[k]) continue;
+        const zr::Tile& first = p->tiles_by_owned[bounds[k]];
+        const zr::Tile& last = p->tiles_by_owned[bounds[k + 1] - 1];
+        const int64_t o0 = first.owned, len = last.owned + last.len - first.owned;
+        for (int32_t w = 0; w < p->world_size; ++w) {
+            if (cudaMemcpyAsync(static_cast<uint16_t*>(dev_grad_ptrs[w]) + o0,
+                                static_cast<const uint16_t*>(host_grad_ptrs[w]) + o0, sizeof(uint16_t) * len,
+                                cudaMemcpyHostToDevice, C) != cudaSuccess)
+                return ZR_ERR_CUDA;
+        }
+        if (cudaEventRecord(ev_in[k], C) != cudaSuccess || cudaStreamWaitEvent(S, ev_in[k], 0) != cudaSuccess)
+            return ZR_ERR_CUDA;
+        const zr::LaunchArgs c = chunk_args(k);
+        if (!clip) {
+            if (zr::launch_tiles(zr::Pass::kStep, c, dev_grads, false, false, S) != cudaSuccess) return ZR_ERR_CUDA;
+            if (cudaEventRecord(ev_done[k], S) != cudaSuccess || !copy_out(k)) return ZR_ERR_CUDA;
+        } else if (zr::launch_tiles(zr::Pass::kSumsq, c, dev_grads, false, scratch, S) != cudaSuccess) {
+            return ZR_ERR_CUDA;
         }
     }
-    if (!flush()) return ZR_ERR_CUDA;
+    if (clip) {
+        if (zr::launch_clip_combine(p->d_tile_partials, n_tiles, p->d_sumsq_partials, p->world_size, p->rank,
+                                    p->hp.max_grad_norm, p->d_clip_coef, p->d_own_sumsq, S) != cudaSuccess)
+            return ZR_ERR_CUDA;
+        a.clip_coef = p->d_clip_coef;
+        for (int k = 0; k < K; ++k) {
+            if (bounds[k + 1] == bounds[k]) continue;
+            const zr::LaunchArgs c = chunk_args(k);
+            if (zr::launch_tiles(zr::Pass::kStepClip, c, dev_grads, scratch, false, S) != cudaSuccess)
+                return ZR_ERR_CUDA;
+            if (cudaEventRecord(ev_done[k], S) != cudaSuccess || !copy_out(k)) return ZR_ERR_CUDA;
+        }
+    }
+    // The caller's stream reaches this point only when every copy is done.
+    if (cudaEventRecord(ev_end, D) != cudaSuccess || cudaStreamWaitEvent(S, ev_end, 0) != cudaSuccess)
+        return ZR_ERR_CUDA;
     return ZR_OK;
 }
 

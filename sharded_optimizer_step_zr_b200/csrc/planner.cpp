@@ -146,6 +146,7 @@ void build_tiles(zr_plan& p) {
             tile.global = global;
             tile.len = static_cast<int32_t>(len);
             tile.bucket = b;
+            tile.index = static_cast<int32_t>(p.tiles.size());
             const bool vec = (owned % 8 == 0) && (len % 8 == 0);
             tile.flags = (vec ? kTileVector : 0) | ((vec && global % 8 == 0) ? kTileStoreVector : 0);
             p.tiles.push_back(tile);
@@ -164,6 +165,9 @@ void build_tiles(zr_plan& p) {
         }
     }
     p.bucket_first_tile[p.n_buckets] = static_cast<int32_t>(p.tiles.size());
+    p.tiles_by_owned = p.tiles;
+    std::sort(p.tiles_by_owned.begin(), p.tiles_by_owned.end(),
+              [](const Tile& x, const Tile& y) { return x.owned < y.owned; });
 }
 
 // Self-check of the tile list before anything reaches a kernel: the tiles
@@ -247,6 +251,8 @@ WorkspaceLayout workspace_layout(const zr_plan& p) {
     WorkspaceLayout L{};
     uint64_t off = 0;
     L.tiles = off;
+    off = align256(off + sizeof(Tile) * std::max<size_t>(1, p.tiles.size()));
+    L.tiles_by_owned = off;
     off = align256(off + sizeof(Tile) * std::max<size_t>(1, p.tiles.size()));
     L.tile_partials = off;
     off = align256(off + (p.clip_enabled() ? sizeof(double) * std::max<size_t>(1, p.tiles.size()) : 0));

@@ -1,6 +1,8 @@
 // Internal types shared by the planner, the C ABI layer and the kernels.
 #pragma once
 
+#include <cuda_runtime.h>
+
 #include <cstdint>
 #include <vector>
 
@@ -16,7 +18,8 @@ struct Tile {
     int32_t len;       // element count, 1..kTileElems
     int32_t flags;     // kTileVector | kTileStoreVector
     int32_t bucket;
-    int32_t reserved;
+    int32_t index;     // position in the plan's tile list (bucket order):
+                       // where the tile's clip partial is stored
 };
 static_assert(sizeof(Tile) == 32, "Tile is 32 bytes");
 
@@ -53,8 +56,6 @@ struct LaunchArgs {
     int32_t w_is_pow2;
     float inv_w;               // 1/W when W is a power of two (exact)
     int32_t reverse;           // CTA b takes tile n_tiles - 1 - b (see the clip pass 2)
-    int32_t tile_base;         // index of tiles[0] in the plan's whole tile list
-                               // (per-tile partials are stored at that index)
     float* master;
     float* m;
     float* v;
@@ -97,17 +98,29 @@ struct zr_plan {
     std::vector<zr_segment> segments;    // all ranks
     std::vector<zr::Tile> tiles;         // this rank, bucket by bucket
     std::vector<int32_t> bucket_first_tile;  // n_buckets + 1 entries
+    std::vector<zr::Tile> tiles_by_owned;    // the same tiles sorted by owned offset
 
     // device binding
     int device = -1;
     void* d_workspace = nullptr;
     uint64_t workspace_bytes = 0;
     zr::Tile* d_tiles = nullptr;
+    zr::Tile* d_tiles_by_owned = nullptr;
     double* d_tile_partials = nullptr;
     float* d_clip_coef = nullptr;
     double* d_own_sumsq = nullptr;
     float* d_g_scratch = nullptr;
     double* d_sumsq_partials = nullptr;   // caller-owned, world_size doubles
+
+    // zr_step_host's copy streams and events, created on its first call
+    // (host-side resources, not part of the plan's observable state).
+    static constexpr int kHostChunks = 4;
+    mutable cudaStream_t h2d_stream = nullptr;
+    mutable cudaStream_t d2h_stream = nullptr;
+    mutable cudaEvent_t host_events[2 * kHostChunks + 2] = {};
+    mutable bool host_pipeline_ready = false;
+
+    ~zr_plan();
 
     bool clip_enabled() const { return hp.max_grad_norm > 0.0f; }
     bool clip_uses_scratch() const { return clip_enabled() && world_size > 4; }
@@ -120,7 +133,7 @@ zr_status build_plan(zr_plan& p, int32_t n_tensors, const int32_t* ndims,
                      const int64_t* const* shapes);
 // Workspace layout: offsets of each region, total bytes.
 struct WorkspaceLayout {
-    uint64_t tiles, tile_partials, clip_coef, own_sumsq, g_scratch, total;
+    uint64_t tiles, tiles_by_owned, tile_partials, clip_coef, own_sumsq, g_scratch, total;
 };
 WorkspaceLayout workspace_layout(const zr_plan& p);
 AdamScalars adam_scalars(const zr_adamw& hp, int64_t step);

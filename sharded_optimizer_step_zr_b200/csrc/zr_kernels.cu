@@ -266,7 +266,7 @@ zr_tile_kernel(const GradPtrs<CAP> gp, const LaunchArgs a) {
     }
     if constexpr (PASS == Pass::kSumsq) {
         const double total = block_sum(sq);
-        if (threadIdx.x == 0) a.tile_partials[a.tile_base + tix] = total;
+        if (threadIdx.x == 0) a.tile_partials[tile.index] = total;
     }
 }
 

@@ -215,3 +215,45 @@ def test_bad_alignment_rejected_on_device():
     with pytest.raises(zr.ZrError) as e:
         zr.zr_step(gr.plan.handle, gr.grads, gr.master.data_ptr() + 4, gr.m, gr.v, out, 1)
     assert e.value.status == zr.ZR_ERR_ALIGNMENT
+
+
+@pytest.mark.parametrize("shapes, W, rank, mode, max_norm", [
+    (synth.gpt2_small_shapes()[:30], 8, 1, 0, 0.0),               # flat, many chunks
+    ([(4096 * 3 + 5,), (17,), (1,), (300, 7)], 3, 2, 0, 0.0),     # ragged tiles, pad
+    ([(1000, 3), (8191,), (9, 9), (2048,)], 4, 1, 1, 0.05),       # whole-tensor, clip, re-read
+    ([(3000, 7), (5001,), (64, 64), (129,)], 8, 3, 0, 0.05),      # clip with g scratch
+])
+def test_step_host_matches_step(shapes, W, rank, mode, max_norm):
+    """zr_step_host (gradients from pinned host memory, chunked copy-in /
+    step / copy-out pipeline) gives zr_step's results bit for bit."""
+    hp = (3e-4, 0.9, 0.999, 1e-8, 0.1, max_norm)
+    ref = GpuRank(shapes, W, rank, mode, 4096, hp, seed=31)
+    pipe = GpuRank(shapes, W, rank, mode, 4096, hp, seed=31)
+    n = ref.plan.owned_numel
+    P = ref.plan.padded_numel
+    out_ref = torch.zeros(P, dtype=torch.bfloat16, device=DEV)
+    out_dev = torch.zeros(P, dtype=torch.bfloat16, device=DEV)
+    host_out = torch.full((P,), -1, dtype=torch.int16).pin_memory()
+    dev_grads = [torch.zeros(max(n, 8), dtype=torch.bfloat16, device=DEV) for _ in range(W)]
+    others = torch.tensor([0.5] * W, dtype=torch.float64, device=DEV)
+    for t in (1, 2):
+        ref.fill_grads(t, 1e-2, 0.01)
+        host_grads = [g.cpu().pin_memory() for g in ref.grads]
+        if max_norm > 0:
+            ref.plan.partials.copy_(others)
+            pipe.plan.partials.copy_(others)
+        ref.step(out_ref, t)
+        pipe.plan.step_host(host_grads, dev_grads, pipe.master, pipe.m, pipe.v, out_dev,
+                            host_out.view(torch.bfloat16), t)
+        torch.cuda.synchronize()
+        for a, b, what in zip(ref.state(), pipe.state(), ("master", "m", "v")):
+            assert np.array_equal(bits32(a), bits32(b)), f"{what} step {t}"
+        for w in range(W):
+            assert torch.equal(dev_grads[w][:n].view(torch.int16), ref.grads[w][:n].view(torch.int16))
+        assert torch.equal(out_ref.view(torch.int16), out_dev.view(torch.int16))
+        oplan = oracle.Plan(shapes, W, mode, 4096)
+        mine = oplan.owned_global_index(rank)
+        assert np.array_equal(host_out.numpy()[mine], out_ref.view(torch.int16).cpu().numpy()[mine])
+        rest = np.ones(P, dtype=bool)
+        rest[mine] = False
+        assert np.all(host_out.numpy()[rest] == -1)
