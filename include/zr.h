@@ -81,7 +81,9 @@ typedef enum {
     ZR_ERR_NO_WORKSPACE = 3,  /* zr_plan_set_workspace not called / too small */
     ZR_ERR_CUDA = 4,          /* a CUDA runtime call failed                  */
     ZR_ERR_UNSUPPORTED = 5,   /* W above ZR_MAX_WORLD_SIZE, no sm_100 device */
-    ZR_ERR_BUFFER_TOO_SMALL = 6
+    ZR_ERR_BUFFER_TOO_SMALL = 6,
+    ZR_ERR_IO = 7,            /* a checkpoint file could not be read or written */
+    ZR_ERR_MISMATCH = 8       /* a checkpoint does not belong to this plan, or is corrupt */
 } zr_status;
 
 typedef enum { ZR_PARTITION_FLAT = 0, ZR_PARTITION_WHOLE_TENSOR = 1 } zr_partition;
@@ -231,6 +233,40 @@ zr_status zr_grad_sumsq(const zr_plan* plan, const void* const* grad_ptrs, doubl
  * floats, 16-byte aligned). */
 zr_status zr_debug_reduce(const zr_plan* plan, const void* const* grad_ptrs, float* g_out,
                           zr_stream_t stream);
+
+/* Checkpoints of the sharded optimizer state ("DDP -> ZeRO -> TP/PP/CP"
+ * blog, section 3.3: sharded state must be gathered to be saved as a whole
+ * model).  One file per rank: a 256-byte header -- magic "ZRSHARD1",
+ * version 1, W, rank, mode, element counts, a hash of the tensors and one of
+ * the partition (tensors, W, mode), the step, the AdamW hyperparameters and
+ * a 64-bit FNV-1a checksum of the payload -- then master, m and v (fp32,
+ * owned order).  The bf16 parameters need no checkpoint of their own: after
+ * a step the all-gather buffer param_out already holds them whole.
+ *
+ * zr_state_save: copies this rank's master, m, v (device, owned_numel fp32
+ * each) to the host after the work queued on `stream` (it synchronises the
+ * stream) and writes them with `step` to `path` (through a temporary file
+ * renamed into place).  zr_state_load: reads `path`, checks that it belongs
+ * to this plan's partition and rank and that its checksum holds, copies the
+ * state to the device (synchronising `stream`) and returns the saved step in
+ * *step (may be NULL).  Both allocate host memory for one shard.
+ * Errors: ZR_ERR_IO (file), ZR_ERR_MISMATCH (another partition or rank, or a
+ * corrupt file), ZR_ERR_CUDA, ZR_ERR_INVALID_ARG. */
+zr_status zr_state_save(const zr_plan* plan, const char* path, const float* master, const float* m,
+                        const float* v, int64_t step, zr_stream_t stream);
+zr_status zr_state_load(const zr_plan* plan, const char* path, float* master, float* m, float* v,
+                        int64_t* step, zr_stream_t stream);
+
+/* Elastic resume: writes to dst_path the shard of `target`'s rank under
+ * `target`'s partition, built from src_paths[0..n_src), the complete set of
+ * shards (rank r at index r) that another partition of the same tensors
+ * saved (any W, either mode, same step).  Host only; reads each source
+ * shard whole once.  A target with W = 1 and the flat mode yields the whole
+ * fp32 state in declaration order.  Errors: ZR_ERR_IO, ZR_ERR_MISMATCH
+ * (shards of other tensors, missing or out-of-order ranks, different steps,
+ * corrupt payloads), ZR_ERR_INVALID_ARG. */
+zr_status zr_state_reshard(const zr_plan* target, const char* const* src_paths, int32_t n_src,
+                           const char* dst_path);
 
 /* Size of the library-owned scratch array used by zr_step_no_alloc. */
 #define ZR_NO_ALLOC_SCRATCH_BYTES (4u << 20)

@@ -32,6 +32,8 @@ ZR_ERR_NO_WORKSPACE = 3
 ZR_ERR_CUDA = 4
 ZR_ERR_UNSUPPORTED = 5
 ZR_ERR_BUFFER_TOO_SMALL = 6
+ZR_ERR_IO = 7
+ZR_ERR_MISMATCH = 8
 ZR_PARTITION_FLAT = 0
 ZR_PARTITION_WHOLE_TENSOR = 1
 ZR_MAX_WORLD_SIZE = 512
@@ -40,7 +42,8 @@ EXPORTED = [
     "zr_plan_create", "zr_plan_query", "zr_plan_segments", "zr_plan_workspace_bytes",
     "zr_plan_set_workspace", "zr_plan_set_sumsq_partials", "zr_step", "zr_step_bucket",
     "zr_step_finish", "zr_step_host",
-    "zr_grad_sumsq", "zr_debug_reduce", "zr_step_no_alloc", "zr_plan_destroy", "zr_status_string",
+    "zr_grad_sumsq", "zr_debug_reduce", "zr_step_no_alloc", "zr_state_save", "zr_state_load",
+    "zr_state_reshard", "zr_plan_destroy", "zr_status_string",
 ]
 ZR_NO_ALLOC_SCRATCH_BYTES = 4 << 20
 
@@ -72,6 +75,9 @@ _lib.zr_step_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_grad_sumsq.argtypes = [_vp, _vp, _vp, _vp]
 _lib.zr_debug_reduce.argtypes = [_vp, _vp, _vp, _vp]
 _lib.zr_step_no_alloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
+_lib.zr_state_save.argtypes = [_vp, ctypes.c_char_p, _vp, _vp, _vp, _i64, _vp]
+_lib.zr_state_load.argtypes = [_vp, ctypes.c_char_p, _vp, _vp, _vp, _P(_i64), _vp]
+_lib.zr_state_reshard.argtypes = [_vp, _vp, _i32, ctypes.c_char_p]
 _lib.zr_plan_destroy.argtypes = [_vp]
 _lib.zr_plan_destroy.restype = None
 _lib.zr_status_string.argtypes = [ctypes.c_int]
@@ -224,6 +230,25 @@ def zr_step_no_alloc(plan: int, grads, master, m, v, param_out, sumsq_partials, 
                           f"the library's {ZR_NO_ALLOC_SCRATCH_BYTES} byte static scratch on a "
                           "compute capability 10.x device; use zr_step with a workspace)")
     _check(st, "zr_step_no_alloc")
+
+
+def zr_state_save(plan: int, path: str, master, m, v, step: int, stream=None) -> None:
+    _check(_lib.zr_state_save(plan, os.fsencode(path), _addr(master), _addr(m), _addr(v), int(step),
+                              _stream(stream)), "zr_state_save")
+
+
+def zr_state_load(plan: int, path: str, master, m, v, stream=None) -> int:
+    """Loads the shard into master/m/v and returns its step."""
+    step = _i64()
+    _check(_lib.zr_state_load(plan, os.fsencode(path), _addr(master), _addr(m), _addr(v),
+                              ctypes.byref(step), _stream(stream)), "zr_state_load")
+    return step.value
+
+
+def zr_state_reshard(target_plan: int, src_paths, dst_path: str) -> None:
+    arr = (ctypes.c_char_p * max(1, len(src_paths)))(*[os.fsencode(p) for p in src_paths])
+    _check(_lib.zr_state_reshard(target_plan, arr, len(src_paths), os.fsencode(dst_path)),
+           "zr_state_reshard")
 
 
 def raw_call(name: str, *args) -> int:

@@ -67,6 +67,8 @@ const char* zr_status_string(zr_status s) {
         case ZR_ERR_CUDA: return "ZR_ERR_CUDA: a CUDA runtime call failed";
         case ZR_ERR_UNSUPPORTED: return "ZR_ERR_UNSUPPORTED: unsupported configuration or device";
         case ZR_ERR_BUFFER_TOO_SMALL: return "ZR_ERR_BUFFER_TOO_SMALL: output array too small";
+        case ZR_ERR_IO: return "ZR_ERR_IO: checkpoint file could not be read or written";
+        case ZR_ERR_MISMATCH: return "ZR_ERR_MISMATCH: checkpoint of another partition, rank or step, or corrupt";
     }
     return "unknown zr_status";
 }
