@@ -64,10 +64,13 @@ def host_global_sumsq(oplan, wl, step, threads):
     return S, parts
 
 
-@pytest.mark.parametrize("name", ["gpt2_124m_w8", "llama_7b_w64", "gpt_1p3b_w8_whole_clip"])
-def test_full_size_sampled(name):
+@pytest.mark.parametrize("name, rank", [("gpt2_124m_w8", None), ("llama_7b_w64", None),
+                                        ("llama_7b_w64", 63),   # parameter offsets beyond 2**32
+                                        ("gpt_1p3b_w8_whole_clip", None)])
+def test_full_size_sampled(name, rank):
     wl = synth.WORKLOADS[name]
-    rank, W = wl.ranks[0], wl.world_size
+    rank = wl.ranks[0] if rank is None else rank
+    W = wl.world_size
     clip = wl.max_grad_norm > 0
     plan = ZrPlan(wl.shapes, W, rank, wl.mode, wl.bucket_cap_bytes, *wl.hp, device=DEV)
     n = plan.owned_numel

@@ -98,6 +98,12 @@ def test_edge_shapes(shapes, W, mode, cap):
     run_all_ranks(shapes, W, mode, cap, 2, 1e-3, 0.01)
 
 
+def test_max_world_size():
+    """W = 512, the ABI's maximum (the pointer array's largest instantiation):
+    first, middle and last rank."""
+    run_all_ranks([(512 * 40 + 3,), (100,)], 512, 0, 1 << 20, 2, 1e-3, 0.01, ranks=[0, 255, 511])
+
+
 def test_special_values():
     """±0, subnormals, huge values, inf and NaN in the replicas."""
     shapes = [(4096 + 24,)]
