@@ -234,6 +234,57 @@ zr_status zr_grad_sumsq(const zr_plan* plan, const void* const* grad_ptrs, doubl
 zr_status zr_debug_reduce(const zr_plan* plan, const void* const* grad_ptrs, float* g_out,
                           zr_stream_t stream);
 
+/* ---------------------------------------------------------------------
+ * ZeRO across GPUs over peer memory (NVLink / NVSwitch), one process per GPU
+ * ("CS336 lecture 8", ZeRO-1 sketch: reduce-scatter of the gradients, update
+ * of the owned slice, all-gather of the updated parameters).  The same
+ * fused kernel does all three: grad_ptrs may point into other GPUs' memory
+ * (peer loads are the reduce-scatter), and with gather targets set, every
+ * bf16 result is stored into every rank's parameter buffer (peer stores are
+ * the all-gather).  Ordering between ranks is the caller's: every replica's
+ * gradients must be complete before any rank's step starts, and no rank may
+ * read its parameter buffer before every rank's step has completed (for
+ * example: synchronise the stream, then a process-group barrier, on both
+ * sides).  Nothing in the kernels waits on another GPU.
+ * ------------------------------------------------------------------- */
+
+/* Owner-major layout of a full gradient buffer: rank r's owned elements, in
+ * its owned order, start at offsets[r]; each rank's region is rounded up to
+ * a multiple of 8 elements so that every region starts 16-byte aligned;
+ * offsets[W] is the buffer's length in elements.  (In the flat mode with a
+ * chunk that is a multiple of 8 this is exactly the global layout.)  When
+ * every replica keeps its full gradient in this layout, the pointer to
+ * replica w's buffer plus offsets[r] elements is what rank r passes as
+ * grad_ptrs[w].  offsets: world_size + 1 entries. */
+zr_status zr_plan_owner_offsets(const zr_plan* plan, int64_t* offsets);
+
+/* Make zr_step, zr_step_bucket and zr_step_finish store each bf16 result in
+ * targets[0..world_size) (rank w's parameter buffer, global layout, local
+ * or peer-mapped, 16-byte aligned) instead of param_out, which may then be
+ * NULL.  The pointer array is copied into the workspace (synchronising
+ * `stream`); targets == NULL goes back to param_out.  zr_step_host refuses a
+ * plan with gather targets (ZR_ERR_UNSUPPORTED).  Needs a bound workspace. */
+zr_status zr_plan_set_gather_targets(zr_plan* plan, void* const* targets, zr_stream_t stream);
+
+/* A device buffer as another process can map it: the CUDA IPC handle of the
+ * allocation that holds it and the buffer's offset in that allocation. */
+typedef struct {
+    unsigned char handle[64];
+    uint64_t offset;
+    uint64_t allocation_bytes;
+} zr_ipc_handle;
+
+/* zr_ipc_export: describe device_ptr (any address inside a cudaMalloc
+ * allocation of this process) for another process.  zr_ipc_open: map a
+ * handle exported by another process (same or other GPU; peer access is
+ * enabled as needed) and return the buffer's address; release it with
+ * zr_ipc_close.  A process cannot open its own handles (use the pointer).
+ * Errors: ZR_ERR_INVALID_ARG, ZR_ERR_CUDA (no GPU driver, memory that IPC
+ * cannot share such as virtual-memory-management allocations). */
+zr_status zr_ipc_export(const void* device_ptr, zr_ipc_handle* out);
+zr_status zr_ipc_open(const zr_ipc_handle* handle, void** device_ptr);
+zr_status zr_ipc_close(void* device_ptr);
+
 /* Checkpoints of the sharded optimizer state ("DDP -> ZeRO -> TP/PP/CP"
  * blog, section 3.3: sharded state must be gathered to be saved as a whole
  * model).  One file per rank: a 256-byte header -- magic "ZRSHARD1",

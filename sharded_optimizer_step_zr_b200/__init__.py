@@ -43,7 +43,8 @@ EXPORTED = [
     "zr_plan_set_workspace", "zr_plan_set_sumsq_partials", "zr_step", "zr_step_bucket",
     "zr_step_finish", "zr_step_host",
     "zr_grad_sumsq", "zr_debug_reduce", "zr_step_no_alloc", "zr_state_save", "zr_state_load",
-    "zr_state_reshard", "zr_plan_destroy", "zr_status_string",
+    "zr_state_reshard", "zr_plan_owner_offsets", "zr_plan_set_gather_targets", "zr_ipc_export",
+    "zr_ipc_open", "zr_ipc_close", "zr_plan_destroy", "zr_status_string",
 ]
 ZR_NO_ALLOC_SCRATCH_BYTES = 4 << 20
 
@@ -58,6 +59,11 @@ class zr_segment(ctypes.Structure):
                 ("reserved", ctypes.c_int32), ("offset_in_tensor", ctypes.c_int64),
                 ("length", ctypes.c_int64), ("global_offset", ctypes.c_int64),
                 ("owned_offset", ctypes.c_int64)]
+
+
+class zr_ipc_handle(ctypes.Structure):
+    _fields_ = [("handle", ctypes.c_ubyte * 64), ("offset", ctypes.c_uint64),
+                ("allocation_bytes", ctypes.c_uint64)]
 
 
 _vp, _i32, _i64, _u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64
@@ -78,6 +84,11 @@ _lib.zr_step_no_alloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_state_save.argtypes = [_vp, ctypes.c_char_p, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_state_load.argtypes = [_vp, ctypes.c_char_p, _vp, _vp, _vp, _P(_i64), _vp]
 _lib.zr_state_reshard.argtypes = [_vp, _vp, _i32, ctypes.c_char_p]
+_lib.zr_plan_owner_offsets.argtypes = [_vp, _vp]
+_lib.zr_plan_set_gather_targets.argtypes = [_vp, _vp, _vp]
+_lib.zr_ipc_export.argtypes = [_vp, _P(zr_ipc_handle)]
+_lib.zr_ipc_open.argtypes = [_P(zr_ipc_handle), _P(_vp)]
+_lib.zr_ipc_close.argtypes = [_vp]
 _lib.zr_plan_destroy.argtypes = [_vp]
 _lib.zr_plan_destroy.restype = None
 _lib.zr_status_string.argtypes = [ctypes.c_int]
@@ -249,6 +260,35 @@ def zr_state_reshard(target_plan: int, src_paths, dst_path: str) -> None:
     arr = (ctypes.c_char_p * max(1, len(src_paths)))(*[os.fsencode(p) for p in src_paths])
     _check(_lib.zr_state_reshard(target_plan, arr, len(src_paths), os.fsencode(dst_path)),
            "zr_state_reshard")
+
+
+def zr_plan_owner_offsets(plan: int, world_size: int):
+    arr = (ctypes.c_int64 * (world_size + 1))()
+    _check(_lib.zr_plan_owner_offsets(plan, arr), "zr_plan_owner_offsets")
+    return list(arr)
+
+
+def zr_plan_set_gather_targets(plan: int, targets, stream=None) -> None:
+    arr = _ptr_array(targets) if targets is not None else None
+    _check(_lib.zr_plan_set_gather_targets(plan, arr, _stream(stream)), "zr_plan_set_gather_targets")
+
+
+def zr_ipc_export(buffer) -> bytes:
+    """The handle of a device buffer (tensor or address) as bytes."""
+    h = zr_ipc_handle()
+    _check(_lib.zr_ipc_export(_addr(buffer), ctypes.byref(h)), "zr_ipc_export")
+    return bytes(h)
+
+
+def zr_ipc_open(handle: bytes) -> int:
+    h = zr_ipc_handle.from_buffer_copy(handle)
+    out = ctypes.c_void_p()
+    _check(_lib.zr_ipc_open(ctypes.byref(h), ctypes.byref(out)), "zr_ipc_open")
+    return out.value
+
+
+def zr_ipc_close(address: int) -> None:
+    _check(_lib.zr_ipc_close(address), "zr_ipc_close")
 
 
 def raw_call(name: str, *args) -> int:

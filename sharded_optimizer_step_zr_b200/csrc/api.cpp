@@ -34,7 +34,23 @@ zr::LaunchArgs base_args(const zr_plan* p) {
     const bool pow2 = (p->world_size & (p->world_size - 1)) == 0;
     a.w_is_pow2 = pow2 ? 1 : 0;
     a.inv_w = pow2 ? 1.0f / static_cast<float>(p->world_size) : 0.0f;
+    a.n_targets = p->n_gather_targets;
+    a.targets = p->d_gather_targets;
     return a;
+}
+
+// The bf16 destination: param_out, or the plan's gather targets (then
+// param_out may be NULL).
+zr_status check_param_out(const zr_plan* p, const void* param_out) {
+    if (p->n_gather_targets > 0) return (param_out && !aligned16(param_out)) ? ZR_ERR_ALIGNMENT : ZR_OK;
+    if (!param_out) return ZR_ERR_INVALID_ARG;
+    return aligned16(param_out) ? ZR_OK : ZR_ERR_ALIGNMENT;
+}
+
+zr_status check_state(const float* master, const float* m, const float* v) {
+    if (!master || !m || !v) return ZR_ERR_INVALID_ARG;
+    if (!aligned16(master) || !aligned16(m) || !aligned16(v)) return ZR_ERR_ALIGNMENT;
+    return ZR_OK;
 }
 
 zr_status ensure_host_pipeline(const zr_plan* p) {
@@ -155,6 +171,8 @@ zr_status zr_plan_set_workspace(zr_plan* p, void* d_ws, uint64_t bytes, zr_strea
     p->d_tile_partials = p->clip_enabled() ? reinterpret_cast<double*>(base + L.tile_partials) : nullptr;
     p->d_clip_coef = reinterpret_cast<float*>(base + L.clip_coef);
     p->d_own_sumsq = reinterpret_cast<double*>(base + L.own_sumsq);
+    p->d_gather_targets = reinterpret_cast<uint16_t**>(base + L.gather_targets);
+    p->n_gather_targets = 0;
     p->d_g_scratch = p->clip_uses_scratch() ? reinterpret_cast<float*>(base + L.g_scratch) : nullptr;
     if (!p->tiles.empty()) {
         const size_t bytes_tiles = sizeof(zr::Tile) * p->tiles.size();
@@ -174,6 +192,38 @@ zr_status zr_plan_set_sumsq_partials(zr_plan* p, double* d_partials) {
     return ZR_OK;
 }
 
+zr_status zr_plan_owner_offsets(const zr_plan* p, int64_t* offsets) {
+    if (!p || !offsets) return ZR_ERR_INVALID_ARG;
+    // Each rank's region starts on a 16-byte boundary (8 bf16 elements), as
+    // the step's vector loads need.
+    int64_t at = 0;
+    for (int32_t r = 0; r < p->world_size; ++r) {
+        offsets[r] = at;
+        at += (p->rank_numel[r] + 7) / 8 * 8;
+    }
+    offsets[p->world_size] = at;
+    return ZR_OK;
+}
+
+zr_status zr_plan_set_gather_targets(zr_plan* p, void* const* targets, zr_stream_t stream) {
+    if (!p) return ZR_ERR_INVALID_ARG;
+    if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
+    if (!targets) {
+        p->n_gather_targets = 0;
+        return ZR_OK;
+    }
+    for (int32_t w = 0; w < p->world_size; ++w) {
+        if (!targets[w]) return ZR_ERR_INVALID_ARG;
+        if (!aligned16(targets[w])) return ZR_ERR_ALIGNMENT;
+    }
+    if (cudaMemcpyAsync(p->d_gather_targets, targets, sizeof(void*) * p->world_size, cudaMemcpyHostToDevice,
+                        reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess ||
+        cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return ZR_ERR_CUDA;
+    p->n_gather_targets = p->world_size;
+    return ZR_OK;
+}
+
 zr_status zr_step(const zr_plan* p, const void* const* grad_ptrs, float* master, float* m, float* v,
                   void* param_out, int64_t step, zr_stream_t stream) {
     if (!p || step < 1) return ZR_ERR_INVALID_ARG;
@@ -181,8 +231,7 @@ zr_status zr_step(const zr_plan* p, const void* const* grad_ptrs, float* master,
     if (p->owned_numel() == 0) return ZR_OK;
     zr_status st = check_grads(p, grad_ptrs);
     if (st != ZR_OK) return st;
-    if (!master || !m || !v || !param_out) return ZR_ERR_INVALID_ARG;
-    if (!aligned16(master) || !aligned16(m) || !aligned16(v) || !aligned16(param_out)) return ZR_ERR_ALIGNMENT;
+    if ((st = check_state(master, m, v)) != ZR_OK || (st = check_param_out(p, param_out)) != ZR_OK) return st;
     if (p->clip_enabled() && !p->d_sumsq_partials) return ZR_ERR_NO_WORKSPACE;
 
     zr::LaunchArgs a = base_args(p);
@@ -229,8 +278,7 @@ zr_status zr_step_bucket(const zr_plan* p, int32_t bucket, const void* const* gr
     a.n_tiles = count;
     void* s = stream;
     if (!p->clip_enabled()) {
-        if (!master || !m || !v || !param_out) return ZR_ERR_INVALID_ARG;
-        if (!aligned16(master) || !aligned16(m) || !aligned16(v) || !aligned16(param_out)) return ZR_ERR_ALIGNMENT;
+        if ((st = check_state(master, m, v)) != ZR_OK || (st = check_param_out(p, param_out)) != ZR_OK) return st;
         a.master = master;
         a.m = m;
         a.v = v;
@@ -259,8 +307,8 @@ zr_status zr_step_finish(const zr_plan* p, const void* const* grad_ptrs, float* 
     } else {
         grad_ptrs = nullptr;                         // pass 2 reads the g scratch only
     }
-    if (!master || !m || !v || !param_out) return ZR_ERR_INVALID_ARG;
-    if (!aligned16(master) || !aligned16(m) || !aligned16(v) || !aligned16(param_out)) return ZR_ERR_ALIGNMENT;
+    zr_status st2 = check_state(master, m, v);
+    if (st2 != ZR_OK || (st2 = check_param_out(p, param_out)) != ZR_OK) return st2;
     zr::LaunchArgs a = base_args(p);
     a.master = master;
     a.m = m;
@@ -316,6 +364,7 @@ zr_status zr_step_host(const zr_plan* p, const void* const* host_grad_ptrs, void
                        int64_t step, zr_stream_t stream) {
     if (!p || !host_grad_ptrs || !dev_grad_ptrs || !host_param_out || step < 1) return ZR_ERR_INVALID_ARG;
     if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
+    if (p->n_gather_targets > 0) return ZR_ERR_UNSUPPORTED;   // copies back this rank's buffer only
     const int64_t n = p->owned_numel();
     if (n == 0) return ZR_OK;
     for (int32_t w = 0; w < p->world_size; ++w)

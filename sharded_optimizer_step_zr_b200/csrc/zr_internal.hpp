@@ -56,6 +56,9 @@ struct LaunchArgs {
     int32_t w_is_pow2;
     float inv_w;               // 1/W when W is a power of two (exact)
     int32_t reverse;           // CTA b takes tile n_tiles - 1 - b (see the clip pass 2)
+    int32_t n_targets;         // 0: bf16 results to param_out; else to each of targets[0..n)
+    uint16_t* const* targets;  // device array of parameter buffers (every rank's, for the
+                               // all-gather by peer stores)
     float* master;
     float* m;
     float* v;
@@ -111,6 +114,8 @@ struct zr_plan {
     double* d_own_sumsq = nullptr;
     float* d_g_scratch = nullptr;
     double* d_sumsq_partials = nullptr;   // caller-owned, world_size doubles
+    uint16_t** d_gather_targets = nullptr; // workspace: world_size parameter buffers
+    int32_t n_gather_targets = 0;          // 0 until zr_plan_set_gather_targets
 
     // zr_step_host's copy streams and events, created on its first call
     // (host-side resources, not part of the plan's observable state).
@@ -133,7 +138,7 @@ zr_status build_plan(zr_plan& p, int32_t n_tensors, const int32_t* ndims,
                      const int64_t* const* shapes);
 // Workspace layout: offsets of each region, total bytes.
 struct WorkspaceLayout {
-    uint64_t tiles, tiles_by_owned, tile_partials, clip_coef, own_sumsq, g_scratch, total;
+    uint64_t tiles, tiles_by_owned, tile_partials, clip_coef, own_sumsq, gather_targets, g_scratch, total;
 };
 WorkspaceLayout workspace_layout(const zr_plan& p);
 AdamScalars adam_scalars(const zr_adamw& hp, int64_t step);

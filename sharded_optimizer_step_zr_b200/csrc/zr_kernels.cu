@@ -101,6 +101,25 @@ __device__ __forceinline__ void adamw(const AdamScalars& c, float g, float& p, f
     v = v_new;
 }
 
+// The bf16 results go to this rank's parameter buffer, or, when the plan has
+// gather targets, to every rank's: the all-gather done by peer stores in the
+// same pass that computes the values.
+__device__ __forceinline__ void store_params8(const LaunchArgs& a, int64_t go, uint4 q) {
+    if (a.n_targets == 0) {
+        __stcs(reinterpret_cast<uint4*>(a.param_out + go), q);
+        return;
+    }
+    for (int d = 0; d < a.n_targets; ++d) __stcs(reinterpret_cast<uint4*>(a.targets[d] + go), q);
+}
+
+__device__ __forceinline__ void store_param1(const LaunchArgs& a, int64_t go, uint16_t u) {
+    if (a.n_targets == 0) {
+        a.param_out[go] = u;
+        return;
+    }
+    for (int d = 0; d < a.n_targets; ++d) a.targets[d][go] = u;
+}
+
 // Left fold of W replicas for 8 consecutive owned elements at `off`.  The
 // loads of one group of G replicas are all issued before the first add.
 template <int CAP, int G>
@@ -229,14 +248,14 @@ zr_tile_kernel(const GradPtrs<CAP> gp, const LaunchArgs a) {
                     q.y = pack_bf16x2(p[2], p[3]);
                     q.z = pack_bf16x2(p[4], p[5]);
                     q.w = pack_bf16x2(p[6], p[7]);
-                    __stcs(reinterpret_cast<uint4*>(a.param_out + go), q);
+                    store_params8(a, go, q);
                 } else {
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         __nv_bfloat16 h = __float2bfloat16_rn(p[k]);
                         uint16_t u;
                         memcpy(&u, &h, 2);
-                        a.param_out[go + k] = u;
+                        store_param1(a, go + k, u);
                     }
                 }
             }
@@ -260,7 +279,7 @@ zr_tile_kernel(const GradPtrs<CAP> gp, const LaunchArgs a) {
                 __nv_bfloat16 h = __float2bfloat16_rn(p);
                 uint16_t u;
                 memcpy(&u, &h, 2);
-                a.param_out[tile.global + e] = u;
+                store_param1(a, tile.global + e, u);
             }
         }
     }

@@ -1,0 +1,111 @@
+"""PeerZero: one rank of a ZeRO-1/2 job across GPUs, one process per GPU.
+
+The fused step reads this rank's owned slice of every replica's gradient
+buffer through peer loads (the reduce-scatter) and stores each updated bf16
+parameter into every rank's parameter buffer through peer stores (the
+all-gather) -- over NVLink / NVSwitch on a multi-GPU node.  Buffers are
+shared between the processes with CUDA IPC; torch.distributed carries the
+handles, the barriers around the step and, with clipping, the exchange of
+the per-rank sums of squares.
+
+Every replica keeps its full gradient in the plan's owner-major layout
+(``grad_view(t)`` is tensor t's slice of it, for the backward pass to write
+into); ``param_buffer`` holds the full bf16 parameters in the global layout.
+"""
+from __future__ import annotations
+
+from . import (ZR_PARTITION_FLAT, zr_ipc_close, zr_ipc_export, zr_ipc_open, zr_plan_owner_offsets,
+               zr_plan_set_gather_targets, zr_step)
+from .plan import ZrPlan
+
+
+class PeerZero:
+    def __init__(self, group, shapes, mode=ZR_PARTITION_FLAT, bucket_cap_bytes=25 << 20, lr=3e-4,
+                 beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.1, max_grad_norm=0.0, device=None):
+        import torch
+        import torch.distributed as dist
+        self.dist, self.group = dist, group
+        self.world_size = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+        self.device = device
+        self.plan = ZrPlan(shapes, self.world_size, self.rank, mode, bucket_cap_bytes, lr, beta1, beta2,
+                           eps, weight_decay, max_grad_norm, device=device)
+        self.offsets = zr_plan_owner_offsets(self.plan.handle, self.world_size)
+        P = self.plan.padded_numel
+        # One allocation holds both shared buffers, so each peer maps one
+        # IPC handle per rank: the gradient buffer, then (256-byte aligned)
+        # the parameter buffer.
+        half = max(128, (max(P, self.offsets[-1]) + 127) // 128 * 128)
+        self._shared = torch.zeros(2 * half, dtype=torch.bfloat16, device=device)
+        self.grad_buffer = self._shared[:half]
+        self.param_buffer = self._shared[half:]
+        everyone = [None] * self.world_size
+        dist.all_gather_object(everyone, zr_ipc_export(self._shared), group=group)
+        self._opened = []
+        grad_bases, param_bases = [], []
+        for w, handle in enumerate(everyone):
+            base = self._shared.data_ptr() if w == self.rank else zr_ipc_open(handle)
+            if w != self.rank:
+                self._opened.append(base)
+            grad_bases.append(base)
+            param_bases.append(base + 2 * half)
+        start = 2 * self.offsets[self.rank]                 # bytes: bf16 elements
+        self.grad_ptrs = [b + start for b in grad_bases]
+        zr_plan_set_gather_targets(self.plan.handle, param_bases)
+        self._segments = self.plan.segments()
+        dist.barrier(group)
+
+    def grad_pieces(self, tensor_index):
+        """[(offset in the tensor, view of the owner-major buffer)] of tensor
+        `tensor_index`'s gradient, one piece per owner."""
+        pieces = sorted((s["offset_in_tensor"], s["owner"], s["owned_offset"], s["length"])
+                        for s in self._segments if s["tensor"] == tensor_index)
+        return [(off, self.grad_buffer[self.offsets[r] + o: self.offsets[r] + o + n])
+                for off, r, o, n in pieces]
+
+    def grad_view(self, tensor_index, shape=None):
+        """Tensor `tensor_index`'s gradient as one view of the owner-major
+        buffer: always possible for whole-tensor ownership, and for flat
+        partitions whose chunk is a multiple of 8 elements."""
+        pieces = self.grad_pieces(tensor_index)
+        start = pieces[0][1].data_ptr()
+        n = 0
+        for _, view in pieces:
+            if view.data_ptr() != start + 2 * n:
+                raise ValueError("tensor is split across rank regions; use grad_pieces()")
+            n += view.numel()
+        v = self.grad_buffer[(start - self.grad_buffer.data_ptr()) // 2:][:n]
+        return v.view(shape) if shape is not None else v
+
+    def _exchange_sumsq(self):
+        import torch
+        dist = self.dist
+        part = self.plan.partials
+        self.plan.grad_sumsq(self.grad_ptrs, part[self.rank:self.rank + 1])
+        backend = dist.get_backend(self.group)
+        mine = part[self.rank:self.rank + 1].clone()
+        if backend != "nccl":
+            mine = mine.cpu()
+        gathered = [torch.empty_like(mine) for _ in range(self.world_size)]
+        dist.all_gather(gathered, mine, group=self.group)
+        part.copy_(torch.cat(gathered).to(part.device))
+
+    def step(self, master, m, v, step):
+        """One optimizer step of this rank (every rank calls it together)."""
+        import torch
+        torch.cuda.current_stream().synchronize()      # this replica's gradients are written
+        self.dist.barrier(self.group)                  # ... and every other replica's
+        if self.plan.max_grad_norm > 0:
+            self._exchange_sumsq()
+        zr_step(self.plan.handle, self.grad_ptrs, master, m, v, None, step)
+        torch.cuda.current_stream().synchronize()
+        self.dist.barrier(self.group)                  # every slice is in every parameter buffer
+
+    def close(self):
+        if self._opened:
+            self.dist.barrier(self.group)
+            for addr in self._opened:
+                zr_ipc_close(addr)
+            self._opened = []
+        self.plan.close()

@@ -1,0 +1,104 @@
+"""ZeRO across processes over shared device memory (CUDA IPC), on the one
+GPU this suite has: two processes, one rank each.  Each rank's fused step
+reads its slice of both replicas' gradient buffers through IPC mappings (the
+reduce-scatter) and stores its bf16 results into both ranks' parameter
+buffers (the all-gather); barriers on the host order the phases, and no
+kernel waits on the other process.  Results must equal the oracle's: the
+rank's fp32 state bit for bit, and both full parameter buffers bit for bit
+against the unsharded step."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+pytestmark = pytest.mark.gpu
+
+
+def _port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, shapes, mode, max_norm, q):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import torch
+    import torch.distributed as dist
+    import oracle
+    import synth
+    from sharded_optimizer_step_zr_b200.peer import PeerZero
+    import datetime
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=90))
+    try:
+        hp = (3e-4, 0.9, 0.999, 1e-8, 0.1, max_norm)
+        pz = PeerZero(dist.group.WORLD, shapes, mode, 4096, *hp)
+        segs = pz.plan.segments()
+        N, P = pz.plan.total_numel, pz.plan.padded_numel
+        runs_of = [synth.rank_runs(segs, r) for r in range(world)]
+        n = pz.plan.owned_numel
+        master = torch.empty(max(n, 8), dtype=torch.float32, device="cuda:0")
+        synth.fill_owned_master(master, runs_of[rank], 4, n_valid=N)
+        m, v = torch.zeros_like(master), torch.zeros_like(master)
+        oplan = oracle.Plan(shapes, world, mode, 4096)
+        idx_all = torch.arange(P, dtype=torch.int64)
+        o_master = synth.master_f32(4, idx_all, n_valid=N).numpy().copy()
+        o_m, o_v = np.zeros(P, np.float32), np.zeros(P, np.float32)
+        o_out = np.zeros(P, np.uint16)
+        for t in (1, 2):
+            # this process is replica `rank`: its full gradient, owner-major
+            for r in range(world):
+                a, b = pz.offsets[r], pz.offsets[r + 1]
+                synth.fill_owned_grad(pz.grad_buffer[a:b], runs_of[r], 4, t, rank, 1e-2, 0.01, n_valid=N)
+            pz.step(master, m, v, t)
+            reps = [synth.grad_bf16(4, t, w, idx_all, 1e-2, 0.01, n_valid=N).view(torch.int16).numpy()
+                    .view(np.uint16).copy() for w in range(world)]
+            c = None
+            if max_norm > 0:
+                c = oracle.clip_coef(oracle.sumsq(oracle.reduce([x[:N] for x in reps])), max_norm)
+            oracle.ddp_step(reps, o_master, o_m, o_v, o_out, hp, t, clip=c)
+        gi = oplan.owned_global_index(rank)
+        same_state = all(np.array_equal(x[:n].cpu().numpy().view(np.uint32), y[gi].view(np.uint32))
+                         for x, y in ((master, o_master), (m, o_m), (v, o_v)))
+        close_state = all(np.allclose(x[:n].cpu().numpy(), y[gi], rtol=2e-6, atol=1e-9)
+                          for x, y in ((master, o_master), (m, o_m), (v, o_v)))
+        got = pz.param_buffer[:P].cpu().view(torch.int16).numpy().view(np.uint16)
+        ulp = int(np.max(np.abs(got.astype(np.int64) - o_out.astype(np.int64)))) if P else 0
+        q.put((rank, bool(same_state), bool(close_state), ulp, bool(np.array_equal(got, o_out))))
+        pz.close()
+    except Exception as e:  # report, do not hang the other rank's barrier forever
+        q.put((rank, "error", repr(e), None, None))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("shapes, mode, max_norm", [
+    ([(300, 7), (1001,), (64, 64), (4099,)], 0, 0.0),
+    ([(300, 7), (1001,), (64, 64), (4099,), (17,)], 1, 0.0),
+    ([(300, 7), (1001,), (64, 64), (4099,)], 0, 0.05),
+])
+def test_two_processes_share_one_gpu(shapes, mode, max_norm):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, shapes, mode, max_norm, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=240) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=60)
+    for r in results:
+        assert r[1] != "error", r
+        rank, same_state, close_state, ulp, same_out = r
+        assert close_state, r
+        assert ulp <= 1, r
+        if max_norm == 0:
+            assert same_state and same_out, r
+    assert all(p.exitcode == 0 for p in procs)
