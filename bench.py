@@ -316,8 +316,11 @@ def run_zr(args):
     v = torch.zeros_like(master)
     param_out = torch.zeros(plan.padded_numel, dtype=torch.bfloat16, device=dev)
     if clip:
-        # other ranks' sums of squares: the emulated scalar all-gather
+        # the scalar exchange of the clip: this rank's S_r, and the other
+        # ranks' entries set to the same value (their gradients have the same
+        # statistics), so the norm has its real magnitude, S ~ W * S_r
         plan.grad_sumsq(grads, plan.partials[zr_rank:zr_rank + 1])
+        plan.partials.fill_(float(plan.partials[zr_rank].item()))
     torch.cuda.synchronize()
 
     step_no = 0
@@ -334,7 +337,7 @@ def run_zr(args):
     K = args.steps
     sampler = ClockSampler(dev.index)
     if dist:
-        dist.barrier()
+        dist.barrier(device_ids=[local])
     torch.cuda.synchronize()
     with sampler:
         t_start = torch.cuda.Event(enable_timing=True)
@@ -346,7 +349,7 @@ def run_zr(args):
         t_end.record(stream)
         torch.cuda.synchronize()
     if dist:
-        dist.barrier()
+        dist.barrier(device_ids=[local])
     local_ms = t_start.elapsed_time(t_end)
     total_ms, owned_total = reduce_timing(dist, local_ms, n * K, dev)
     value = owned_total / (total_ms * 1e-3) / 1e9
@@ -374,7 +377,7 @@ def run_zr(args):
         K2 = max(3, min(K, 50))
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if dist:
-            dist.barrier()
+            dist.barrier(device_ids=[local])
         torch.cuda.synchronize()
         a.record(stream)
         for _ in range(K2):
@@ -393,7 +396,7 @@ def run_zr(args):
         cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
 
     if dist:
-        dist.barrier()
+        dist.barrier(device_ids=[local])
         dist.destroy_process_group()
     if grank != 0:
         return

@@ -170,6 +170,20 @@ zr_status zr_plan_set_sumsq_partials(zr_plan* plan, double* d_partials);
 zr_status zr_step(const zr_plan* plan, const void* const* grad_ptrs, float* master, float* m,
                   float* v, void* param_out, int64_t step, zr_stream_t stream);
 
+/* zr_step for CUDA-graph capture: the step count lives in device memory.
+ * *d_step (int64, device, 8-byte aligned) holds the number of steps already
+ * taken; the call first advances it on the device and computes the AdamW
+ * scalars there (fp64 from the fp32 hyperparameters, rounded once to fp32,
+ * as zr_step does on the host), then runs the step as zr_step(t = new
+ * count).  Nothing in it depends on host values that change from step to
+ * step, so a graph that captured it replays as the next step each time.
+ * Results equal zr_step's (device and host fp64 pow may differ in the last
+ * fp64 place; after the rounding to fp32 the scalars agree except in rare
+ * ties).  Errors: as zr_step. */
+zr_status zr_step_device_count(const zr_plan* plan, const void* const* grad_ptrs, float* master,
+                               float* m, float* v, void* param_out, int64_t* d_step,
+                               zr_stream_t stream);
+
 /* One bucket of the step, for overlapping the optimizer with the backward
  * pass ("Scaling training to thousands of GPUs", 03:41 DP: a bucket's
  * collective starts as soon as backward has produced its gradients;

@@ -40,7 +40,8 @@ ZR_MAX_WORLD_SIZE = 512
 
 EXPORTED = [
     "zr_plan_create", "zr_plan_query", "zr_plan_segments", "zr_plan_workspace_bytes",
-    "zr_plan_set_workspace", "zr_plan_set_sumsq_partials", "zr_step", "zr_step_bucket",
+    "zr_plan_set_workspace", "zr_plan_set_sumsq_partials", "zr_step", "zr_step_device_count",
+    "zr_step_bucket",
     "zr_step_finish", "zr_step_host",
     "zr_grad_sumsq", "zr_debug_reduce", "zr_step_no_alloc", "zr_state_save", "zr_state_load",
     "zr_state_reshard", "zr_plan_owner_offsets", "zr_plan_set_gather_targets", "zr_ipc_export",
@@ -75,6 +76,7 @@ _lib.zr_plan_workspace_bytes.argtypes = [_vp, _P(_u64)]
 _lib.zr_plan_set_workspace.argtypes = [_vp, _vp, _u64, _vp]
 _lib.zr_plan_set_sumsq_partials.argtypes = [_vp, _vp]
 _lib.zr_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
+_lib.zr_step_device_count.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.zr_step_bucket.argtypes = [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_step_finish.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_step_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
@@ -198,6 +200,12 @@ def zr_plan_set_sumsq_partials(plan: int, partials) -> None:
 def zr_step(plan: int, grads, master, m, v, param_out, step: int, stream=None) -> None:
     _check(_lib.zr_step(plan, _ptr_array(grads), _addr(master), _addr(m), _addr(v),
                         _addr(param_out), int(step), _stream(stream)), "zr_step")
+
+
+def zr_step_device_count(plan: int, grads, master, m, v, param_out, d_step, stream=None) -> None:
+    _check(_lib.zr_step_device_count(plan, _ptr_array(grads), _addr(master), _addr(m), _addr(v),
+                                     _addr(param_out), _addr(d_step), _stream(stream)),
+           "zr_step_device_count")
 
 
 def zr_step_bucket(plan: int, bucket: int, grads, master, m, v, param_out, step: int,

@@ -172,6 +172,7 @@ zr_status zr_plan_set_workspace(zr_plan* p, void* d_ws, uint64_t bytes, zr_strea
     p->d_clip_coef = reinterpret_cast<float*>(base + L.clip_coef);
     p->d_own_sumsq = reinterpret_cast<double*>(base + L.own_sumsq);
     p->d_gather_targets = reinterpret_cast<uint16_t**>(base + L.gather_targets);
+    p->d_scalars = reinterpret_cast<zr::AdamScalars*>(base + L.dev_scalars);
     p->n_gather_targets = 0;
     p->d_g_scratch = p->clip_uses_scratch() ? reinterpret_cast<float*>(base + L.g_scratch) : nullptr;
     if (!p->tiles.empty()) {
@@ -224,8 +225,23 @@ zr_status zr_plan_set_gather_targets(zr_plan* p, void* const* targets, zr_stream
     return ZR_OK;
 }
 
+zr_status step_impl(const zr_plan* p, const void* const* grad_ptrs, float* master, float* m, float* v,
+                    void* param_out, int64_t step, int64_t* d_step, zr_stream_t stream);
+
 zr_status zr_step(const zr_plan* p, const void* const* grad_ptrs, float* master, float* m, float* v,
                   void* param_out, int64_t step, zr_stream_t stream) {
+    return step_impl(p, grad_ptrs, master, m, v, param_out, step, nullptr, stream);
+}
+
+zr_status zr_step_device_count(const zr_plan* p, const void* const* grad_ptrs, float* master, float* m, float* v,
+                               void* param_out, int64_t* d_step, zr_stream_t stream) {
+    if (!d_step) return ZR_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(d_step) & 7u) != 0) return ZR_ERR_ALIGNMENT;
+    return step_impl(p, grad_ptrs, master, m, v, param_out, 1, d_step, stream);
+}
+
+zr_status step_impl(const zr_plan* p, const void* const* grad_ptrs, float* master, float* m, float* v,
+                    void* param_out, int64_t step, int64_t* d_step, zr_stream_t stream) {
     if (!p || step < 1) return ZR_ERR_INVALID_ARG;
     if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
     if (p->owned_numel() == 0) return ZR_OK;
@@ -241,6 +257,12 @@ zr_status zr_step(const zr_plan* p, const void* const* grad_ptrs, float* master,
     a.param_out = static_cast<uint16_t*>(param_out);
     a.s = zr::adam_scalars(p->hp, step);
     void* s = stream;
+    if (d_step) {
+        // The count and the scalars live in device memory, so a captured
+        // graph of this call replays as the next step each time.
+        if (zr::launch_device_scalars(d_step, p->hp, p->d_scalars, s) != cudaSuccess) return ZR_ERR_CUDA;
+        a.dev_scalars = p->d_scalars;
+    }
     if (!p->clip_enabled())
         return cuda_status(static_cast<cudaError_t>(zr::launch_tiles(zr::Pass::kStep, a, grad_ptrs, false, false, s)));
 

@@ -262,6 +262,8 @@ WorkspaceLayout workspace_layout(const zr_plan& p) {
     off = align256(off + sizeof(double));
     L.gather_targets = off;
     off = align256(off + sizeof(void*) * static_cast<uint64_t>(p.world_size));
+    L.dev_scalars = off;
+    off = align256(off + sizeof(AdamScalars));
     L.g_scratch = off;
     off = align256(off + (p.clip_uses_scratch() ? sizeof(float) * static_cast<uint64_t>(p.owned_numel()) : 0));
     L.total = off;

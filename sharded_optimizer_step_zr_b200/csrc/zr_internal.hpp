@@ -67,12 +67,14 @@ struct LaunchArgs {
     double* tile_partials;     // kSumsq: one double per tile
     const float* clip_coef;    // kStepClip: device scalar
     AdamScalars s;
+    const AdamScalars* dev_scalars;   // when set, the step's scalars are read from here instead of s
 };
 
 // Kernel launchers (zr_kernels.cu).  grad_ptrs: host array of W device
 // pointers.  Return cudaError_t as int.
 int launch_tiles(Pass pass, const LaunchArgs& a, const void* const* grad_ptrs, bool g_from_scratch,
                  bool write_g_scratch, void* stream);
+int launch_device_scalars(int64_t* d_step, const zr_adamw& hp, AdamScalars* out, void* stream);
 int launch_clip_combine(const double* tile_partials, int32_t n_tiles, double* partials_all,
                         int32_t world_size, int32_t rank, float max_norm, float* clip_coef_out,
                         double* sumsq_out, void* stream);
@@ -115,6 +117,7 @@ struct zr_plan {
     float* d_g_scratch = nullptr;
     double* d_sumsq_partials = nullptr;   // caller-owned, world_size doubles
     uint16_t** d_gather_targets = nullptr; // workspace: world_size parameter buffers
+    zr::AdamScalars* d_scalars = nullptr;  // workspace: scalars computed on the device
     int32_t n_gather_targets = 0;          // 0 until zr_plan_set_gather_targets
 
     // zr_step_host's copy streams and events, created on its first call
@@ -138,7 +141,8 @@ zr_status build_plan(zr_plan& p, int32_t n_tensors, const int32_t* ndims,
                      const int64_t* const* shapes);
 // Workspace layout: offsets of each region, total bytes.
 struct WorkspaceLayout {
-    uint64_t tiles, tiles_by_owned, tile_partials, clip_coef, own_sumsq, gather_targets, g_scratch, total;
+    uint64_t tiles, tiles_by_owned, tile_partials, clip_coef, own_sumsq, gather_targets, dev_scalars, g_scratch,
+        total;
 };
 WorkspaceLayout workspace_layout(const zr_plan& p);
 AdamScalars adam_scalars(const zr_adamw& hp, int64_t step);

@@ -8,8 +8,8 @@
 //   * one 128-thread CTA per tile of up to 2048 owned elements (tiles never
 //     cross a bucket; the hardware block scheduler balances them across the
 //     148 SMs, five CTAs per SM);
-//   * each thread owns 8 consecutive elements per iteration and issues the W
-//     16-byte gradient loads of a group (up to 16 replicas) back to back,
+//   * each thread owns 8 consecutive elements per iteration and issues the
+//     16-byte gradient loads of a group of up to 8 replicas back to back,
 //     plus the 32-byte master / m / v loads, before consuming any of them;
 //   * the fold is a strict left fold in rank order in fp32, exactly the
 //     reduce of the definition; the AdamW arithmetic uses round-to-nearest
@@ -101,23 +101,26 @@ __device__ __forceinline__ void adamw(const AdamScalars& c, float g, float& p, f
     v = v_new;
 }
 
-// The bf16 results go to this rank's parameter buffer, or, when the plan has
-// gather targets, to every rank's: the all-gather done by peer stores in the
-// same pass that computes the values.
+// The bf16 results go to this rank's parameter buffer, or (GATHER) to every
+// rank's: the all-gather done by peer stores in the same pass that computes
+// the values.  A compile-time choice, so that the single-buffer kernels keep
+// their register allocation.
+template <bool GATHER>
 __device__ __forceinline__ void store_params8(const LaunchArgs& a, int64_t go, uint4 q) {
-    if (a.n_targets == 0) {
+    if constexpr (!GATHER) {
         __stcs(reinterpret_cast<uint4*>(a.param_out + go), q);
-        return;
+    } else {
+        for (int d = 0; d < a.n_targets; ++d) __stcs(reinterpret_cast<uint4*>(a.targets[d] + go), q);
     }
-    for (int d = 0; d < a.n_targets; ++d) __stcs(reinterpret_cast<uint4*>(a.targets[d] + go), q);
 }
 
+template <bool GATHER>
 __device__ __forceinline__ void store_param1(const LaunchArgs& a, int64_t go, uint16_t u) {
-    if (a.n_targets == 0) {
+    if constexpr (!GATHER) {
         a.param_out[go] = u;
-        return;
+    } else {
+        for (int d = 0; d < a.n_targets; ++d) a.targets[d][go] = u;
     }
-    for (int d = 0; d < a.n_targets; ++d) a.targets[d][go] = u;
 }
 
 // Left fold of W replicas for 8 consecutive owned elements at `off`.  The
@@ -177,13 +180,15 @@ __device__ double block_sum(double x) {
 // the tile kernel
 // ---------------------------------------------------------------------------
 
-template <int CAP, int G, Pass PASS, bool G_FROM_SCRATCH, bool WRITE_G>
+template <int CAP, int G, Pass PASS, bool G_FROM_SCRATCH, bool WRITE_G, bool DEV_SCALARS, bool GATHER>
 __global__ void __launch_bounds__(kThreads)
 zr_tile_kernel(const GradPtrs<CAP> gp, const LaunchArgs a) {
     const int32_t tix = a.reverse ? a.n_tiles - 1 - static_cast<int32_t>(blockIdx.x)
                                   : static_cast<int32_t>(blockIdx.x);
     const Tile tile = a.tiles[tix];
     const int W = a.world_size;
+    AdamScalars sc = a.s;
+    if constexpr (DEV_SCALARS) sc = *a.dev_scalars;   // computed on the device for this step
     float coef = 1.0f;
     if constexpr (PASS == Pass::kStepClip) coef = *a.clip_coef;
     double sq = 0.0;
@@ -234,7 +239,7 @@ zr_tile_kernel(const GradPtrs<CAP> gp, const LaunchArgs a) {
                 float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
                 float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-                for (int k = 0; k < 8; ++k) adamw(a.s, g[k], p[k], mm[k], vv[k]);
+                for (int k = 0; k < 8; ++k) adamw(sc, g[k], p[k], mm[k], vv[k]);
                 st_state16(a.master + o, make_float4(p[0], p[1], p[2], p[3]));
                 st_state16(a.master + o + 4, make_float4(p[4], p[5], p[6], p[7]));
                 st_state16(a.m + o, make_float4(mm[0], mm[1], mm[2], mm[3]));
@@ -248,14 +253,14 @@ zr_tile_kernel(const GradPtrs<CAP> gp, const LaunchArgs a) {
                     q.y = pack_bf16x2(p[2], p[3]);
                     q.z = pack_bf16x2(p[4], p[5]);
                     q.w = pack_bf16x2(p[6], p[7]);
-                    store_params8(a, go, q);
+                    store_params8<GATHER>(a, go, q);
                 } else {
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         __nv_bfloat16 h = __float2bfloat16_rn(p[k]);
                         uint16_t u;
                         memcpy(&u, &h, 2);
-                        store_param1(a, go + k, u);
+                        store_param1<GATHER>(a, go + k, u);
                     }
                 }
             }
@@ -272,14 +277,14 @@ zr_tile_kernel(const GradPtrs<CAP> gp, const LaunchArgs a) {
             if constexpr (PASS == Pass::kStep || PASS == Pass::kStepClip) {
                 if constexpr (PASS == Pass::kStepClip) g = __fmul_rn(g, coef);
                 float p = a.master[o], mm = a.m[o], vv = a.v[o];
-                adamw(a.s, g, p, mm, vv);
+                adamw(sc, g, p, mm, vv);
                 a.master[o] = p;
                 a.m[o] = mm;
                 a.v[o] = vv;
                 __nv_bfloat16 h = __float2bfloat16_rn(p);
                 uint16_t u;
                 memcpy(&u, &h, 2);
-                store_param1(a, tile.global + e, u);
+                store_param1<GATHER>(a, tile.global + e, u);
             }
         }
     }
@@ -287,6 +292,26 @@ zr_tile_kernel(const GradPtrs<CAP> gp, const LaunchArgs a) {
         const double total = block_sum(sq);
         if (threadIdx.x == 0) a.tile_partials[tile.index] = total;
     }
+}
+
+// One thread: advance the device step count and compute the AdamW scalars
+// for the new step, in fp64 from the fp32 hyperparameters and rounded once
+// to fp32 -- the same expressions as the host computes for zr_step.
+__global__ void zr_device_scalars_kernel(int64_t* d_step, const zr_adamw hp, AdamScalars* out) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    const int64_t step = *d_step + 1;
+    *d_step = step;
+    const double b1 = hp.beta1, b2 = hp.beta2, lr = hp.lr, t = static_cast<double>(step);
+    AdamScalars s;
+    s.beta1 = hp.beta1;
+    s.beta2 = hp.beta2;
+    s.one_minus_beta1 = static_cast<float>(1.0 - b1);
+    s.one_minus_beta2 = static_cast<float>(1.0 - b2);
+    s.step_size = static_cast<float>(lr / (1.0 - pow(b1, t)));
+    s.bc2_sqrt = static_cast<float>(sqrt(1.0 - pow(b2, t)));
+    s.decay = static_cast<float>(1.0 - lr * static_cast<double>(hp.weight_decay));
+    s.eps = hp.eps;
+    *out = s;
 }
 
 // One block: S_r = sum of the per-tile partials in a fixed order, stored as
@@ -331,26 +356,40 @@ zr_clip_combine_kernel(const double* __restrict__ tile_partials, int32_t n_tiles
     }
 }
 
-template <int CAP, int G, Pass PASS, bool FROM, bool WRITE>
+template <int CAP, int G, Pass PASS, bool FROM, bool WRITE, bool DEVSC, bool GATHER>
 cudaError_t launch_one(const LaunchArgs& a, const void* const* grad_ptrs, cudaStream_t stream) {
     // grad_ptrs may be NULL for the pass that reads the g scratch instead.
     GradPtrs<CAP> gp;
     for (int w = 0; w < CAP; ++w)
         gp.p[w] = (grad_ptrs != nullptr && w < a.world_size) ? static_cast<const uint16_t*>(grad_ptrs[w]) : nullptr;
-    zr_tile_kernel<CAP, G, PASS, FROM, WRITE><<<a.n_tiles, kThreads, 0, stream>>>(gp, a);
+    zr_tile_kernel<CAP, G, PASS, FROM, WRITE, DEVSC, GATHER><<<a.n_tiles, kThreads, 0, stream>>>(gp, a);
     return cudaGetLastError();
 }
 
-template <Pass PASS, bool FROM, bool WRITE>
+template <Pass PASS, bool FROM, bool WRITE, bool DEVSC = false, bool GATHER = false>
 cudaError_t dispatch_w(const LaunchArgs& a, const void* const* grad_ptrs, cudaStream_t stream) {
-    const int W = a.world_size;
-    if (FROM) return launch_one<1, 1, PASS, FROM, WRITE>(a, grad_ptrs, stream);
-    if (W <= 2) return launch_one<2, 2, PASS, FROM, WRITE>(a, grad_ptrs, stream);
-    if (W <= 4) return launch_one<4, 4, PASS, FROM, WRITE>(a, grad_ptrs, stream);
-    if (W <= 8) return launch_one<8, 8, PASS, FROM, WRITE>(a, grad_ptrs, stream);
-    if (W <= 16) return launch_one<16, 16, PASS, FROM, WRITE>(a, grad_ptrs, stream);
-    if (W <= 64) return launch_one<64, 8, PASS, FROM, WRITE>(a, grad_ptrs, stream);
-    return launch_one<ZR_MAX_WORLD_SIZE, 8, PASS, FROM, WRITE>(a, grad_ptrs, stream);
+    if constexpr (FROM) {
+        return launch_one<1, 1, PASS, FROM, WRITE, DEVSC, GATHER>(a, grad_ptrs, stream);
+    } else {
+        const int W = a.world_size;
+        if (W <= 2) return launch_one<2, 2, PASS, FROM, WRITE, DEVSC, GATHER>(a, grad_ptrs, stream);
+        if (W <= 4) return launch_one<4, 4, PASS, FROM, WRITE, DEVSC, GATHER>(a, grad_ptrs, stream);
+        if (W <= 8) return launch_one<8, 8, PASS, FROM, WRITE, DEVSC, GATHER>(a, grad_ptrs, stream);
+        if (W <= 16) return launch_one<16, 8, PASS, FROM, WRITE, DEVSC, GATHER>(a, grad_ptrs, stream);
+        if (W <= 64) return launch_one<64, 8, PASS, FROM, WRITE, DEVSC, GATHER>(a, grad_ptrs, stream);
+        return launch_one<ZR_MAX_WORLD_SIZE, 8, PASS, FROM, WRITE, DEVSC, GATHER>(a, grad_ptrs, stream);
+    }
+}
+
+// The passes that write parameters, with the device-scalar and gather-target
+// variants chosen from the launch arguments.
+template <Pass PASS, bool FROM>
+cudaError_t dispatch_update(const LaunchArgs& a, const void* const* grad_ptrs, cudaStream_t s) {
+    const bool dev = a.dev_scalars != nullptr, gather = a.n_targets > 0;
+    if (dev && gather) return dispatch_w<PASS, FROM, false, true, true>(a, grad_ptrs, s);
+    if (dev) return dispatch_w<PASS, FROM, false, true, false>(a, grad_ptrs, s);
+    if (gather) return dispatch_w<PASS, FROM, false, false, true>(a, grad_ptrs, s);
+    return dispatch_w<PASS, FROM, false, false, false>(a, grad_ptrs, s);
 }
 
 }  // namespace
@@ -360,16 +399,21 @@ int launch_tiles(Pass pass, const LaunchArgs& a, const void* const* grad_ptrs, b
     if (a.n_tiles == 0) return cudaSuccess;
     cudaStream_t s = static_cast<cudaStream_t>(stream_v);
     switch (pass) {
-        case Pass::kStep: return dispatch_w<Pass::kStep, false, false>(a, grad_ptrs, s);
+        case Pass::kStep: return dispatch_update<Pass::kStep, false>(a, grad_ptrs, s);
         case Pass::kReduceOnly: return dispatch_w<Pass::kReduceOnly, false, false>(a, grad_ptrs, s);
         case Pass::kSumsq:
             return write_g_scratch ? dispatch_w<Pass::kSumsq, false, true>(a, grad_ptrs, s)
                                    : dispatch_w<Pass::kSumsq, false, false>(a, grad_ptrs, s);
         case Pass::kStepClip:
-            return g_from_scratch ? dispatch_w<Pass::kStepClip, true, false>(a, grad_ptrs, s)
-                                  : dispatch_w<Pass::kStepClip, false, false>(a, grad_ptrs, s);
+            return g_from_scratch ? dispatch_update<Pass::kStepClip, true>(a, grad_ptrs, s)
+                                  : dispatch_update<Pass::kStepClip, false>(a, grad_ptrs, s);
     }
     return cudaErrorInvalidValue;
+}
+
+int launch_device_scalars(int64_t* d_step, const zr_adamw& hp, AdamScalars* out, void* stream_v) {
+    zr_device_scalars_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream_v)>>>(d_step, hp, out);
+    return cudaGetLastError();
 }
 
 int launch_clip_combine(const double* tile_partials, int32_t n_tiles, double* partials_all,
