@@ -40,18 +40,20 @@ def check_invariants(plan):
     goff = np.concatenate([[0], np.cumsum(numels)]).astype(np.int64)
     assert plan.total_numel == N
     segs = plan.segments
+    def tiles_exactly(intervals, end):
+        """Intervals (start, length) cover [0, end) exactly once."""
+        at = 0
+        for start, length in sorted(intervals):
+            assert length > 0 and start == at, (start, at)
+            at = start + length
+        assert at == end
+
     # exact cover of [0, padded): every element in exactly one segment
-    cover = np.zeros(plan.padded_numel, dtype=np.int32)
-    for s in segs:
-        assert s["length"] > 0
-        cover[s["global_offset"]: s["global_offset"] + s["length"]] += 1
-    assert np.all(cover == 1)
+    tiles_exactly([(int(s["global_offset"]), int(s["length"])) for s in segs], plan.padded_numel)
     # per rank: owned offsets tile [0, owned_numel) exactly
     for r in range(W):
-        own = np.zeros(int(plan.owned_numel[r]), dtype=np.int32)
-        for s in segs[segs["owner"] == r]:
-            own[s["owned_offset"]: s["owned_offset"] + s["length"]] += 1
-        assert np.all(own == 1)
+        tiles_exactly([(int(s["owned_offset"]), int(s["length"])) for s in segs[segs["owner"] == r]],
+                      int(plan.owned_numel[r]))
     assert plan.owned_numel.sum() == plan.padded_numel
     # tensor pieces concatenate back to [0, numel) and sit at the declared offset
     for t, n in enumerate(numels):
