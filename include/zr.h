@@ -60,7 +60,8 @@
  *   inside a kernel surfaces at the caller's next synchronisation.  On any
  *   error status nothing has been launched.  Buffers must not overlap; the
  *   gradient buffers are read-only.  A plan may be used from one host thread
- *   at a time.
+ *   at a time, and only while the device that was current when its
+ *   workspace was bound is current (else ZR_ERR_INVALID_ARG).
  */
 #ifndef ZR_H_
 #define ZR_H_

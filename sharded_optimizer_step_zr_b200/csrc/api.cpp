@@ -47,6 +47,14 @@ zr_status check_param_out(const zr_plan* p, const void* param_out) {
     return aligned16(param_out) ? ZR_OK : ZR_ERR_ALIGNMENT;
 }
 
+// Kernels launch on the current device; the plan's buffers belong to the
+// device that was current when its workspace was bound.
+zr_status check_device(const zr_plan* p) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ZR_ERR_CUDA;
+    return dev == p->device ? ZR_OK : ZR_ERR_INVALID_ARG;
+}
+
 zr_status check_state(const float* master, const float* m, const float* v) {
     if (!master || !m || !v) return ZR_ERR_INVALID_ARG;
     if (!aligned16(master) || !aligned16(m) || !aligned16(v)) return ZR_ERR_ALIGNMENT;
@@ -244,6 +252,10 @@ zr_status step_impl(const zr_plan* p, const void* const* grad_ptrs, float* maste
                     void* param_out, int64_t step, int64_t* d_step, zr_stream_t stream) {
     if (!p || step < 1) return ZR_ERR_INVALID_ARG;
     if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
+    {
+        const zr_status dst = check_device(p);
+        if (dst != ZR_OK) return dst;
+    }
     if (p->owned_numel() == 0) return ZR_OK;
     zr_status st = check_grads(p, grad_ptrs);
     if (st != ZR_OK) return st;
@@ -290,6 +302,10 @@ zr_status zr_step_bucket(const zr_plan* p, int32_t bucket, const void* const* gr
     if (!p || step < 1) return ZR_ERR_INVALID_ARG;
     if (bucket < 0 || bucket >= p->n_buckets) return ZR_ERR_INVALID_ARG;
     if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
+    {
+        const zr_status dst = check_device(p);
+        if (dst != ZR_OK) return dst;
+    }
     const int32_t first = p->bucket_first_tile[bucket];
     const int32_t count = p->bucket_first_tile[bucket + 1] - first;
     if (count == 0) return ZR_OK;   // this rank owns nothing in the bucket
@@ -320,6 +336,10 @@ zr_status zr_step_finish(const zr_plan* p, const void* const* grad_ptrs, float* 
                          void* param_out, int64_t step, zr_stream_t stream) {
     if (!p || step < 1) return ZR_ERR_INVALID_ARG;
     if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
+    {
+        const zr_status dst = check_device(p);
+        if (dst != ZR_OK) return dst;
+    }
     if (!p->clip_enabled() || p->owned_numel() == 0) return ZR_OK;
     if (!p->d_sumsq_partials) return ZR_ERR_NO_WORKSPACE;
     const bool scratch = p->clip_uses_scratch();
@@ -351,6 +371,10 @@ zr_status zr_step_finish(const zr_plan* p, const void* const* grad_ptrs, float* 
 zr_status zr_grad_sumsq(const zr_plan* p, const void* const* grad_ptrs, double* d_out, zr_stream_t stream) {
     if (!p || !d_out) return ZR_ERR_INVALID_ARG;
     if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
+    {
+        const zr_status dst = check_device(p);
+        if (dst != ZR_OK) return dst;
+    }
     if (!p->clip_enabled()) return ZR_ERR_INVALID_ARG;   // tile partials live in the clip workspace
     if ((reinterpret_cast<uintptr_t>(d_out) & 7u) != 0) return ZR_ERR_ALIGNMENT;
     void* s = stream;
@@ -371,6 +395,10 @@ zr_status zr_grad_sumsq(const zr_plan* p, const void* const* grad_ptrs, double* 
 zr_status zr_debug_reduce(const zr_plan* p, const void* const* grad_ptrs, float* g_out, zr_stream_t stream) {
     if (!p || !g_out) return ZR_ERR_INVALID_ARG;
     if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
+    {
+        const zr_status dst = check_device(p);
+        if (dst != ZR_OK) return dst;
+    }
     if (p->owned_numel() == 0) return ZR_OK;
     zr_status st = check_grads(p, grad_ptrs);
     if (st != ZR_OK) return st;
@@ -386,6 +414,10 @@ zr_status zr_step_host(const zr_plan* p, const void* const* host_grad_ptrs, void
                        int64_t step, zr_stream_t stream) {
     if (!p || !host_grad_ptrs || !dev_grad_ptrs || !host_param_out || step < 1) return ZR_ERR_INVALID_ARG;
     if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
+    {
+        const zr_status dst = check_device(p);
+        if (dst != ZR_OK) return dst;
+    }
     if (p->n_gather_targets > 0) return ZR_ERR_UNSUPPORTED;   // copies back this rank's buffer only
     const int64_t n = p->owned_numel();
     if (n == 0) return ZR_OK;

@@ -110,6 +110,7 @@ __device__ __forceinline__ void store_params8(const LaunchArgs& a, int64_t go, u
     if constexpr (!GATHER) {
         __stcs(reinterpret_cast<uint4*>(a.param_out + go), q);
     } else {
+#pragma unroll 1
         for (int d = 0; d < a.n_targets; ++d) __stcs(reinterpret_cast<uint4*>(a.targets[d] + go), q);
     }
 }
@@ -119,6 +120,7 @@ __device__ __forceinline__ void store_param1(const LaunchArgs& a, int64_t go, ui
     if constexpr (!GATHER) {
         a.param_out[go] = u;
     } else {
+#pragma unroll 1
         for (int d = 0; d < a.n_targets; ++d) a.targets[d][go] = u;
     }
 }
