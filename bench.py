@@ -37,7 +37,7 @@ UNIT = "Gparams/s"
 DEFAULT_CONFIG = "gpt2_124m_w8"
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCE = os.path.join(ROOT, "sharded_optimizer_step_zr_b200", "csrc", "zr_kernels.cu")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+PROFILES = os.path.join(ROOT, "profiles")
 
 
 def parse():
@@ -118,7 +118,7 @@ def recorded_traffic(workload_name):
     dominant kernel from the committed ncu summary, if it was taken on the
     current kernel source; else None."""
     try:
-        with open(TRAFFIC_FILE) as f:
+        with open(os.path.join(PROFILES, f"zr_tile_kernel_{workload_name}_traffic.json")) as f:
             d = json.load(f)
         e = d.get(workload_name)
         if e and e.get("kernel_source_sha256_16") == kernel_source_hash():
