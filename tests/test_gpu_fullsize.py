@@ -64,11 +64,17 @@ def host_global_sumsq(oplan, wl, step, threads):
     return S, parts
 
 
+SWEEP = {wl.name: wl for wl in synth.sweep_workloads()}
+
+
 @pytest.mark.parametrize("name, rank", [("gpt2_124m_w8", None), ("llama_7b_w64", None),
                                         ("llama_7b_w64", 63),   # parameter offsets beyond 2**32
-                                        ("gpt_1p3b_w8_whole_clip", None)])
+                                        ("gpt_1p3b_w8_whole_clip", None)] +
+                         # the 1.3B sweep: one point per (W, partition) at the 25 MB cap
+                         [(f"sweep_1p3b_{m}_w{w}_cap25", None) for m in ("flat", "whole")
+                          for w in (2, 8, 32, 64)])
 def test_full_size_sampled(name, rank):
-    wl = synth.WORKLOADS[name]
+    wl = synth.WORKLOADS[name] if name in synth.WORKLOADS else SWEEP[name]
     rank = wl.ranks[0] if rank is None else rank
     W = wl.world_size
     clip = wl.max_grad_norm > 0
