@@ -233,8 +233,8 @@ zr_status zr_plan_set_gather_targets(zr_plan* p, void* const* targets, zr_stream
     return ZR_OK;
 }
 
-zr_status step_impl(const zr_plan* p, const void* const* grad_ptrs, float* master, float* m, float* v,
-                    void* param_out, int64_t step, int64_t* d_step, zr_stream_t stream);
+static zr_status step_impl(const zr_plan* p, const void* const* grad_ptrs, float* master, float* m, float* v,
+                           void* param_out, int64_t step, int64_t* d_step, zr_stream_t stream);
 
 zr_status zr_step(const zr_plan* p, const void* const* grad_ptrs, float* master, float* m, float* v,
                   void* param_out, int64_t step, zr_stream_t stream) {
@@ -248,15 +248,21 @@ zr_status zr_step_device_count(const zr_plan* p, const void* const* grad_ptrs, f
     return step_impl(p, grad_ptrs, master, m, v, param_out, 1, d_step, stream);
 }
 
-zr_status step_impl(const zr_plan* p, const void* const* grad_ptrs, float* master, float* m, float* v,
-                    void* param_out, int64_t step, int64_t* d_step, zr_stream_t stream) {
+static zr_status step_impl(const zr_plan* p, const void* const* grad_ptrs, float* master, float* m, float* v,
+                           void* param_out, int64_t step, int64_t* d_step, zr_stream_t stream) {
     if (!p || step < 1) return ZR_ERR_INVALID_ARG;
     if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
     {
         const zr_status dst = check_device(p);
         if (dst != ZR_OK) return dst;
     }
-    if (p->owned_numel() == 0) return ZR_OK;
+    if (p->owned_numel() == 0) {
+        // Nothing to update, but a device step count still advances, so it
+        // stays equal on every rank.
+        if (d_step)
+            return cuda_status(static_cast<cudaError_t>(zr::launch_device_scalars(d_step, p->hp, p->d_scalars, stream)));
+        return ZR_OK;
+    }
     zr_status st = check_grads(p, grad_ptrs);
     if (st != ZR_OK) return st;
     if ((st = check_state(master, m, v)) != ZR_OK || (st = check_param_out(p, param_out)) != ZR_OK) return st;

@@ -47,3 +47,17 @@ def test_captured_step_replays_as_successive_steps(max_norm):
             assert_state_close(b, a, f"{what} step {t}")
             assert np.array_equal(bits32(a), bits32(b)), f"{what} step {t} not bit-identical"
         assert torch.equal(out_e.view(torch.int16), out_g.view(torch.int16))
+
+
+def test_device_count_advances_on_a_rank_that_owns_nothing():
+    """Whole-tensor ownership with more ranks than tensors: rank 5 owns
+    nothing, yet its device step count advances with every call."""
+    import sharded_optimizer_step_zr_b200 as zr
+    g = GpuRank([(64,), (32,)], 8, 5, 1, 1 << 20, (3e-4, 0.9, 0.999, 1e-8, 0.1, 0.0), seed=3)
+    assert g.plan.owned_numel == 0
+    d_step = torch.zeros(1, dtype=torch.int64, device=DEV)
+    out = torch.zeros(96 + 8, dtype=torch.bfloat16, device=DEV)
+    for t in (1, 2, 3):
+        zr.zr_step_device_count(g.plan.handle, g.grads, g.master, g.m, g.v, out, d_step)
+    torch.cuda.synchronize()
+    assert int(d_step.item()) == 3
