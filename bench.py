@@ -189,42 +189,54 @@ class ClockSampler:
 # CPU arm: the oracle on a bounded sample
 # ---------------------------------------------------------------------------
 
+class OracleSample:
+    """A bounded sample of one rank's shard for the oracle (test
+    infrastructure, used by the CPU baseline only): the rank's first owned
+    elements with the workload's gradient statistics, as their own W-replica
+    flat plan of one tensor."""
+
+    def __init__(self, wl, rank, max_elems):
+        import numpy as np
+        import oracle
+        import synth
+        import torch
+        oplan = oracle.Plan(wl.shapes, wl.world_size, wl.mode, wl.bucket_cap_bytes)
+        self.n = n = min(int(oplan.owned_numel[rank]), max_elems)
+        self.owned = int(oplan.owned_numel[rank])
+        idx = torch.from_numpy(oplan.owned_global_index(rank)[:n])
+        self.grads = [synth.grad_bf16(wl.seed, 1, w, idx, wl.grad_sigma, wl.outlier_frac,
+                                      n_valid=oplan.total_numel).view(torch.int16).numpy()
+                      .view(np.uint16).copy() for w in range(wl.world_size)]
+        self.master = synth.master_f32(wl.seed, idx, n_valid=oplan.total_numel).numpy().copy()
+        self.m = np.zeros(n, np.float32)
+        self.v = np.zeros(n, np.float32)
+        self.plan = oracle.Plan([(n * wl.world_size,)], wl.world_size, oracle.FLAT, 1 << 62)
+        self.out = np.zeros(self.plan.padded_numel, np.uint16)
+        self.wl, self.rank, self.t = wl, rank, 0
+
+    def run(self, target_seconds):
+        """Oracle steps on the sample until `target_seconds` of CPU work;
+        returns (Gparams/s, description)."""
+        import oracle
+        clip = 1.0 if self.wl.max_grad_norm > 0 else None
+        steps, t0 = 0, time.perf_counter()
+        while True:
+            self.t += 1
+            oracle.rank_step(self.plan, 0, self.grads, self.master, self.m, self.v, self.out,
+                             self.wl.hp, self.t, clip=clip)
+            if clip is not None:
+                oracle.sumsq(oracle.reduce(self.grads))      # the clip's extra reduce pass
+            steps += 1
+            el = time.perf_counter() - t0
+            if el >= target_seconds:
+                break
+        desc = (f"oracle rank_step on {self.n} of rank {self.rank}'s {self.owned} owned params "
+                f"(W={self.wl.world_size}), {steps} steps, {el:.1f} s, 1 thread")
+        return self.n * steps / el / 1e9, desc
+
+
 def oracle_sample_rate(wl, rank, target_seconds, max_elems=1 << 21):
-    """Time the oracle's rank step (single thread) on the first owned
-    elements of `rank` for the workload's gradient statistics; repeat steps
-    until `target_seconds` of CPU work.  Returns (Gparams/s, description)."""
-    import numpy as np
-    import oracle
-    import synth
-    oplan = oracle.Plan(wl.shapes, wl.world_size, wl.mode, wl.bucket_cap_bytes)
-    n = min(int(oplan.owned_numel[rank]), max_elems)
-    # the sample: owned elements [0, n) of this rank, as their own small plan
-    # with the same W (flat, one tensor of n elements owned by every rank)
-    idx = oplan.owned_global_index(rank)[:n]
-    import torch
-    t_idx = torch.from_numpy(idx)
-    grads = [synth.grad_bf16(wl.seed, 1, w, t_idx, wl.grad_sigma, wl.outlier_frac,
-                             n_valid=oplan.total_numel).view(torch.int16).numpy().view(np.uint16).copy()
-             for w in range(wl.world_size)]
-    master = synth.master_f32(wl.seed, t_idx, n_valid=oplan.total_numel).numpy().copy()
-    m = np.zeros(n, np.float32)
-    v = np.zeros(n, np.float32)
-    sample_plan = oracle.Plan([(n * wl.world_size,)], wl.world_size, oracle.FLAT, 1 << 62)
-    out = np.zeros(sample_plan.padded_numel, np.uint16)
-    clip = 1.0 if wl.max_grad_norm > 0 else None
-    steps, t0 = 0, time.perf_counter()
-    while True:
-        oracle.rank_step(sample_plan, 0, grads, master, m, v, out, wl.hp, steps + 1, clip=clip)
-        if clip is not None:
-            oracle.sumsq(oracle.reduce(grads))      # the clip's extra reduce pass
-        steps += 1
-        el = time.perf_counter() - t0
-        if el >= target_seconds:
-            break
-    rate = n * steps / el / 1e9
-    desc = (f"oracle rank_step on {n} of rank {rank}'s {int(oplan.owned_numel[rank])} owned params "
-            f"(W={wl.world_size}), {steps} steps, {el:.1f} s, 1 thread")
-    return rate, desc
+    return OracleSample(wl, rank, max_elems).run(target_seconds)
 
 
 def run_reference(args):
@@ -234,10 +246,11 @@ def run_reference(args):
     wl = workload(args.config)
     K, Wm = args.steps, args.warmup
     budget = max(0.05, min(2.0, 120.0 / max(1, K + Wm)))
+    sample = OracleSample(wl, wl.ranks[0], 1 << 18)
     rates = []
     desc = ""
     for i in range(Wm + K):
-        r, desc = oracle_sample_rate(wl, wl.ranks[0], budget, max_elems=1 << 18)
+        r, desc = sample.run(budget)
         if i >= Wm:
             rates.append(r)
     value = statistics.median(rates)
