@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--per-bucket", action="store_true",
                     help="step bucket by bucket (zr_step_bucket per bucket, then zr_step_finish)")
+    ap.add_argument("--overlap", action="store_true",
+                    help="exposed optimizer time behind an emulated backward pass: one zr_step "
+                         "after it, against zr_step_bucket as each bucket's gradients complete")
     ap.add_argument("--sweep", action="store_true",
                     help="1.3B set: bucket cap x W x partition; one JSON record per point")
     return ap.parse_args()
@@ -496,8 +499,131 @@ def run_sweep(args):
             torch.cuda.empty_cache()
 
 
+def run_overlap(args):
+    """Bucket-by-bucket stepping overlapped with the backward pass.
+
+    The backward pass is emulated by one bf16 matmul per bucket on a compute
+    stream, in bucket (backward) order, each sized in proportion to the
+    bucket's parameter count and together about 20 times the optimizer
+    step; an event marks each bucket's gradients as ready.  Measured:
+    (a) the backward alone; (b) the backward, then one zr_step; (c) the
+    backward with zr_step_bucket launched on a second stream as each bucket
+    completes (then zr_step_finish).  The optimizer time left exposed is
+    (b) - (a) against (c) - (a)."""
+    import torch
+    import synth
+    from sharded_optimizer_step_zr_b200.plan import ZrPlan
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    wl = workload(args.config)
+    W, rank = wl.world_size, wl.ranks[0]
+    plan = ZrPlan(wl.shapes, W, rank, wl.mode, wl.bucket_cap_bytes, *wl.hp, device=dev)
+    n = plan.owned_numel
+    runs = plan.runs()
+    grads = [torch.empty(n, dtype=torch.bfloat16, device=dev) for _ in range(W)]
+    for w in range(W):
+        synth.fill_owned_grad(grads[w], runs, wl.seed, 1, w, wl.grad_sigma, wl.outlier_frac,
+                              n_valid=plan.total_numel)
+    master = torch.empty(n, dtype=torch.float32, device=dev)
+    synth.fill_owned_master(master, runs, wl.seed, n_valid=plan.total_numel)
+    m, v = torch.zeros_like(master), torch.zeros_like(master)
+    out = torch.zeros(plan.padded_numel, dtype=torch.bfloat16, device=dev)
+    if wl.max_grad_norm > 0:
+        plan.grad_sumsq(grads, plan.partials[rank:rank + 1])
+        plan.partials.fill_(float(plan.partials[rank].item()))
+    segs = plan.segments()
+    bucket_params = [0] * plan.n_buckets
+    for sgm in segs:
+        bucket_params[sgm["bucket"]] += sgm["length"]
+    compute, opt = torch.cuda.Stream(), torch.cuda.Stream()
+    step_no = [0]
+
+    def step_once(stream):
+        step_no[0] += 1
+        with torch.cuda.stream(stream):
+            plan.step(grads, master, m, v, out, step_no[0], stream)
+
+    # size the emulated backward: total ~20x one optimizer step
+    for _ in range(3):
+        step_once(compute)
+    torch.cuda.synchronize()
+    a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a_.record(compute)
+    for _ in range(5):
+        step_once(compute)
+    b_.record(compute)
+    torch.cuda.synchronize()
+    opt_ms = a_.elapsed_time(b_) / 5
+    x = torch.randn(4096, 4096, dtype=torch.bfloat16, device=dev)
+    with torch.cuda.stream(compute):
+        for _ in range(3):
+            torch.matmul(x, x)
+    torch.cuda.synchronize()
+    a_.record(compute)
+    for _ in range(10):
+        with torch.cuda.stream(compute):
+            torch.matmul(x, x)
+    b_.record(compute)
+    torch.cuda.synchronize()
+    mm_ms = a_.elapsed_time(b_) / 10
+    total = sum(bucket_params)
+    reps = [max(1, round(20.0 * opt_ms / mm_ms * p / total)) for p in bucket_params]
+    ready = [torch.cuda.Event() for _ in range(plan.n_buckets)]
+
+    def backward():
+        with torch.cuda.stream(compute):
+            for b in range(plan.n_buckets):
+                for _ in range(reps[b]):
+                    torch.matmul(x, x)
+                ready[b].record(compute)
+
+    my_buckets = sorted({sgm["bucket"] for sgm in segs if sgm["owner"] == rank})
+
+    def time_it(fn, iters=args.steps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(compute)
+        for _ in range(iters):
+            fn()
+        opt.wait_stream(compute)
+        compute.wait_stream(opt)
+        t1.record(compute)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1) / iters
+
+    def sequential():
+        backward()
+        step_once(compute)
+
+    def overlapped():
+        backward()
+        step_no[0] += 1
+        for b in my_buckets:
+            opt.wait_event(ready[b])
+            with torch.cuda.stream(opt):
+                plan.step_bucket(b, grads, master, m, v, out, step_no[0], opt)
+        with torch.cuda.stream(opt):
+            plan.step_finish(grads, master, m, v, out, step_no[0], opt)
+        compute.wait_stream(opt)      # the next backward reads the new parameters
+
+    back_ms = time_it(backward)
+    seq_ms = time_it(sequential)
+    ovl_ms = time_it(overlapped)
+    print(json.dumps({"mode": "overlap", "workload": wl.name, "rank": rank, "owned_params": n,
+                      "buckets_stepped": len(my_buckets), "optimizer_step_ms": opt_ms,
+                      "backward_ms": back_ms, "backward_then_step_ms": seq_ms,
+                      "backward_with_bucket_steps_ms": ovl_ms,
+                      "exposed_ms_single_step": seq_ms - back_ms,
+                      "exposed_ms_per_bucket": ovl_ms - back_ms}), flush=True)
+
+
 def main():
     args = parse()
+    if args.overlap:
+        run_overlap(args)
+        return
     if args.sweep:
         run_sweep(args)
         return
