@@ -261,7 +261,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": K, "warmup": Wm, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": wl.name, "param_set": wl.param_set, "W": wl.world_size,
+        "config": {"workload": wl.name, "W": wl.world_size,
                    "rank": wl.ranks[0], "partition": "flat" if wl.mode == 0 else "whole_tensor",
                    "bucket_cap_mb": wl.bucket_cap_mb},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
@@ -423,7 +423,7 @@ def run_zr(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": wl.name, "param_set": wl.param_set, "W": W, "rank": zr_rank,
+        "config": {"workload": wl.name, "W": W, "rank": zr_rank,
                    "partition": "flat" if wl.mode == 0 else "whole_tensor",
                    "bucket_cap_mb": wl.bucket_cap_mb, "clip": clip, "owned_params": n,
                    "per_bucket": bool(args.per_bucket), "buckets_stepped": len(my_buckets),
