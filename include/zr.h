@@ -334,6 +334,23 @@ zr_status zr_state_load(const zr_plan* plan, const char* path, float* master, fl
 zr_status zr_state_reshard(const zr_plan* target, const char* const* src_paths, int32_t n_src,
                            const char* dst_path);
 
+/* Gather to a whole model on save: from src_paths[0..n_src), the complete
+ * set of shards (rank r at index r) of any partition of `plan`'s tensors
+ * (`plan` supplies the shapes only; its W, rank and mode do not matter),
+ * writes the master weights of all total_numel parameters in declaration
+ * order -- tensor by tensor, each row-major, no pad -- to out_path as a raw
+ * little-endian array: fp32 (ZR_EXPORT_F32) or bf16 rounded to nearest even
+ * (ZR_EXPORT_BF16, the value the step writes into the all-gather buffer).
+ * No header: the file is exactly total_numel * 4 or * 2 bytes.  Host only;
+ * reads each shard whole once, holds the output in host memory and writes it
+ * through a temporary file renamed into place; *n_written (may be NULL)
+ * receives total_numel.  Errors as zr_state_reshard, and ZR_ERR_INVALID_ARG
+ * for an unknown dtype. */
+#define ZR_EXPORT_F32 0
+#define ZR_EXPORT_BF16 1
+zr_status zr_state_export_params(const zr_plan* plan, const char* const* src_paths, int32_t n_src,
+                                 int32_t dtype, const char* out_path, int64_t* n_written);
+
 /* Size of the library-owned scratch array used by zr_step_no_alloc. */
 #define ZR_NO_ALLOC_SCRATCH_BYTES (4u << 20)
 

@@ -44,7 +44,7 @@ EXPORTED = [
     "zr_step_bucket",
     "zr_step_finish", "zr_step_host",
     "zr_grad_sumsq", "zr_debug_reduce", "zr_step_no_alloc", "zr_state_save", "zr_state_load",
-    "zr_state_reshard", "zr_plan_owner_offsets", "zr_plan_set_gather_targets", "zr_ipc_export",
+    "zr_state_reshard", "zr_state_export_params", "zr_plan_owner_offsets", "zr_plan_set_gather_targets", "zr_ipc_export",
     "zr_ipc_open", "zr_ipc_close", "zr_plan_destroy", "zr_status_string",
 ]
 ZR_NO_ALLOC_SCRATCH_BYTES = 4 << 20
@@ -86,6 +86,7 @@ _lib.zr_step_no_alloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_state_save.argtypes = [_vp, ctypes.c_char_p, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_state_load.argtypes = [_vp, ctypes.c_char_p, _vp, _vp, _vp, _P(_i64), _vp]
 _lib.zr_state_reshard.argtypes = [_vp, _vp, _i32, ctypes.c_char_p]
+_lib.zr_state_export_params.argtypes = [_vp, _vp, _i32, _i32, ctypes.c_char_p, _vp]
 _lib.zr_plan_owner_offsets.argtypes = [_vp, _vp]
 _lib.zr_plan_set_gather_targets.argtypes = [_vp, _vp, _vp]
 _lib.zr_ipc_export.argtypes = [_vp, _P(zr_ipc_handle)]
@@ -268,6 +269,20 @@ def zr_state_reshard(target_plan: int, src_paths, dst_path: str) -> None:
     arr = (ctypes.c_char_p * max(1, len(src_paths)))(*[os.fsencode(p) for p in src_paths])
     _check(_lib.zr_state_reshard(target_plan, arr, len(src_paths), os.fsencode(dst_path)),
            "zr_state_reshard")
+
+
+ZR_EXPORT_F32 = 0
+ZR_EXPORT_BF16 = 1
+
+
+def zr_state_export_params(plan: int, src_paths, dtype: int, out_path: str) -> int:
+    """Writes the whole model's master weights (declaration order, raw fp32
+    or bf16) from a complete shard set; returns the element count."""
+    arr = (ctypes.c_char_p * max(1, len(src_paths)))(*[os.fsencode(p) for p in src_paths])
+    n = _i64()
+    _check(_lib.zr_state_export_params(plan, arr, len(src_paths), int(dtype), os.fsencode(out_path),
+                                       ctypes.byref(n)), "zr_state_export_params")
+    return n.value
 
 
 def zr_plan_owner_offsets(plan: int, world_size: int):

@@ -104,6 +104,75 @@ bool read_header(const char* path, ShardHeader* h, File* file) {
     return std::memcmp(h->magic, kMagic, 8) == 0 && h->version == kVersion;
 }
 
+// A complete set of shards of one partition, read and checked: the headers,
+// each rank's payload (master, m, v) and the partition's segments sorted by
+// global offset.
+struct ShardSet {
+    std::vector<ShardHeader> hs;
+    std::vector<std::vector<float>> payload;
+    std::vector<zr_segment> segs;
+};
+
+zr_status read_shard_set(const zr_plan& like, const char* const* src_paths, int32_t n_src, ShardSet* set) {
+    if (!src_paths || n_src < 1) return ZR_ERR_INVALID_ARG;
+    // Every source header: one complete partition of `like`'s tensors,
+    // ranks 0..n_src-1 in order, one step.
+    std::vector<ShardHeader>& hs = set->hs;
+    hs.resize(n_src);
+    for (int32_t r = 0; r < n_src; ++r) {
+        if (!src_paths[r]) return ZR_ERR_INVALID_ARG;
+        File f;
+        if (!read_header(src_paths[r], &hs[r], &f)) return f.f ? ZR_ERR_MISMATCH : ZR_ERR_IO;
+        if (hs[r].shapes_hash != shapes_hash(like) || hs[r].world_size != n_src || hs[r].rank != r ||
+            hs[r].mode != hs[0].mode || hs[r].partition_hash != hs[0].partition_hash || hs[r].step != hs[0].step ||
+            hs[r].total_numel != like.total_numel)
+            return ZR_ERR_MISMATCH;
+    }
+    // The source partition's segments, from a plan of the same tensors.
+    std::vector<int32_t> ndims(like.n_tensors, 1);
+    std::vector<const int64_t*> shape_ptrs(like.n_tensors);
+    for (int32_t t = 0; t < like.n_tensors; ++t) shape_ptrs[t] = &like.numel[t];
+    zr_plan* src_plan = nullptr;
+    zr_status st = zr_plan_create(like.n_tensors, ndims.data(), shape_ptrs.data(), n_src, 0,
+                                  static_cast<zr_partition>(hs[0].mode), 1ull << 62, &like.hp, &src_plan);
+    if (st != ZR_OK) return st;
+    std::unique_ptr<zr_plan, void (*)(zr_plan*)> guard(src_plan, zr_plan_destroy);
+    for (int32_t r = 0; r < n_src; ++r)
+        if (hs[r].owned_numel != src_plan->rank_numel[r] || hs[r].partition_hash != partition_hash(*src_plan))
+            return ZR_ERR_MISMATCH;
+    set->segs = src_plan->segments;
+    std::sort(set->segs.begin(), set->segs.end(),
+              [](const zr_segment& a, const zr_segment& b) { return a.global_offset < b.global_offset; });
+    // Each source payload is read once, whole, and its checksum verified.
+    set->payload.assign(n_src, {});
+    for (int32_t r = 0; r < n_src; ++r) {
+        const int64_t k = hs[r].owned_numel;
+        try {
+            set->payload[r].resize(static_cast<size_t>(3 * k));
+        } catch (...) {
+            return ZR_ERR_INVALID_ARG;
+        }
+        File f;
+        f.f = std::fopen(src_paths[r], "rb");
+        if (!f.f) return ZR_ERR_IO;
+        if (std::fseek(f.f, sizeof(ShardHeader), SEEK_SET) != 0) return ZR_ERR_IO;
+        const size_t bytes = sizeof(float) * static_cast<size_t>(3 * k);
+        if (k > 0 && std::fread(set->payload[r].data(), 1, bytes, f.f) != bytes) return ZR_ERR_IO;
+        if (fnv_words(kFnvOffset, set->payload[r].data(), bytes) != hs[r].payload_checksum) return ZR_ERR_MISMATCH;
+    }
+    return ZR_OK;
+}
+
+// Round to nearest, ties to even; a NaN stays a (quiet) NaN, overflow
+// rounds to infinity through the carry into the exponent.
+uint16_t bf16_rne(float x) {
+    uint32_t b;
+    std::memcpy(&b, &x, 4);
+    if ((b & 0x7fffffffu) > 0x7f800000u) return static_cast<uint16_t>((b >> 16) | 0x0040u);
+    b += 0x7fffu + ((b >> 16) & 1u);
+    return static_cast<uint16_t>(b >> 16);
+}
+
 }  // namespace
 
 extern "C" {
@@ -194,30 +263,12 @@ zr_status zr_state_load(const zr_plan* p, const char* path, float* master, float
 zr_status zr_state_reshard(const zr_plan* target, const char* const* src_paths, int32_t n_src,
                            const char* dst_path) {
     if (!target || !src_paths || n_src < 1 || !dst_path) return ZR_ERR_INVALID_ARG;
-    // Read every source header; they must form one complete partition of
-    // the target's tensors, ranks 0..n_src-1 in order.
-    std::vector<ShardHeader> hs(n_src);
-    for (int32_t r = 0; r < n_src; ++r) {
-        if (!src_paths[r]) return ZR_ERR_INVALID_ARG;
-        File f;
-        if (!read_header(src_paths[r], &hs[r], &f)) return f.f ? ZR_ERR_MISMATCH : ZR_ERR_IO;
-        if (hs[r].shapes_hash != shapes_hash(*target) || hs[r].world_size != n_src || hs[r].rank != r ||
-            hs[r].mode != hs[0].mode || hs[r].partition_hash != hs[0].partition_hash || hs[r].step != hs[0].step ||
-            hs[r].total_numel != target->total_numel)
-            return ZR_ERR_MISMATCH;
-    }
-    // The source partition's segments, from a plan of the same tensors.
-    std::vector<int32_t> ndims(target->n_tensors, 1);
-    std::vector<const int64_t*> shape_ptrs(target->n_tensors);
-    for (int32_t t = 0; t < target->n_tensors; ++t) shape_ptrs[t] = &target->numel[t];
-    zr_plan* src_plan = nullptr;
-    zr_status st = zr_plan_create(target->n_tensors, ndims.data(), shape_ptrs.data(), n_src, 0,
-                                  static_cast<zr_partition>(hs[0].mode), 1ull << 62, &target->hp, &src_plan);
+    ShardSet set;
+    zr_status st = read_shard_set(*target, src_paths, n_src, &set);
     if (st != ZR_OK) return st;
-    std::unique_ptr<zr_plan, void (*)(zr_plan*)> guard(src_plan, zr_plan_destroy);
-    for (int32_t r = 0; r < n_src; ++r)
-        if (hs[r].owned_numel != src_plan->rank_numel[r] || hs[r].partition_hash != partition_hash(*src_plan))
-            return ZR_ERR_MISMATCH;
+    const std::vector<ShardHeader>& hs = set.hs;
+    const std::vector<zr_segment>& src_segs = set.segs;
+    const std::vector<std::vector<float>>& payload = set.payload;
 
     // Global position -> (source rank, owned offset) for the target's owned
     // elements: walk the target's segments and, inside each, the source
@@ -228,26 +279,6 @@ zr_status zr_state_reshard(const zr_plan* target, const char* const* src_paths, 
         out.assign(static_cast<size_t>(3 * n), 0.0f);
     } catch (...) {
         return ZR_ERR_INVALID_ARG;
-    }
-    std::vector<zr_segment> src_segs = src_plan->segments;
-    std::sort(src_segs.begin(), src_segs.end(),
-              [](const zr_segment& a, const zr_segment& b) { return a.global_offset < b.global_offset; });
-    // Each source payload is read once, whole, and its checksum verified.
-    std::vector<std::vector<float>> payload(n_src);
-    for (int32_t r = 0; r < n_src; ++r) {
-        const int64_t k = hs[r].owned_numel;
-        try {
-            payload[r].resize(static_cast<size_t>(3 * k));
-        } catch (...) {
-            return ZR_ERR_INVALID_ARG;
-        }
-        File f;
-        f.f = std::fopen(src_paths[r], "rb");
-        if (!f.f) return ZR_ERR_IO;
-        if (std::fseek(f.f, sizeof(ShardHeader), SEEK_SET) != 0) return ZR_ERR_IO;
-        const size_t bytes = sizeof(float) * static_cast<size_t>(3 * k);
-        if (k > 0 && std::fread(payload[r].data(), 1, bytes, f.f) != bytes) return ZR_ERR_IO;
-        if (fnv_words(kFnvOffset, payload[r].data(), bytes) != hs[r].payload_checksum) return ZR_ERR_MISMATCH;
     }
     for (const zr_segment& t : target->segments) {
         if (t.owner != target->rank || t.tensor < 0) continue;   // the target's own pad stays 0
@@ -297,6 +328,50 @@ zr_status zr_state_reshard(const zr_plan* target, const char* const* src_paths, 
         if (std::fflush(o.f) != 0) return ZR_ERR_IO;
     }
     if (std::rename(tmp.c_str(), dst_path) != 0) return ZR_ERR_IO;
+    return ZR_OK;
+}
+
+zr_status zr_state_export_params(const zr_plan* plan, const char* const* src_paths, int32_t n_src, int32_t dtype,
+                                 const char* out_path, int64_t* n_written) {
+    if (!plan || !src_paths || n_src < 1 || !out_path) return ZR_ERR_INVALID_ARG;
+    if (dtype != ZR_EXPORT_F32 && dtype != ZR_EXPORT_BF16) return ZR_ERR_INVALID_ARG;
+    ShardSet set;
+    zr_status st = read_shard_set(*plan, src_paths, n_src, &set);
+    if (st != ZR_OK) return st;
+    // Every tensor element has exactly one source segment; the pad (tensor
+    // -1) is not a parameter and is left out.
+    const int64_t N = plan->total_numel;
+    const size_t elem = dtype == ZR_EXPORT_BF16 ? 2 : 4;
+    std::vector<unsigned char> out;
+    try {
+        out.assign(static_cast<size_t>(N) * elem, 0);
+    } catch (...) {
+        return ZR_ERR_INVALID_ARG;
+    }
+    int64_t covered = 0;
+    for (const zr_segment& sg : set.segs) {
+        if (sg.tensor < 0) continue;
+        if (sg.global_offset < 0 || sg.global_offset + sg.length > N) return ZR_ERR_MISMATCH;
+        const float* src = set.payload[sg.owner].data() + sg.owned_offset;   // master: the first third
+        if (dtype == ZR_EXPORT_F32) {
+            std::memcpy(out.data() + 4 * sg.global_offset, src, 4 * static_cast<size_t>(sg.length));
+        } else {
+            uint16_t* dst = reinterpret_cast<uint16_t*>(out.data()) + sg.global_offset;
+            for (int64_t j = 0; j < sg.length; ++j) dst[j] = bf16_rne(src[j]);
+        }
+        covered += sg.length;
+    }
+    if (covered != N) return ZR_ERR_MISMATCH;
+    const std::string tmp = std::string(out_path) + ".tmp";
+    {
+        File o;
+        o.f = std::fopen(tmp.c_str(), "wb");
+        if (!o.f) return ZR_ERR_IO;
+        if (N > 0 && std::fwrite(out.data(), 1, out.size(), o.f) != out.size()) return ZR_ERR_IO;
+        if (std::fflush(o.f) != 0) return ZR_ERR_IO;
+    }
+    if (std::rename(tmp.c_str(), out_path) != 0) return ZR_ERR_IO;
+    if (n_written) *n_written = N;
     return ZR_OK;
 }
 

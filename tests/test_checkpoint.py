@@ -118,3 +118,64 @@ def test_reshard_rejects_inconsistent_sets(tmp_path):
         assert not os.path.exists(out)
     finally:
         zr.zr_plan_destroy(h)
+
+
+SPECIAL = np.array([0x3F808000, 0x3F818000, 0x3F80C000, 0x80000000, 0x00000001, 0x807FFFFF, 0x7F7FFFFF,
+                    0xFF7FFFFF, 0x7F800000, 0xFF800000, 0x7FC00000, 0xFF812345, 0x7F800001, 0x3F7FFFFF],
+                   dtype=np.uint32).view(np.float32)
+
+
+@pytest.mark.parametrize("W, mode", [(4, 0), (3, 1), (1, 0), (8, 0)])
+def test_export_params_gathers_the_whole_model(tmp_path, W, mode):
+    """zr_state_export_params: the whole model's master weights in
+    declaration order from a shard set, as fp32 (the unsharded state bit for
+    bit) and as bf16 (the oracle's RNE of it); special values -- ties,
+    signed zeros, subnormals, the largest finite values, infinities and NaNs
+    -- are planted in the state to pin the rounding."""
+    N, master, m, v = unsharded_state()
+    master = master.copy()
+    pos = np.random.default_rng(W * 10 + mode).choice(N, size=SPECIAL.size, replace=False)
+    master[pos] = SPECIAL
+    paths = write_partition(str(tmp_path), (N, master, m, v), W, mode, 2, "src")
+    h = zr.zr_plan_create(SHAPES, 2, 1, 1 - mode, 4096)      # any plan of the same tensors
+    try:
+        f32 = os.path.join(str(tmp_path), "model_f32.bin")
+        b16 = os.path.join(str(tmp_path), "model_bf16.bin")
+        assert zr.zr_state_export_params(h, paths, zr.ZR_EXPORT_F32, f32) == N
+        assert zr.zr_state_export_params(h, paths, zr.ZR_EXPORT_BF16, b16) == N
+    finally:
+        zr.zr_plan_destroy(h)
+    got32 = np.fromfile(f32, dtype="<u4")
+    got16 = np.fromfile(b16, dtype="<u2")
+    assert got32.size == N and got16.size == N
+    assert np.array_equal(got32, master.view(np.uint32))
+    want16 = oracle.f32_to_bf16_array(master)
+    nan = np.isnan(master)
+    assert np.array_equal(got16[~nan], want16[~nan])
+    # a NaN stays a NaN of the same sign
+    assert np.all((got16[nan] & 0x7F80) == 0x7F80) and np.all(got16[nan] & 0x007F)
+    assert np.array_equal(got16[nan] >> 15, want16[nan] >> 15)
+
+
+def test_export_params_rejects_bad_sets(tmp_path):
+    state = unsharded_state(steps=1)
+    paths = write_partition(str(tmp_path), state, 3, 0, 1, "a")
+    h = zr.zr_plan_create(SHAPES, 3, 0, 0, 4096)
+    out = os.path.join(str(tmp_path), "model.bin")
+    try:
+        with pytest.raises(zr.ZrError) as e:
+            zr.zr_state_export_params(h, paths[:2], zr.ZR_EXPORT_BF16, out)
+        assert e.value.status == zr.ZR_ERR_MISMATCH
+        with pytest.raises(zr.ZrError) as e:
+            zr.zr_state_export_params(h, paths, 7, out)
+        assert e.value.status == zr.ZR_ERR_INVALID_ARG
+        hx = zr.zr_plan_create([(10,), (20,)], 2, 0, 0, 4096)
+        try:
+            with pytest.raises(zr.ZrError) as e:
+                zr.zr_state_export_params(hx, paths, zr.ZR_EXPORT_F32, out)
+            assert e.value.status == zr.ZR_ERR_MISMATCH
+        finally:
+            zr.zr_plan_destroy(hx)
+        assert not os.path.exists(out)
+    finally:
+        zr.zr_plan_destroy(h)

@@ -57,6 +57,13 @@ def test_elastic_resume_on_another_partition(tmp_path):
         p = os.path.join(str(tmp_path), f"w4_r{r}.zrs")
         zr.zr_state_save(g.plan.handle, p, g.master, g.m, g.v, steps)
         paths.append(p)
+    # gather to a whole model on save: the bf16 export of the shard set is
+    # the all-gather buffer the step wrote, bit for bit
+    full = os.path.join(str(tmp_path), "model_bf16.bin")
+    N = zr.zr_state_export_params(src[0].plan.handle, paths, zr.ZR_EXPORT_BF16, full)
+    torch.cuda.synchronize()
+    assert np.array_equal(np.fromfile(full, dtype="<u2"),
+                          out[:N].cpu().view(torch.int16).numpy().view(np.uint16))
     # resume on W = 3, whole-tensor ownership
     dst = []
     for r in range(3):
