@@ -9,12 +9,15 @@ the fp32 master / m / v, and the bf16 write into the all-gather buffer.
 Inputs are seeded synthetic data resident in HBM before the timed region;
 each step's bytes exceed the 126 MB L2, so no flush is needed between steps.
 
-N > 1 (torchrun, one process per GPU): process i runs ZeRO rank i mod W of
-the same workload on its own GPU -- independent shards, no data-path
+N > 1 (torchrun, one process per GPU): process i runs ZeRO rank (r0 + i) mod
+W of the same workload (r0: the workload's timed rank) on its own GPU -- independent shards, no data-path
 collective (weak scaling); the step time is the max over processes.
 
---impl reference times the oracle (plain single-threaded C on the host) on a
-bounded sample of the same workload and prints the same JSON line.
+--impl reference times the oracle (plain C on the host, unchanged) on a
+bounded sample of the same workload, split into disjoint slices stepped by
+--cpu-threads host threads (default: every core the process may use), and
+prints the same JSON line.  The GPU arm's cpu_baseline is the same
+measurement, with the one-thread rate beside it.
 """
 from __future__ import annotations
 
@@ -50,6 +53,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--cpu-threads", type=int, default=0,
+                    help="host threads for the oracle baseline (0: every core this process may use, at most 32)")
     ap.add_argument("--per-bucket", action="store_true",
                     help="step bucket by bucket (zr_step_bucket per bucket, then zr_step_finish)")
     ap.add_argument("--overlap", action="store_true",
@@ -57,7 +62,10 @@ def parse():
                          "after it, against zr_step_bucket as each bucket's gradients complete")
     ap.add_argument("--sweep", action="store_true",
                     help="1.3B set: bucket cap x W x partition; one JSON record per point")
-    return ap.parse_args()
+    args = ap.parse_args()
+    if args.cpu_threads <= 0:
+        args.cpu_threads = host_threads()
+    return args
 
 
 def workload(name):
@@ -198,15 +206,16 @@ class OracleSample:
     elements with the workload's gradient statistics, as their own W-replica
     flat plan of one tensor."""
 
-    def __init__(self, wl, rank, max_elems):
+    def __init__(self, wl, rank, max_elems, offset=0):
         import numpy as np
         import oracle
         import synth
         import torch
         oplan = oracle.Plan(wl.shapes, wl.world_size, wl.mode, wl.bucket_cap_bytes)
-        self.n = n = min(int(oplan.owned_numel[rank]), max_elems)
         self.owned = int(oplan.owned_numel[rank])
-        idx = torch.from_numpy(oplan.owned_global_index(rank)[:n])
+        offset = min(offset, self.owned)
+        self.n = n = min(self.owned - offset, max_elems)
+        idx = torch.from_numpy(oplan.owned_global_index(rank)[offset:offset + n])
         self.grads = [synth.grad_bf16(wl.seed, 1, w, idx, wl.grad_sigma, wl.outlier_frac,
                                       n_valid=oplan.total_numel).view(torch.int16).numpy()
                       .view(np.uint16).copy() for w in range(wl.world_size)]
@@ -217,12 +226,12 @@ class OracleSample:
         self.out = np.zeros(self.plan.padded_numel, np.uint16)
         self.wl, self.rank, self.t = wl, rank, 0
 
-    def run(self, target_seconds):
-        """Oracle steps on the sample until `target_seconds` of CPU work;
-        returns (Gparams/s, description)."""
+    def steps_until(self, deadline):
+        """Oracle steps on the sample until perf_counter() passes `deadline`;
+        returns the number of steps."""
         import oracle
         clip = 1.0 if self.wl.max_grad_norm > 0 else None
-        steps, t0 = 0, time.perf_counter()
+        steps = 0
         while True:
             self.t += 1
             oracle.rank_step(self.plan, 0, self.grads, self.master, self.m, self.v, self.out,
@@ -230,16 +239,65 @@ class OracleSample:
             if clip is not None:
                 oracle.sumsq(oracle.reduce(self.grads))      # the clip's extra reduce pass
             steps += 1
-            el = time.perf_counter() - t0
-            if el >= target_seconds:
-                break
-        desc = (f"oracle rank_step on {self.n} of rank {self.rank}'s {self.owned} owned params "
-                f"(W={self.wl.world_size}), {steps} steps, {el:.1f} s, 1 thread")
-        return self.n * steps / el / 1e9, desc
+            if time.perf_counter() >= deadline:
+                return steps
 
 
-def oracle_sample_rate(wl, rank, target_seconds, max_elems=1 << 21):
-    return OracleSample(wl, rank, max_elems).run(target_seconds)
+class OracleSamples:
+    """`threads` disjoint samples of one rank's shard (consecutive slices of
+    its owned elements), one per host thread.  The oracle's C calls release
+    the interpreter lock and share no state, so the threads step their
+    slices in parallel; the oracle itself is unchanged."""
+
+    def __init__(self, wl, rank, max_elems, threads):
+        self.threads = max(1, int(threads))
+        per = max(1, max_elems // self.threads)
+        self.samples = [OracleSample(wl, rank, per, offset=i * per) for i in range(self.threads)]
+        self.samples = [x for x in self.samples if x.n > 0] or self.samples[:1]
+        self.threads = len(self.samples)
+        self.wl, self.rank, self.owned = wl, rank, self.samples[0].owned
+
+    def run(self, target_seconds):
+        """Every thread steps its slice until `target_seconds` have passed;
+        returns (Gparams/s over all threads, description)."""
+        import concurrent.futures as cf
+        t0 = time.perf_counter()
+        deadline = t0 + target_seconds
+        if self.threads == 1:
+            counts = [self.samples[0].steps_until(deadline)]
+        else:
+            with cf.ThreadPoolExecutor(max_workers=self.threads) as ex:
+                counts = list(ex.map(lambda x: x.steps_until(deadline), self.samples))
+        el = time.perf_counter() - t0
+        done = sum(x.n * c for x, c in zip(self.samples, counts))
+        n = sum(x.n for x in self.samples)
+        desc = (f"oracle rank_step on {n} of rank {self.rank}'s {self.owned} owned params "
+                f"(W={self.wl.world_size}) in {self.threads} slice(s), {min(counts)}-{max(counts)} "
+                f"steps each, {el:.1f} s, {self.threads} thread(s)")
+        return done / el / 1e9, desc
+
+
+def host_threads():
+    """Host cores this process may run on (at most 32)."""
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    return max(1, min(32, n))
+
+
+def cpu_baseline(wl, rank, seconds, threads, max_elems=1 << 21):
+    """The oracle on a bounded sample of the workload: all `threads` host
+    threads over disjoint slices (the reported value, `cores` = threads),
+    and the same sample on one thread beside it."""
+    multi = OracleSamples(wl, rank, max_elems, threads)
+    rate, desc = multi.run(seconds / 2 if multi.threads > 1 else seconds)
+    out = {"value": rate, "unit": UNIT, "cores": multi.threads, "kind": "oracle", "sample": desc}
+    if multi.threads > 1:
+        one = OracleSamples(wl, rank, max_elems, 1)
+        r1, d1 = one.run(seconds / 2)
+        out["single_thread"] = {"value": r1, "sample": d1}
+    return out
 
 
 def run_reference(args):
@@ -249,7 +307,7 @@ def run_reference(args):
     wl = workload(args.config)
     K, Wm = args.steps, args.warmup
     budget = max(0.05, min(2.0, 120.0 / max(1, K + Wm)))
-    sample = OracleSample(wl, wl.ranks[0], 1 << 18)
+    sample = OracleSamples(wl, wl.ranks[0], 1 << 18, args.cpu_threads)
     rates = []
     desc = ""
     for i in range(Wm + K):
@@ -264,7 +322,8 @@ def run_reference(args):
         "config": {"workload": wl.name, "W": wl.world_size,
                    "rank": wl.ranks[0], "partition": "flat" if wl.mode == 0 else "whole_tensor",
                    "bucket_cap_mb": wl.bucket_cap_mb},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": sample.threads, "kind": "oracle",
+                         "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -408,8 +467,7 @@ def run_zr(args):
 
     cpu = None
     if grank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, desc = oracle_sample_rate(wl, zr_rank, args.cpu_seconds)
-        cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
+        cpu = cpu_baseline(wl, zr_rank, args.cpu_seconds, args.cpu_threads)
 
     if dist:
         dist.barrier(device_ids=[local])

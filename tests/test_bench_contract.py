@@ -12,7 +12,7 @@ from conftest import ROOT
 
 def test_reference_arm_prints_one_json_line():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                          "--steps", "2", "--warmup", "1"], capture_output=True, text=True,
+                          "--steps", "2", "--warmup", "1", "--cpu-threads", "2"], capture_output=True, text=True,
                          timeout=600, cwd=ROOT)
     assert out.returncode == 0, out.stderr[-2000:]
     lines = [l for l in out.stdout.splitlines() if l.strip()]
@@ -23,7 +23,8 @@ def test_reference_arm_prints_one_json_line():
         assert k in d, k
     assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "Gparams/s"
     assert d["config"]["workload"] == bench.DEFAULT_CONFIG
-    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 2
+    assert "2 thread(s)" in d["cpu_baseline"]["sample"] and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
     assert d["value"] > 0
 
@@ -42,3 +43,19 @@ def test_shard_rank_and_workloads():
     assert [bench.shard_rank(wl, i, 8) for i in range(8)] == [3, 4, 5, 6, 7, 0, 1, 2]
     assert bench.workload("gpt2_124m_w8").world_size == 8
     assert len(synth.sweep_workloads()) == 40
+
+
+def test_threaded_oracle_sample_covers_disjoint_slices():
+    wl = synth.WORKLOADS["tiny"]
+    multi = bench.OracleSamples(wl, 0, 1 << 12, 4)
+    assert multi.threads == 4 and [x.n for x in multi.samples] == [1024] * 4
+    # consecutive, disjoint slices of the rank's owned elements
+    import oracle
+    oplan = oracle.Plan(wl.shapes, wl.world_size, wl.mode, wl.bucket_cap_bytes)
+    idx = oplan.owned_global_index(0)
+    one = bench.OracleSample(wl, 0, 4096)
+    for i, x in enumerate(multi.samples):
+        assert (x.master == one.master[i * 1024:(i + 1) * 1024]).all()
+    rate, desc = multi.run(0.2)
+    assert rate > 0 and "4 thread(s)" in desc
+    assert idx.size == multi.owned
