@@ -61,24 +61,36 @@ zr_status check_state(const float* master, const float* m, const float* v) {
     return ZR_OK;
 }
 
+void release_host_pipeline(const zr_plan* p) {
+    for (cudaEvent_t& e : p->host_events) {
+        if (e) cudaEventDestroy(e);
+        e = nullptr;
+    }
+    if (p->h2d_stream) cudaStreamDestroy(p->h2d_stream);
+    if (p->d2h_stream) cudaStreamDestroy(p->d2h_stream);
+    p->h2d_stream = p->d2h_stream = nullptr;
+    p->host_pipeline_ready = false;
+}
+
+// The copy streams and events of zr_step_host, created on first use; a
+// failure part way releases what was created, so a later call starts over.
 zr_status ensure_host_pipeline(const zr_plan* p) {
     if (p->host_pipeline_ready) return ZR_OK;
-    if (cudaStreamCreateWithFlags(&p->h2d_stream, cudaStreamNonBlocking) != cudaSuccess) return ZR_ERR_CUDA;
-    if (cudaStreamCreateWithFlags(&p->d2h_stream, cudaStreamNonBlocking) != cudaSuccess) return ZR_ERR_CUDA;
+    bool ok = cudaStreamCreateWithFlags(&p->h2d_stream, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&p->d2h_stream, cudaStreamNonBlocking) == cudaSuccess;
     for (cudaEvent_t& e : p->host_events)
-        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return ZR_ERR_CUDA;
+        ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+        release_host_pipeline(p);
+        return ZR_ERR_CUDA;
+    }
     p->host_pipeline_ready = true;
     return ZR_OK;
 }
 
 }  // namespace
 
-zr_plan::~zr_plan() {
-    for (cudaEvent_t e : host_events)
-        if (e) cudaEventDestroy(e);
-    if (h2d_stream) cudaStreamDestroy(h2d_stream);
-    if (d2h_stream) cudaStreamDestroy(d2h_stream);
-}
+zr_plan::~zr_plan() { release_host_pipeline(this); }
 
 extern "C" {
 
