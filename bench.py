@@ -46,7 +46,7 @@ PROFILES = os.path.join(ROOT, "profiles")
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="zr", choices=["zr", "reference"])
     ap.add_argument("--config", default=DEFAULT_CONFIG)
@@ -157,28 +157,35 @@ class ClockSampler:
         except Exception:
             self._ok = False
 
-    def _run(self):
+    def _sample(self):
         nv = self._nv
-        names = {
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            for k, bit in self._names.items():
+                if r & bit:
+                    self.reasons.add(k)
+        except Exception:
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(0.002)
+
+    def _reason_bits(self):
+        nv = self._nv
+        return {
             "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
             "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
             "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
             "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
             "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
         }
-        while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-                for k, bit in names.items():
-                    if r & bit:
-                        self.reasons.add(k)
-            except Exception:
-                pass
-            time.sleep(0.002)
 
     def __enter__(self):
         if self._ok:
+            self._names = self._reason_bits()
             self._t = threading.Thread(target=self._run, daemon=True)
             self._t.start()
         return self
@@ -187,6 +194,10 @@ class ClockSampler:
         if self._ok:
             self._stop.set()
             self._t.join()
+            if not self.samples:
+                # a region shorter than one NVML round trip: read the clocks
+                # as it ends, the device having just drained the timed work
+                self._sample()
 
     def summary(self):
         if not self._ok:

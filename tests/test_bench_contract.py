@@ -59,3 +59,48 @@ def test_threaded_oracle_sample_covers_disjoint_slices():
     rate, desc = multi.run(0.2)
     assert rate > 0 and "4 thread(s)" in desc
     assert idx.size == multi.owned
+
+
+class _FakeNvml:
+    """Stands in for pynvml: a fixed SM clock and throttle-reason mask."""
+    NVML_CLOCK_SM = 1
+    nvmlClocksEventReasonSwPowerCap = 0x4
+    nvmlClocksEventReasonHwSlowdown = 0x8
+
+    def __init__(self, mhz, reasons):
+        self.mhz, self.mask, self.calls = mhz, reasons, 0
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return i
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        self.calls += 1
+        return self.mhz
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return self.mask
+
+
+def test_clock_sampler_against_a_fake_nvml(monkeypatch):
+    import time
+    fake = _FakeNvml(1800, 0x4 | 0x8)
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    with bench.ClockSampler(0) as s:
+        time.sleep(0.05)
+    out = s.summary()
+    assert out["sm_mhz"] == 1800 and out["sm_max_mhz"] == 1965 and out["samples"] >= 1
+    assert out["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    # a region too short for the thread's first read still gets one, at its end
+    fake2 = _FakeNvml(1965, 0)
+    monkeypatch.setitem(sys.modules, "pynvml", fake2)
+    s2 = bench.ClockSampler(0)
+    s2._run = lambda: None
+    with s2:
+        pass
+    assert s2.summary()["samples"] == 1 and s2.summary()["reasons"] == []
