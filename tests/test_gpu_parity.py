@@ -93,9 +93,35 @@ def test_tiny_both_ranks_three_steps():
     ([(7, 1024), (100,)], 16, 0, 1 << 20),                 # W = 16
     ([(5000,), (300,)], 33, 0, 1 << 20),                   # W = 33: a partial second load group
     ([(4096,), (512,)], 64, 1, 1 << 20),                   # W = 64, whole-tensor, empty ranks
+    ([(0,), (100,), (3, 0), (2050,)], 2, 0, 4096),         # zero-element tensors among the rest
+    ([(0,), (100,), (3, 0), (2050,)], 3, 1, 4096),         # same, whole-tensor: rank 2 owns nothing
 ])
 def test_edge_shapes(shapes, W, mode, cap):
     run_all_ranks(shapes, W, mode, cap, 2, 1e-3, 0.01)
+
+
+@pytest.mark.parametrize("shapes", [[], [(0,)], [(0,), (3, 0)]])
+@pytest.mark.parametrize("clip", [0.0, 1.0])
+def test_sets_without_parameters(shapes, clip):
+    """No parameters at all (no tensors, or only zero-element ones): every
+    step call succeeds without touching memory, and a device step count
+    still advances."""
+    import sharded_optimizer_step_zr_b200 as zr
+    from sharded_optimizer_step_zr_b200.plan import ZrPlan
+    plan = ZrPlan(shapes, 2, 1, 0, 4096, *HP[:5], max_grad_norm=clip, device=DEV)
+    assert (plan.total_numel, plan.padded_numel, plan.owned_numel) == (0, 0, 0)
+    e16 = torch.empty(0, dtype=torch.bfloat16, device=DEV)
+    e32 = torch.empty(0, dtype=torch.float32, device=DEV)
+    plan.step([e16, e16], e32, e32, e32, e16, 1)
+    for b in range(plan.n_buckets):
+        plan.step_bucket(b, [e16, e16], e32, e32, e32, e16, 1)
+    plan.step_finish([e16, e16], e32, e32, e32, e16, 1)
+    d_step = torch.zeros(1, dtype=torch.int64, device=DEV)
+    for _ in range(3):
+        zr.zr_step_device_count(plan.handle, [e16, e16], e32, e32, e32, e16, d_step)
+    torch.cuda.synchronize()
+    assert d_step.item() == 3
+    plan.close()
 
 
 def test_max_world_size():
