@@ -297,13 +297,26 @@ def host_threads():
     return max(1, min(32, n))
 
 
+def cpu_model():
+    """The host CPU's model name, as the kernel reports it (None if unknown)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def cpu_baseline(wl, rank, seconds, threads, max_elems=1 << 21):
     """The oracle on a bounded sample of the workload: all `threads` host
     threads over disjoint slices (the reported value, `cores` = threads),
     and the same sample on one thread beside it."""
     multi = OracleSamples(wl, rank, max_elems, threads)
     rate, desc = multi.run(seconds / 2 if multi.threads > 1 else seconds)
-    out = {"value": rate, "unit": UNIT, "cores": multi.threads, "kind": "oracle", "sample": desc}
+    out = {"value": rate, "unit": UNIT, "cores": multi.threads, "kind": "oracle", "sample": desc,
+           "cpu": cpu_model()}
     if multi.threads > 1:
         one = OracleSamples(wl, rank, max_elems, 1)
         r1, d1 = one.run(seconds / 2)
@@ -334,7 +347,7 @@ def run_reference(args):
                    "rank": wl.ranks[0], "partition": "flat" if wl.mode == 0 else "whole_tensor",
                    "bucket_cap_mb": wl.bucket_cap_mb},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": sample.threads, "kind": "oracle",
-                         "sample": desc},
+                         "sample": desc, "cpu": cpu_model()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
