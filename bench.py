@@ -124,16 +124,19 @@ def kernel_source_hash():
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def recorded_traffic(workload_name):
-    """dram__bytes_read.sum + dram__bytes_write.sum per launch of the step's
-    dominant kernel from the committed ncu summary, if it was taken on the
-    current kernel source; else None."""
+def recorded_traffic(workload_name, clip):
+    """dram__bytes_read.sum + dram__bytes_write.sum from the committed ncu
+    record of the workload, if it was taken on the current kernel source,
+    else None: per launch of zr_tile_kernel for a step without clipping, per
+    step (its three launches) with clipping -- the same unit as the line's
+    `achieved`."""
+    name = f"zr_clip_step_{workload_name}" if clip else f"zr_tile_kernel_{workload_name}"
     try:
-        with open(os.path.join(PROFILES, f"zr_tile_kernel_{workload_name}_traffic.json")) as f:
+        with open(os.path.join(PROFILES, f"{name}_traffic.json")) as f:
             d = json.load(f)
         e = d.get(workload_name)
         if e and e.get("kernel_source_sha256_16") == kernel_source_hash():
-            return float(e["bytes_per_launch"])
+            return float(e["bytes_per_step"] if clip else e["bytes_per_launch"])
     except Exception:
         pass
     return None
@@ -462,7 +465,8 @@ def run_zr(args):
     avg_ms = local_ms / K
     achieved = alg_bytes / (avg_ms * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
-    traffic = recorded_traffic(wl.name)
+    # (bucket-by-bucket steps launch per bucket: no per-launch record)
+    traffic = None if args.per_bucket else recorded_traffic(wl.name, clip)
 
     # end to end through zr_step_host: pinned host gradients in, result out
     e2e = None

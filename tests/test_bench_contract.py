@@ -104,3 +104,18 @@ def test_clock_sampler_against_a_fake_nvml(monkeypatch):
     with s2:
         pass
     assert s2.summary()["samples"] == 1 and s2.summary()["reasons"] == []
+
+
+def test_recorded_traffic_is_close_to_the_algorithmic_bytes():
+    """The committed ncu DRAM records, taken on the current kernel source,
+    stay within a few percent of the algorithmic bytes (no re-reads); a
+    write-back still in L2 when the kernel ends makes them a little lower."""
+    from sharded_optimizer_step_zr_b200.plan import ZrPlan
+    for name, clip in (("gpt2_124m_w8", False), ("llama_7b_w64", False), ("gpt_1p3b_w8_whole_clip", True)):
+        wl = synth.WORKLOADS[name]
+        t = bench.recorded_traffic(name, clip)
+        assert t is not None, name
+        plan = ZrPlan(wl.shapes, wl.world_size, wl.ranks[0], wl.mode, wl.bucket_cap_bytes, *wl.hp, bind=False)
+        alg = plan.owned_numel * bench.bytes_per_owned_param(wl.world_size, clip)
+        plan.close()
+        assert 0.9 * alg <= t <= 1.02 * alg, (name, t, alg)
