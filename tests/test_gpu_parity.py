@@ -124,6 +124,44 @@ def test_sets_without_parameters(shapes, clip):
     plan.close()
 
 
+@pytest.mark.parametrize("t0", [1000, 10 ** 6, 2 ** 33 + 5])
+def test_large_step_numbers(t0):
+    """Three steps from step number t0 (bias corrections near or exactly 1;
+    2**33 + 5 needs the 64-bit step), eager zr_step and the device-resident
+    count (preset to t0 - 1) each against the oracle, bit for bit."""
+    import sharded_optimizer_step_zr_b200 as zr
+    shapes = [(4096 * 2 + 13,), (300, 3)]
+    W = 4
+    oplan = oracle.Plan(shapes, W, 0, 1 << 20)
+    P = oplan.padded_numel
+    for r in (0, W - 1):
+        eager = GpuRank(shapes, W, r, 0, 1 << 20, HP, seed=77)
+        counted = GpuRank(shapes, W, r, 0, 1 << 20, HP, seed=77)
+        orc = OracleRank(oplan, r, seed=77)
+        out_e = torch.zeros(P, dtype=torch.bfloat16, device=DEV)
+        out_c = torch.zeros(P, dtype=torch.bfloat16, device=DEV)
+        out_o = np.zeros(P, np.uint16)
+        d_step = torch.full((1,), t0 - 1, dtype=torch.int64, device=DEV)
+        for k in range(3):
+            # gradients from generator steps 1..3; optimizer step numbers t0..t0+2
+            eager.fill_grads(k + 1, 1e-3, 0.01)
+            counted.fill_grads(k + 1, 1e-3, 0.01)
+            orc.make_grads(k + 1, 1e-3, 0.01)
+            eager.step(out_e, t0 + k)
+            zr.zr_step_device_count(counted.plan.handle, counted.grads, counted.master, counted.m, counted.v,
+                                    out_c, d_step)
+            orc.step(out_o, HP, t0 + k)
+        torch.cuda.synchronize()
+        assert d_step.item() == t0 + 2
+        for g in (eager, counted):
+            for got, want in zip(g.state(), (orc.master, orc.m, orc.v)):
+                assert np.array_equal(bits32(got), bits32(want)), (t0, r)
+        mine = oplan.owned_global_index(r)
+        mine = mine[mine < oplan.total_numel]
+        for out in (out_e, out_c):
+            assert np.array_equal(u16(out)[mine], out_o[mine])
+
+
 def test_max_world_size():
     """W = 512, the ABI's maximum (the pointer array's largest instantiation):
     first, middle and last rank."""

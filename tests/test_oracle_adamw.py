@@ -93,3 +93,28 @@ def test_scalars_follow_their_definitions():
         abs(s["step_size"] - 3e-4 / (1 - np.float64(np.float32(0.9)) ** 2)) < 1e-10
     assert abs(s["bc2_sqrt"] - np.sqrt(1 - np.float64(np.float32(0.999)) ** 2)) < 1e-7
     assert abs(s["decay"] - (1 - 3e-4 * 0.1)) < 1e-7
+
+
+@pytest.mark.parametrize("t", [10 ** 6, 2 ** 33 + 5])
+def test_bias_corrections_vanish_at_large_steps(t):
+    """At these step numbers β1^t and β2^t (β2 = 0.999: below e^-999) are
+    below the smallest fp64 subnormal, so both bias corrections are exactly
+    1: step_size is fp32(lr) and sqrt(1 - β2^t) is 1.  The step number is a
+    64-bit integer: 2**33 + 5 cut to 32 bits would be step 5, whose
+    corrections are far from 1."""
+    s = oracle.adamw_scalars(HP, t)
+    assert s["step_size"] == np.float32(3e-4)
+    assert s["bc2_sqrt"] == 1.0
+    # the element step is then AdamW without bias correction
+    g = np.array([1e-3, -2e-2, 0.0], np.float32)
+    p = np.array([0.5, -0.25, 1.0], np.float32)
+    m = np.array([2e-4, -1e-3, 0.0], np.float32)
+    v = np.array([3e-7, 4e-4, 0.0], np.float32)
+    p64, m64, v64 = p.astype(np.float64), m.astype(np.float64), v.astype(np.float64)
+    b1, b2 = np.float64(np.float32(0.9)), np.float64(np.float32(0.999))
+    m_new = b1 * m64 + (1 - b1) * g
+    v_new = b2 * v64 + (1 - b2) * g.astype(np.float64) ** 2
+    want = p64 * (1 - 3e-4 * 0.1) - 3e-4 * m_new / (np.sqrt(v_new) + 1e-8)
+    oracle.adamw(HP, t, g, p, m, v)
+    assert np.allclose(p, want, rtol=2e-6, atol=1e-9)
+    assert np.allclose(m, m_new, rtol=2e-6, atol=1e-12) and np.allclose(v, v_new, rtol=2e-6, atol=1e-15)
