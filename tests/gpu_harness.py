@@ -90,7 +90,8 @@ def assert_state_close(got, want, what):
     got = np.asarray(got, dtype=np.float64)
     want = np.asarray(want, dtype=np.float64)
     both_nan = np.isnan(got) & np.isnan(want)
-    ok = both_nan | (np.abs(got - want) <= 1e-9 + 2e-6 * np.abs(want)) | (got == want)
+    with np.errstate(invalid="ignore"):           # inf - inf: decided by got == want
+        ok = both_nan | (np.abs(got - want) <= 1e-9 + 2e-6 * np.abs(want)) | (got == want)
     if not ok.all():
         bad = np.flatnonzero(~ok)[:5]
         raise AssertionError(f"{what}: {(~ok).sum()} mismatches, e.g. at {bad}: got {got[bad]} want {want[bad]}")
