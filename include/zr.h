@@ -351,6 +351,47 @@ zr_status zr_state_reshard(const zr_plan* target, const char* const* src_paths, 
 zr_status zr_state_export_params(const zr_plan* plan, const char* const* src_paths, int32_t n_src,
                                  int32_t dtype, const char* out_path, int64_t* n_written);
 
+/* Checked mode: a stand-in for a memory sanitizer at run time.  The plan's
+ * tile tables live in the caller's workspace, so a kernel that writes there
+ * by mistake (a race on the workspace, a stray pointer) would send the next
+ * step to wrong or out-of-bounds addresses.  The pages have no counterpart;
+ * it follows from this library's caller-owned workspace.
+ *
+ * zr_plan_verify enqueues on `stream` two kernels that test every tile of
+ * both device tables against the invariants the planner guarantees (length
+ * 1..2048, owned and global ranges inside the rank's owned count and
+ * padded_numel, 16-byte vector flags only where the alignment holds, bucket
+ * and index in range, each bucket-order tile at its own index) and compare
+ * an order-independent 64-bit hash of each table with the one taken on the
+ * host when zr_plan_set_workspace uploaded it.  If anything fails, now or at
+ * an earlier check, both tables are overwritten with empty tiles, so the
+ * steps queued after it update nothing and write nothing (their results
+ * are then missing, not wrong); zr_plan_set_workspace re-uploads the tables
+ * and clears the status.  Nothing waits on anything; a check costs two
+ * small launches reading 64 bytes per tile.
+ * zr_plan_set_checked(plan, 1) makes every call that launches the tile
+ * kernels (zr_step, zr_step_device_count, zr_step_bucket, zr_step_finish,
+ * zr_step_host, zr_grad_sumsq, zr_debug_reduce) run that check first on its
+ * stream; 0 (the default) turns it off.  zr_step_no_alloc uploads its own
+ * table on every call and is not affected.
+ * zr_plan_check_result synchronises `stream` and reads the status:
+ * bad_tiles = tiles that failed an invariant (both tables, counted at every
+ * check since the workspace was bound), first_bad = the smallest failing
+ * position (i for the bucket-order table, n_tiles + i for the owned-order
+ * one) or -1, hash_mismatch = bit 0 for the bucket-order table, bit 1 for
+ * the owned-order one, tables_emptied = 1 once a failure has emptied them.
+ * Errors: ZR_ERR_INVALID_ARG, ZR_ERR_NO_WORKSPACE, ZR_ERR_CUDA. */
+typedef struct {
+    uint64_t bad_tiles;
+    int64_t first_bad;
+    uint32_t hash_mismatch;
+    uint32_t tables_emptied;
+} zr_check_result;
+
+zr_status zr_plan_set_checked(zr_plan* plan, int32_t enable);
+zr_status zr_plan_verify(const zr_plan* plan, zr_stream_t stream);
+zr_status zr_plan_check_result(const zr_plan* plan, zr_check_result* out, zr_stream_t stream);
+
 /* Size of the library-owned scratch array used by zr_step_no_alloc. */
 #define ZR_NO_ALLOC_SCRATCH_BYTES (4u << 20)
 

@@ -44,10 +44,16 @@ EXPORTED = [
     "zr_step_bucket",
     "zr_step_finish", "zr_step_host",
     "zr_grad_sumsq", "zr_debug_reduce", "zr_step_no_alloc", "zr_state_save", "zr_state_load",
-    "zr_state_reshard", "zr_state_export_params", "zr_plan_owner_offsets", "zr_plan_set_gather_targets", "zr_ipc_export",
+    "zr_state_reshard", "zr_state_export_params", "zr_plan_set_checked", "zr_plan_verify",
+    "zr_plan_check_result", "zr_plan_owner_offsets", "zr_plan_set_gather_targets", "zr_ipc_export",
     "zr_ipc_open", "zr_ipc_close", "zr_plan_destroy", "zr_status_string",
 ]
 ZR_NO_ALLOC_SCRATCH_BYTES = 4 << 20
+
+
+class zr_check_result(ctypes.Structure):
+    _fields_ = [("bad_tiles", ctypes.c_uint64), ("first_bad", ctypes.c_int64),
+                ("hash_mismatch", ctypes.c_uint32), ("tables_emptied", ctypes.c_uint32)]
 
 
 class zr_adamw(ctypes.Structure):
@@ -87,6 +93,9 @@ _lib.zr_state_save.argtypes = [_vp, ctypes.c_char_p, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_state_load.argtypes = [_vp, ctypes.c_char_p, _vp, _vp, _vp, _P(_i64), _vp]
 _lib.zr_state_reshard.argtypes = [_vp, _vp, _i32, ctypes.c_char_p]
 _lib.zr_state_export_params.argtypes = [_vp, _vp, _i32, _i32, ctypes.c_char_p, _vp]
+_lib.zr_plan_set_checked.argtypes = [_vp, _i32]
+_lib.zr_plan_verify.argtypes = [_vp, _vp]
+_lib.zr_plan_check_result.argtypes = [_vp, _P(zr_check_result), _vp]
 _lib.zr_plan_owner_offsets.argtypes = [_vp, _vp]
 _lib.zr_plan_set_gather_targets.argtypes = [_vp, _vp, _vp]
 _lib.zr_ipc_export.argtypes = [_vp, _P(zr_ipc_handle)]
@@ -283,6 +292,20 @@ def zr_state_export_params(plan: int, src_paths, dtype: int, out_path: str) -> i
     _check(_lib.zr_state_export_params(plan, arr, len(src_paths), int(dtype), os.fsencode(out_path),
                                        ctypes.byref(n)), "zr_state_export_params")
     return n.value
+
+
+def zr_plan_set_checked(plan: int, enable: bool) -> None:
+    _check(_lib.zr_plan_set_checked(plan, 1 if enable else 0), "zr_plan_set_checked")
+
+
+def zr_plan_verify(plan: int, stream=None) -> None:
+    _check(_lib.zr_plan_verify(plan, _stream(stream)), "zr_plan_verify")
+
+
+def zr_plan_check_result(plan: int, stream=None) -> dict:
+    r = zr_check_result()
+    _check(_lib.zr_plan_check_result(plan, ctypes.byref(r), _stream(stream)), "zr_plan_check_result")
+    return {name: getattr(r, name) for name, _ in zr_check_result._fields_}
 
 
 def zr_plan_owner_offsets(plan: int, world_size: int):

@@ -55,6 +55,21 @@ zr_status check_device(const zr_plan* p) {
     return dev == p->device ? ZR_OK : ZR_ERR_INVALID_ARG;
 }
 
+// Checked mode: verify the device tile tables before a launch that reads
+// them (the status words reset for the hashes, then the two check kernels).
+zr_status verify_tables(const zr_plan* p, zr_stream_t stream) {
+    if (p->tiles.empty()) return ZR_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(p->d_check + 3, 0, 2 * sizeof(uint64_t), s) != cudaSuccess) return ZR_ERR_CUDA;
+    return cuda_status(static_cast<cudaError_t>(zr::launch_verify_tables(
+        p->d_tiles, p->d_tiles_by_owned, static_cast<int32_t>(p->tiles.size()), p->owned_numel(), p->padded_numel,
+        p->n_buckets, p->hash_tiles, p->hash_tiles_by_owned, p->d_check, s)));
+}
+
+zr_status verify_if_checked(const zr_plan* p, zr_stream_t stream) {
+    return p->checked ? verify_tables(p, stream) : ZR_OK;
+}
+
 zr_status check_state(const float* master, const float* m, const float* v) {
     if (!master || !m || !v) return ZR_ERR_INVALID_ARG;
     if (!aligned16(master) || !aligned16(m) || !aligned16(v)) return ZR_ERR_ALIGNMENT;
@@ -193,16 +208,55 @@ zr_status zr_plan_set_workspace(zr_plan* p, void* d_ws, uint64_t bytes, zr_strea
     p->d_own_sumsq = reinterpret_cast<double*>(base + L.own_sumsq);
     p->d_gather_targets = reinterpret_cast<uint16_t**>(base + L.gather_targets);
     p->d_scalars = reinterpret_cast<zr::AdamScalars*>(base + L.dev_scalars);
+    p->d_check = reinterpret_cast<uint64_t*>(base + L.check);
     p->n_gather_targets = 0;
     p->d_g_scratch = p->clip_uses_scratch() ? reinterpret_cast<float*>(base + L.g_scratch) : nullptr;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (!p->tiles.empty()) {
         const size_t bytes_tiles = sizeof(zr::Tile) * p->tiles.size();
-        cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
         if (cudaMemcpyAsync(p->d_tiles, p->tiles.data(), bytes_tiles, cudaMemcpyHostToDevice, s) != cudaSuccess ||
             cudaMemcpyAsync(p->d_tiles_by_owned, p->tiles_by_owned.data(), bytes_tiles, cudaMemcpyHostToDevice, s) !=
                 cudaSuccess)
             return ZR_ERR_CUDA;
     }
+    // Checked mode's reference hashes and fresh status words (no failure,
+    // smallest failing position all ones).
+    p->hash_tiles = zr::table_hash(p->tiles);
+    p->hash_tiles_by_owned = zr::table_hash(p->tiles_by_owned);
+    if (cudaMemsetAsync(p->d_check, 0, sizeof(uint64_t) * zr::kCheckWords, s) != cudaSuccess ||
+        cudaMemsetAsync(p->d_check + 1, 0xFF, sizeof(uint64_t), s) != cudaSuccess)
+        return ZR_ERR_CUDA;
+    return ZR_OK;
+}
+
+zr_status zr_plan_set_checked(zr_plan* p, int32_t enable) {
+    if (!p) return ZR_ERR_INVALID_ARG;
+    p->checked = enable != 0;
+    return ZR_OK;
+}
+
+zr_status zr_plan_verify(const zr_plan* p, zr_stream_t stream) {
+    if (!p) return ZR_ERR_INVALID_ARG;
+    if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
+    const zr_status dst = check_device(p);
+    if (dst != ZR_OK) return dst;
+    return verify_tables(p, stream);
+}
+
+zr_status zr_plan_check_result(const zr_plan* p, zr_check_result* out, zr_stream_t stream) {
+    if (!p || !out) return ZR_ERR_INVALID_ARG;
+    if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
+    const zr_status dst = check_device(p);
+    if (dst != ZR_OK) return dst;
+    uint64_t w[zr::kCheckWords];
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(w, p->d_check, sizeof w, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return ZR_ERR_CUDA;
+    out->bad_tiles = w[0];
+    out->first_bad = w[1] == ~0ull ? -1 : static_cast<int64_t>(w[1]);
+    out->hash_mismatch = static_cast<uint32_t>(w[2]);
+    out->tables_emptied = (w[0] != 0 || w[2] != 0) ? 1u : 0u;
     return ZR_OK;
 }
 
@@ -280,6 +334,10 @@ static zr_status step_impl(const zr_plan* p, const void* const* grad_ptrs, float
     if ((st = check_state(master, m, v)) != ZR_OK || (st = check_param_out(p, param_out)) != ZR_OK) return st;
     if (p->clip_enabled() && !p->d_sumsq_partials) return ZR_ERR_NO_WORKSPACE;
 
+    {
+        const zr_status cs = verify_if_checked(p, stream);
+        if (cs != ZR_OK) return cs;
+    }
     zr::LaunchArgs a = base_args(p);
     a.master = master;
     a.m = m;
@@ -329,6 +387,10 @@ zr_status zr_step_bucket(const zr_plan* p, int32_t bucket, const void* const* gr
     if (count == 0) return ZR_OK;   // this rank owns nothing in the bucket
     zr_status st = check_grads(p, grad_ptrs);
     if (st != ZR_OK) return st;
+    {
+        const zr_status cs = verify_if_checked(p, stream);
+        if (cs != ZR_OK) return cs;
+    }
     zr::LaunchArgs a = base_args(p);
     a.tiles = p->d_tiles + first;
     a.n_tiles = count;
@@ -369,6 +431,10 @@ zr_status zr_step_finish(const zr_plan* p, const void* const* grad_ptrs, float* 
     }
     zr_status st2 = check_state(master, m, v);
     if (st2 != ZR_OK || (st2 = check_param_out(p, param_out)) != ZR_OK) return st2;
+    {
+        const zr_status cs = verify_if_checked(p, stream);
+        if (cs != ZR_OK) return cs;
+    }
     zr::LaunchArgs a = base_args(p);
     a.master = master;
     a.m = m;
@@ -401,6 +467,10 @@ zr_status zr_grad_sumsq(const zr_plan* p, const void* const* grad_ptrs, double* 
     }
     zr_status st = check_grads(p, grad_ptrs);
     if (st != ZR_OK) return st;
+    {
+        const zr_status cs = verify_if_checked(p, stream);
+        if (cs != ZR_OK) return cs;
+    }
     zr::LaunchArgs a = base_args(p);
     a.tile_partials = p->d_tile_partials;
     int e = zr::launch_tiles(zr::Pass::kSumsq, a, grad_ptrs, false, false, s);
@@ -421,6 +491,10 @@ zr_status zr_debug_reduce(const zr_plan* p, const void* const* grad_ptrs, float*
     zr_status st = check_grads(p, grad_ptrs);
     if (st != ZR_OK) return st;
     if (!aligned16(g_out)) return ZR_ERR_ALIGNMENT;
+    {
+        const zr_status cs = verify_if_checked(p, stream);
+        if (cs != ZR_OK) return cs;
+    }
     zr::LaunchArgs a = base_args(p);
     a.g_buf = g_out;
     return cuda_status(static_cast<cudaError_t>(
@@ -476,6 +550,8 @@ zr_status zr_step_host(const zr_plan* p, const void* const* host_grad_ptrs, void
     cudaEvent_t* ev_done = p->host_events + zr_plan::kHostChunks;   // K: chunk k's parameters written
     cudaEvent_t ev_start = p->host_events[2 * zr_plan::kHostChunks];
     cudaEvent_t ev_end = p->host_events[2 * zr_plan::kHostChunks + 1];
+    st = verify_if_checked(p, stream);
+    if (st != ZR_OK) return st;
     // The copies may overwrite the device gradient buffers only after the
     // work already queued on the caller's stream.
     if (cudaEventRecord(ev_start, S) != cudaSuccess || cudaStreamWaitEvent(C, ev_start, 0) != cudaSuccess ||

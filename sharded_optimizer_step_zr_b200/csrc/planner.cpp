@@ -8,6 +8,7 @@
 // pass produces their gradients (reverse declaration order), capped by
 // bucket_cap_bytes of bf16 gradient.
 #include <algorithm>
+#include <cstring>
 #include <cmath>
 #include <limits>
 #include <queue>
@@ -264,10 +265,22 @@ WorkspaceLayout workspace_layout(const zr_plan& p) {
     off = align256(off + sizeof(void*) * static_cast<uint64_t>(p.world_size));
     L.dev_scalars = off;
     off = align256(off + sizeof(AdamScalars));
+    L.check = off;
+    off = align256(off + sizeof(uint64_t) * kCheckWords);
     L.g_scratch = off;
     off = align256(off + (p.clip_uses_scratch() ? sizeof(float) * static_cast<uint64_t>(p.owned_numel()) : 0));
     L.total = off;
     return L;
+}
+
+uint64_t table_hash(const std::vector<Tile>& tiles) {
+    uint64_t h = 0;
+    for (size_t i = 0; i < tiles.size(); ++i) {
+        uint64_t w[kTileWords];
+        std::memcpy(w, &tiles[i], sizeof(Tile));
+        for (int j = 0; j < kTileWords; ++j) h += tile_word_hash(w[j], kTileWords * i + j);
+    }
+    return h;
 }
 
 AdamScalars adam_scalars(const zr_adamw& hp, int64_t step) {

@@ -33,6 +33,32 @@ constexpr int kThreads = 128;                  // threads per CTA
 constexpr int kElemsPerThreadIter = 8;         // one 16-byte bf16 vector
 constexpr int kTileElems = kThreads * kElemsPerThreadIter * 2;  // 2048
 
+#if defined(__CUDACC__)
+#define ZR_HOST_DEVICE __host__ __device__
+#else
+#define ZR_HOST_DEVICE
+#endif
+
+// Order-independent 64-bit hash of a tile table, for checked mode: the sum
+// (mod 2^64) over the table's 64-bit words w_k (k = word position) of
+// f(w_k + k * 0x9E3779B97F4A7C15), f the splitmix64 output function (Steele,
+// Lea & Flood 2014).  Any change of one word changes the sum except with
+// probability about 2^-64, and the sum can be formed in any order.
+ZR_HOST_DEVICE inline uint64_t tile_word_hash(uint64_t w, uint64_t k) {
+    uint64_t z = w + k * 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+constexpr int kTileWords = static_cast<int>(sizeof(Tile) / sizeof(uint64_t));   // 4
+
+// Checked mode's status words in the workspace: [0] tiles failing a check
+// (both tables, cumulative), [1] the smallest failing position (bucket-order
+// table i, owned-order table n_tiles + i; all ones when none), [2] hash
+// mismatch bits (1: bucket-order table, 2: owned-order table), [3], [4] the
+// hashes of the two tables as last computed on the device.
+constexpr int kCheckWords = 5;
+
 // AdamW scalars for one step, fp64 on the host rounded once to fp32.
 struct AdamScalars {
     float beta1, beta2, one_minus_beta1, one_minus_beta2;
@@ -78,6 +104,13 @@ int launch_device_scalars(int64_t* d_step, const zr_adamw& hp, AdamScalars* out,
 int launch_clip_combine(const double* tile_partials, int32_t n_tiles, double* partials_all,
                         int32_t world_size, int32_t rank, float max_norm, float* clip_coef_out,
                         double* sumsq_out, void* stream);
+// Checked mode: verify both device tile tables against the tile invariants
+// and the hashes taken on the host at upload, then, if anything failed (now
+// or before), overwrite both tables with empty tiles.  `check` holds
+// kCheckWords words; words 3 and 4 must be zeroed before the launch.
+int launch_verify_tables(Tile* tiles, Tile* tiles_by_owned, int32_t n_tiles, int64_t n_owned, int64_t n_out,
+                         int32_t n_buckets, uint64_t hash_tiles, uint64_t hash_by_owned, uint64_t* check,
+                         void* stream);
 
 }  // namespace zr
 
@@ -119,6 +152,10 @@ struct zr_plan {
     uint16_t** d_gather_targets = nullptr; // workspace: world_size parameter buffers
     zr::AdamScalars* d_scalars = nullptr;  // workspace: scalars computed on the device
     int32_t n_gather_targets = 0;          // 0 until zr_plan_set_gather_targets
+    uint64_t* d_check = nullptr;           // workspace: checked mode's status words
+    bool checked = false;                  // verify the tables before every launch
+    uint64_t hash_tiles = 0;               // tile_word_hash sums of the two host tables
+    uint64_t hash_tiles_by_owned = 0;
 
     // zr_step_host's copy streams and events, created on its first call
     // (host-side resources, not part of the plan's observable state).
@@ -141,9 +178,10 @@ zr_status build_plan(zr_plan& p, int32_t n_tensors, const int32_t* ndims,
                      const int64_t* const* shapes);
 // Workspace layout: offsets of each region, total bytes.
 struct WorkspaceLayout {
-    uint64_t tiles, tiles_by_owned, tile_partials, clip_coef, own_sumsq, gather_targets, dev_scalars, g_scratch,
-        total;
+    uint64_t tiles, tiles_by_owned, tile_partials, clip_coef, own_sumsq, gather_targets, dev_scalars, check,
+        g_scratch, total;
 };
 WorkspaceLayout workspace_layout(const zr_plan& p);
+uint64_t table_hash(const std::vector<Tile>& tiles);
 AdamScalars adam_scalars(const zr_adamw& hp, int64_t step);
 }  // namespace zr

@@ -5,9 +5,10 @@ libzr.so's kernels through the C ABI.
 """
 from __future__ import annotations
 
-from . import (ZR_PARTITION_FLAT, zr_debug_reduce, zr_grad_sumsq, zr_plan_create, zr_plan_destroy,
-               zr_plan_query, zr_plan_segments, zr_plan_set_sumsq_partials, zr_plan_set_workspace,
-               zr_plan_workspace_bytes, zr_step, zr_step_bucket, zr_step_finish, zr_step_host)
+from . import (ZR_PARTITION_FLAT, zr_debug_reduce, zr_grad_sumsq, zr_plan_check_result, zr_plan_create,
+               zr_plan_destroy, zr_plan_query, zr_plan_segments, zr_plan_set_checked, zr_plan_set_sumsq_partials,
+               zr_plan_set_workspace, zr_plan_verify, zr_plan_workspace_bytes, zr_step, zr_step_bucket,
+               zr_step_finish, zr_step_host)
 
 
 class ZrPlan:
@@ -85,6 +86,15 @@ class ZrPlan:
 
     def debug_reduce(self, grads, g_out, stream=None):
         zr_debug_reduce(self.handle, grads, g_out, stream)
+
+    def set_checked(self, enable=True):
+        zr_plan_set_checked(self.handle, enable)
+
+    def verify(self, stream=None):
+        zr_plan_verify(self.handle, stream)
+
+    def check_result(self, stream=None):
+        return zr_plan_check_result(self.handle, stream)
 
     def close(self):
         if self.handle:

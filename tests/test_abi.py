@@ -178,3 +178,22 @@ def test_workspace_grows_with_clip_scratch():
     finally:
         for h in (plain, clip8, clip4):
             zr.zr_plan_destroy(h)
+
+
+def test_checked_mode_arguments_without_a_device():
+    """Checked mode's calls reject a missing plan and an unbound workspace
+    before touching the device."""
+    import ctypes
+    assert zr._lib.zr_plan_set_checked(None, 1) == zr.ZR_ERR_INVALID_ARG
+    assert zr._lib.zr_plan_verify(None, None) == zr.ZR_ERR_INVALID_ARG
+    r = zr.zr_check_result()
+    assert zr._lib.zr_plan_check_result(None, ctypes.byref(r), None) == zr.ZR_ERR_INVALID_ARG
+    h = zr.zr_plan_create([(4096,), (100,)], 2, 0, 0, 1 << 20)
+    try:
+        zr.zr_plan_set_checked(h, True)
+        zr.zr_plan_set_checked(h, False)
+        assert zr._lib.zr_plan_verify(h, None) == zr.ZR_ERR_NO_WORKSPACE
+        assert zr._lib.zr_plan_check_result(h, None, None) == zr.ZR_ERR_INVALID_ARG
+        assert zr._lib.zr_plan_check_result(h, ctypes.byref(r), None) == zr.ZR_ERR_NO_WORKSPACE
+    finally:
+        zr.zr_plan_destroy(h)
