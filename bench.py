@@ -60,6 +60,8 @@ def parse():
     ap.add_argument("--overlap", action="store_true",
                     help="exposed optimizer time behind an emulated backward pass: one zr_step "
                          "after it, against zr_step_bucket as each bucket's gradients complete")
+    ap.add_argument("--checked", action="store_true",
+                    help="checked mode: the device tile tables verified before every launch")
     ap.add_argument("--sweep", action="store_true",
                     help="1.3B set: bucket cap x W x partition; one JSON record per point")
     args = ap.parse_args()
@@ -426,6 +428,8 @@ def run_zr(args):
     torch.cuda.synchronize()
 
     step_no = 0
+    if args.checked:
+        plan.set_checked(True)
     run_step = plan.bound_step(grads, master, m, v, param_out, stream)   # arguments marshalled once
     my_buckets = sorted({s["bucket"] for s in plan.segments() if s["owner"] == zr_rank})
     if args.per_bucket:
@@ -465,8 +469,8 @@ def run_zr(args):
     avg_ms = local_ms / K
     achieved = alg_bytes / (avg_ms * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
-    # (bucket-by-bucket steps launch per bucket: no per-launch record)
-    traffic = None if args.per_bucket else recorded_traffic(wl.name, clip)
+    # (bucket-by-bucket or checked steps launch more kernels: no per-launch record)
+    traffic = None if (args.per_bucket or args.checked) else recorded_traffic(wl.name, clip)
 
     # end to end through zr_step_host: pinned host gradients in, result out
     e2e = None
@@ -505,6 +509,8 @@ def run_zr(args):
     launches_per_step = 3 if clip else 1
     if args.per_bucket:
         launches_per_step = len(my_buckets) + (2 if clip else 0)
+    if args.checked:
+        launches_per_step += 2 * (len(my_buckets) + (1 if clip else 0) if args.per_bucket else 1)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -513,6 +519,7 @@ def run_zr(args):
                    "partition": "flat" if wl.mode == 0 else "whole_tensor",
                    "bucket_cap_mb": wl.bucket_cap_mb, "clip": clip, "owned_params": n,
                    "per_bucket": bool(args.per_bucket), "buckets_stepped": len(my_buckets),
+                   "checked": bool(args.checked),
                    "bytes_per_owned_param": bpp,
                    "l2": f"no flush: each step touches {alg_bytes / 1e6:.0f} MB > 126 MB L2"},
         "hbm_gbs": achieved,
