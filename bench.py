@@ -510,7 +510,7 @@ def run_zr(args):
     if args.per_bucket:
         launches_per_step = len(my_buckets) + (2 if clip else 0)
     if args.checked:
-        launches_per_step += 2 * (len(my_buckets) + (1 if clip else 0) if args.per_bucket else 1)
+        launches_per_step += (len(my_buckets) + (1 if clip else 0)) if args.per_bucket else 1
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,

@@ -357,7 +357,7 @@ zr_status zr_state_export_params(const zr_plan* plan, const char* const* src_pat
  * step to wrong or out-of-bounds addresses.  The pages have no counterpart;
  * it follows from this library's caller-owned workspace.
  *
- * zr_plan_verify enqueues on `stream` two kernels that test every tile of
+ * zr_plan_verify enqueues on `stream` one kernel that tests every tile of
  * both device tables against the invariants the planner guarantees (length
  * 1..2048, owned and global ranges inside the rank's owned count and
  * padded_numel, 16-byte vector flags only where the alignment holds, bucket
@@ -367,8 +367,8 @@ zr_status zr_state_export_params(const zr_plan* plan, const char* const* src_pat
  * an earlier check, both tables are overwritten with empty tiles, so the
  * steps queued after it update nothing and write nothing (their results
  * are then missing, not wrong); zr_plan_set_workspace re-uploads the tables
- * and clears the status.  Nothing waits on anything; a check costs two
- * small launches reading 64 bytes per tile.
+ * and clears the status.  Nothing waits on anything; a check is one small
+ * launch reading 64 bytes per tile.
  * zr_plan_set_checked(plan, 1) makes every call that launches the tile
  * kernels (zr_step, zr_step_device_count, zr_step_bucket, zr_step_finish,
  * zr_step_host, zr_grad_sumsq, zr_debug_reduce) run that check first on its

@@ -56,11 +56,10 @@ zr_status check_device(const zr_plan* p) {
 }
 
 // Checked mode: verify the device tile tables before a launch that reads
-// them (the status words reset for the hashes, then the two check kernels).
+// them (one kernel on the caller's stream).
 zr_status verify_tables(const zr_plan* p, zr_stream_t stream) {
     if (p->tiles.empty()) return ZR_OK;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(p->d_check + 3, 0, 2 * sizeof(uint64_t), s) != cudaSuccess) return ZR_ERR_CUDA;
     return cuda_status(static_cast<cudaError_t>(zr::launch_verify_tables(
         p->d_tiles, p->d_tiles_by_owned, static_cast<int32_t>(p->tiles.size()), p->owned_numel(), p->padded_numel,
         p->n_buckets, p->hash_tiles, p->hash_tiles_by_owned, p->d_check, s)));

@@ -3,11 +3,11 @@
 // The tables live in the caller's workspace, so another kernel that writes
 // there by mistake (a race, a stray pointer) would send the next step to
 // wrong or out-of-bounds addresses.  With checked mode on, every launching
-// call first runs these two kernels: the first tests every tile against the
-// invariants the planner guarantees and hashes both tables; the second
-// compares the hashes with the ones the host took when it uploaded the
-// tables and, if anything failed, empties the tables so that the step that
-// follows touches no parameter memory.  Neither waits on anything.
+// call first runs this kernel: it tests every tile against the invariants
+// the planner guarantees, hashes both tables, compares the hashes with the
+// ones the host took when it uploaded the tables and, if anything failed,
+// empties the tables so that the step that
+// follows touches no parameter memory.  Nothing waits on anything.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -43,12 +43,19 @@ __device__ __forceinline__ uint64_t tile_hash(const Tile* table, int32_t i) {
     return h;
 }
 
-// Grid-stride over both tables: count the tiles that break an invariant
-// (a bucket-order tile must also sit at its own index), keep the smallest
-// failing position, and add every tile's words into the two hash sums.
+// One launch.  Grid-stride over both tables: count the tiles that break an
+// invariant (a bucket-order tile must also sit at its own index), keep the
+// smallest failing position, and add every tile's words into the two hash
+// sums.  The last block to finish (a counter of finished blocks; nothing
+// waits) compares the sums with the host's, records mismatches, resets the
+// sums and the counter for the next check and, if anything has failed (now
+// or at an earlier check since the workspace was bound), empties both tables
+// -- every tile gets length 0 and its own position as index -- so that the
+// kernels queued after this one touch no parameter memory.
 __global__ void __launch_bounds__(256)
-zr_verify_tables_kernel(const Tile* tiles, const Tile* by_owned, int32_t n_tiles, int64_t n_owned, int64_t n_out,
-                        int32_t n_buckets, unsigned long long* check) {
+zr_verify_tables_kernel(Tile* tiles, Tile* by_owned, int32_t n_tiles, int64_t n_owned, int64_t n_out,
+                        int32_t n_buckets, unsigned long long hash_tiles, unsigned long long hash_by_owned,
+                        unsigned long long* check) {
     unsigned long long h0 = 0, h1 = 0;
     for (int32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n_tiles; i += gridDim.x * blockDim.x) {
         const Tile a = tiles[i], b = by_owned[i];
@@ -72,21 +79,25 @@ zr_verify_tables_kernel(const Tile* tiles, const Tile* by_owned, int32_t n_tiles
         atomicAdd(&check[3], h0);
         atomicAdd(&check[4], h1);
     }
-}
-
-// After the verification: compare the hashes with the host's, record the
-// mismatches, and if anything has failed (now or at an earlier check since
-// the workspace was bound) empty both tables -- every tile gets length 0 and
-// its own position as index -- so that kernels queued after this touch no
-// parameter memory.  Every block decides from the same words; block 0
-// records the mismatch bits.
-__global__ void __launch_bounds__(256)
-zr_neutralise_tables_kernel(Tile* tiles, Tile* by_owned, int32_t n_tiles, unsigned long long hash_tiles,
-                            unsigned long long hash_by_owned, unsigned long long* check) {
-    const unsigned long long bits = (check[3] != hash_tiles ? 1ull : 0ull) | (check[4] != hash_by_owned ? 2ull : 0ull);
-    if (blockIdx.x == 0 && threadIdx.x == 0 && bits) atomicOr(&check[2], bits);
-    if (bits == 0 && check[0] == 0 && check[2] == 0) return;
-    for (int32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n_tiles; i += gridDim.x * blockDim.x) {
+    __shared__ int last, failed;
+    __syncthreads();                      // every warp of the block has added its sums
+    if (threadIdx.x == 0) {
+        __threadfence();
+        last = atomicAdd(&check[5], 1ull) == gridDim.x - 1ull;
+    }
+    __syncthreads();
+    if (!last) return;
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned long long s0 = atomicExch(&check[3], 0ull), s1 = atomicExch(&check[4], 0ull);
+        atomicExch(&check[5], 0ull);
+        const unsigned long long bits = (s0 != hash_tiles ? 1ull : 0ull) | (s1 != hash_by_owned ? 2ull : 0ull);
+        const unsigned long long mismatch = atomicOr(&check[2], bits) | bits;
+        failed = (mismatch != 0 || atomicAdd(&check[0], 0ull) != 0) ? 1 : 0;
+    }
+    __syncthreads();
+    if (!failed) return;
+    for (int32_t i = threadIdx.x; i < n_tiles; i += blockDim.x) {
         Tile empty{};
         empty.index = i;
         tiles[i] = empty;
@@ -100,13 +111,10 @@ int launch_verify_tables(Tile* tiles, Tile* tiles_by_owned, int32_t n_tiles, int
                          int32_t n_buckets, uint64_t hash_tiles, uint64_t hash_by_owned, uint64_t* check,
                          void* stream_v) {
     if (n_tiles == 0) return cudaSuccess;
-    cudaStream_t s = static_cast<cudaStream_t>(stream_v);
     const int blocks = static_cast<int>(std::min<int64_t>((n_tiles + 255) / 256, 148 * 4));
-    unsigned long long* c = reinterpret_cast<unsigned long long*>(check);
-    zr_verify_tables_kernel<<<blocks, 256, 0, s>>>(tiles, tiles_by_owned, n_tiles, n_owned, n_out, n_buckets, c);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    zr_neutralise_tables_kernel<<<blocks, 256, 0, s>>>(tiles, tiles_by_owned, n_tiles, hash_tiles, hash_by_owned, c);
+    zr_verify_tables_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream_v)>>>(
+        tiles, tiles_by_owned, n_tiles, n_owned, n_out, n_buckets, hash_tiles, hash_by_owned,
+        reinterpret_cast<unsigned long long*>(check));
     return cudaGetLastError();
 }
 

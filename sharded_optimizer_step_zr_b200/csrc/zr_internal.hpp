@@ -56,8 +56,9 @@ constexpr int kTileWords = static_cast<int>(sizeof(Tile) / sizeof(uint64_t));   
 // (both tables, cumulative), [1] the smallest failing position (bucket-order
 // table i, owned-order table n_tiles + i; all ones when none), [2] hash
 // mismatch bits (1: bucket-order table, 2: owned-order table), [3], [4] the
-// hashes of the two tables as last computed on the device.
-constexpr int kCheckWords = 5;
+// two tables' hash sums while a check runs, [5] the count of its finished
+// blocks (words 3-5 are 0 between checks).
+constexpr int kCheckWords = 6;
 
 // AdamW scalars for one step, fp64 on the host rounded once to fp32.
 struct AdamScalars {
@@ -106,8 +107,9 @@ int launch_clip_combine(const double* tile_partials, int32_t n_tiles, double* pa
                         double* sumsq_out, void* stream);
 // Checked mode: verify both device tile tables against the tile invariants
 // and the hashes taken on the host at upload, then, if anything failed (now
-// or before), overwrite both tables with empty tiles.  `check` holds
-// kCheckWords words; words 3 and 4 must be zeroed before the launch.
+// or before), overwrite both tables with empty tiles.  One launch; `check`
+// holds kCheckWords words, zeroed (word 1 all ones) when the workspace is
+// bound.
 int launch_verify_tables(Tile* tiles, Tile* tiles_by_owned, int32_t n_tiles, int64_t n_owned, int64_t n_out,
                          int32_t n_buckets, uint64_t hash_tiles, uint64_t hash_by_owned, uint64_t* check,
                          void* stream);
