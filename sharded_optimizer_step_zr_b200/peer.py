@@ -19,6 +19,23 @@ from . import (ZR_PARTITION_FLAT, zr_ipc_close, zr_ipc_export, zr_ipc_open, zr_p
 from .plan import ZrPlan
 
 
+class PeerFailure(RuntimeError):
+    """A peer did not reach a phase boundary of the step (it exited, hung or
+    lost its connection) within the process group's timeout.  Raised on the
+    host before this rank launches anything that would read or write that
+    peer's memory."""
+
+
+def sync_point(dist, group, phase, step):
+    """Every rank's arrival at `phase` of `step`.  The process group's own
+    timeout bounds the wait; a failure becomes a PeerFailure naming the phase
+    and step, so a caller can stop (or rebuild the group) between steps."""
+    try:
+        dist.barrier(group)
+    except Exception as e:      # gloo and NCCL report a lost peer differently
+        raise PeerFailure(f"step {step}, {phase}: a peer did not arrive ({type(e).__name__}: {e})") from e
+
+
 class PeerZero:
     def __init__(self, group, shapes, mode=ZR_PARTITION_FLAT, bucket_cap_bytes=25 << 20, lr=3e-4,
                  beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.1, max_grad_norm=0.0, device=None):
@@ -92,15 +109,16 @@ class PeerZero:
         part.copy_(torch.cat(gathered).to(part.device))
 
     def step(self, master, m, v, step):
-        """One optimizer step of this rank (every rank calls it together)."""
+        """One optimizer step of this rank (every rank calls it together).
+        Raises PeerFailure, before launching, if a peer is missing."""
         import torch
         torch.cuda.current_stream().synchronize()      # this replica's gradients are written
-        self.dist.barrier(self.group)                  # ... and every other replica's
+        sync_point(self.dist, self.group, "gradients ready", step)   # ... and every other replica's
         if self.plan.max_grad_norm > 0:
             self._exchange_sumsq()
         zr_step(self.plan.handle, self.grad_ptrs, master, m, v, None, step)
         torch.cuda.current_stream().synchronize()
-        self.dist.barrier(self.group)                  # every slice is in every parameter buffer
+        sync_point(self.dist, self.group, "parameters gathered", step)   # every slice is in every buffer
 
     def close(self):
         if self._opened:

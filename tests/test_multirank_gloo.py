@@ -110,3 +110,48 @@ def test_two_ranks_gather_equals_unsharded(mode):
                 .view(torch.int16).numpy().view(np.uint16).copy() for w in range(world)]
         oracle.ddp_step(full, master, m, v, out, HP, t)
     assert np.array_equal(results[0][3], out)
+
+
+def _failure_worker(rank, world, port, how, result_q):
+    import sys
+    import datetime
+    import time
+    sys.path.insert(0, ROOT)
+    from sharded_optimizer_step_zr_b200.peer import PeerFailure, sync_point
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    sync_point(dist, None, "gradients ready", 1)         # step 1: everyone arrives
+    if rank == 1:
+        if how == "exit":
+            os._exit(0)                                  # a crash between steps: no clean shutdown
+        time.sleep(20)                                   # a rank that never arrives in time
+        os._exit(0)
+    t0 = time.time()
+    try:
+        sync_point(dist, None, "gradients ready", 2)
+        result_q.put(("no error", time.time() - t0))
+    except PeerFailure as e:
+        result_q.put((str(e), time.time() - t0))
+    result_q.close()
+    result_q.join_thread()                               # the message is sent before the hard exit
+    os._exit(0)
+
+
+@pytest.mark.parametrize("how", ["exit", "hang"])
+def test_missing_peer_raises_before_the_next_launch(how):
+    """A peer that dies between steps, or never arrives, ends the next
+    phase boundary with PeerFailure on the surviving rank (within the
+    group's 5 s timeout plus slack), instead of a hang or a launch that
+    would touch the peer's memory."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_failure_worker, args=(r, 2, port, how, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    msg, waited = q.get(timeout=120)
+    for p in procs:
+        p.join(timeout=60)
+    assert msg.startswith("step 2, gradients ready: a peer did not arrive"), msg
+    assert waited < 30
