@@ -11,6 +11,36 @@ from . import (ZR_PARTITION_FLAT, zr_debug_reduce, zr_grad_sumsq, zr_plan_check_
                zr_step_finish, zr_step_host)
 
 
+def _require_all(specs, device):
+    """Checks buffer arguments before their addresses reach the library,
+    which cannot see sizes.  specs: (buffer, name, dtype, min elements,
+    host?).  Each must be a contiguous torch tensor of that dtype with at
+    least that many elements (all checked first), then on `device` -- or in
+    host memory for host buffers.  A plain integer is a raw address and None
+    an absent buffer: both are left to the library's own checks."""
+    import torch
+    tensors = []
+    for x, what, dtype, numel, host in specs:
+        if x is None or isinstance(x, int):
+            continue
+        if not isinstance(x, torch.Tensor):
+            raise TypeError(f"{what}: expected a torch tensor or an address, got {type(x).__name__}")
+        if x.dtype != dtype:
+            raise ValueError(f"{what}: dtype {x.dtype}, expected {dtype}")
+        if not x.is_contiguous():
+            raise ValueError(f"{what}: not contiguous")
+        if x.numel() < numel:
+            raise ValueError(f"{what}: {x.numel()} elements, the plan needs at least {numel}")
+        tensors.append((x, what, host))
+    for x, what, host in tensors:
+        if host:
+            if x.device.type != "cpu":
+                raise ValueError(f"{what}: must be in host memory, is on {x.device}")
+        elif x.device.type != "cuda" or (device is not None and x.device != device):
+            raise ValueError(f"{what}: must be on {device if device is not None else 'a CUDA device'}, "
+                             f"is on {x.device}")
+
+
 class ZrPlan:
     def __init__(self, shapes, world_size, rank, mode=ZR_PARTITION_FLAT, bucket_cap_bytes=25 << 20,
                  lr=3e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.1, max_grad_norm=0.0,
@@ -27,6 +57,7 @@ class ZrPlan:
         self.owned_numel = info["owned_numel"]
         self.n_buckets = info["n_buckets"]
         self.workspace_bytes = zr_plan_workspace_bytes(self.handle)
+        self.device = None
         self.workspace = None
         self.partials = None
         if bind:
@@ -35,6 +66,10 @@ class ZrPlan:
     def bind(self, device=None, stream=None):
         import torch
         device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+        device = torch.device(device)
+        if device.index is None:
+            device = torch.device("cuda", torch.cuda.current_device())
+        self.device = device
         # torch's caching allocator returns 512-byte aligned blocks
         self.workspace = torch.empty(max(256, self.workspace_bytes), dtype=torch.uint8, device=device)
         zr_plan_set_workspace(self.handle, self.workspace, self.workspace.numel(), stream)
@@ -51,19 +86,44 @@ class ZrPlan:
                 if s["owner"] == self.rank]
         return sorted(runs)
 
+    def check_step_buffers(self, grads, master, m, v, param_out):
+        """The step's buffers against the plan: W bf16 gradient buffers and
+        fp32 master / m / v of owned_numel elements, a bf16 parameter buffer
+        of padded_numel, all on the plan's device.  Raw addresses (ints) and
+        None pass through to the library's own checks."""
+        _require_all(self._step_specs(grads, master, m, v, param_out), self.device)
+
+    def _step_specs(self, grads, master, m, v, param_out):
+        import torch
+        if self.owned_numel == 0:
+            return []
+        specs = []
+        if grads is not None:      # None: a call that reads no gradients (zr_step_finish from scratch)
+            if len(grads) != self.world_size:
+                raise ValueError(f"grads: {len(grads)} buffers, the plan has W = {self.world_size}")
+            specs += [(g, f"grads[{w}]", torch.bfloat16, self.owned_numel, False) for w, g in enumerate(grads)]
+        specs += [(x, name, torch.float32, self.owned_numel, False) for x, name in ((master, "master"), (m, "m"),
+                                                                                      (v, "v"))]
+        specs.append((param_out, "param_out", torch.bfloat16, self.padded_numel, False))
+        return specs
+
     def step(self, grads, master, m, v, param_out, step, stream=None):
+        self.check_step_buffers(grads, master, m, v, param_out)
         zr_step(self.handle, grads, master, m, v, param_out, step, stream)
 
     def step_bucket(self, bucket, grads, master, m, v, param_out, step, stream=None):
+        self.check_step_buffers(grads, master, m, v, param_out)
         zr_step_bucket(self.handle, bucket, grads, master, m, v, param_out, step, stream)
 
     def step_finish(self, grads, master, m, v, param_out, step, stream=None):
+        self.check_step_buffers(grads, master, m, v, param_out)
         zr_step_finish(self.handle, grads, master, m, v, param_out, step, stream)
 
     def bound_step(self, grads, master, m, v, param_out, stream=None):
         """A callable f(step) that runs zr_step on fixed buffers with the
-        arguments marshalled once (for tight loops)."""
+        arguments marshalled (and checked) once (for tight loops)."""
         from . import _addr, _check, _lib, _ptr_array, _stream
+        self.check_step_buffers(grads, master, m, v, param_out)
         arr = _ptr_array(grads)
         args = (self.handle, arr, _addr(master), _addr(m), _addr(v), _addr(param_out))
         s = _stream(stream)
@@ -78,13 +138,28 @@ class ZrPlan:
 
     def step_host(self, host_grads, dev_grads, master, m, v, param_out, host_param_out, step,
                   stream=None):
+        import torch
+        specs = self._step_specs(dev_grads, master, m, v, param_out)
+        if self.owned_numel > 0:
+            if len(host_grads) != self.world_size:
+                raise ValueError(f"host_grads: {len(host_grads)} buffers, the plan has W = {self.world_size}")
+            specs += [(g, f"host_grads[{w}]", torch.bfloat16, self.owned_numel, True)
+                      for w, g in enumerate(host_grads)]
+            specs.append((host_param_out, "host_param_out", torch.bfloat16, self.padded_numel, True))
+        _require_all(specs, self.device)
         zr_step_host(self.handle, host_grads, dev_grads, master, m, v, param_out, host_param_out,
                      step, stream)
 
     def grad_sumsq(self, grads, out, stream=None):
+        import torch
+        specs = [(g, f"grads[{w}]", torch.bfloat16, self.owned_numel, False) for w, g in enumerate(grads)]
+        _require_all(specs + [(out, "out", torch.float64, 1, False)], self.device)
         zr_grad_sumsq(self.handle, grads, out, stream)
 
     def debug_reduce(self, grads, g_out, stream=None):
+        import torch
+        specs = [(g, f"grads[{w}]", torch.bfloat16, self.owned_numel, False) for w, g in enumerate(grads)]
+        _require_all(specs + [(g_out, "g_out", torch.float32, self.owned_numel, False)], self.device)
         zr_debug_reduce(self.handle, grads, g_out, stream)
 
     def set_checked(self, enable=True):

@@ -197,3 +197,38 @@ def test_checked_mode_arguments_without_a_device():
         assert zr._lib.zr_plan_check_result(h, ctypes.byref(r), None) == zr.ZR_ERR_NO_WORKSPACE
     finally:
         zr.zr_plan_destroy(h)
+
+
+def test_plan_rejects_wrong_buffers_before_the_library():
+    """ZrPlan checks tensor arguments against the plan (the C ABI sees only
+    addresses): count, dtype, contiguity, size, then device -- all on the
+    host, before any launch."""
+    import torch
+    from sharded_optimizer_step_zr_b200.plan import ZrPlan
+    plan = ZrPlan([(4096,), (100,)], 2, 1, 0, 1 << 20, bind=False)
+    n, P = plan.owned_numel, plan.padded_numel
+    g = [torch.zeros(n, dtype=torch.bfloat16) for _ in range(2)]
+    st = [torch.zeros(n, dtype=torch.float32) for _ in range(3)]
+    out = torch.zeros(P, dtype=torch.bfloat16)
+    cases = [
+        ((g[:1], *st, out), ValueError, "W = 2"),
+        (([g[0], g[1].float()], *st, out), ValueError, "dtype"),
+        ((g, st[0][: n - 1], st[1], st[2], out), ValueError, "at least"),
+        ((g, st[0], torch.zeros(2 * n, dtype=torch.float32)[::2], st[2], out), ValueError, "contiguous"),
+        ((g, *st, out[: P - 1]), ValueError, "at least"),
+        ((g, *st, out), ValueError, "must be on"),                 # host tensors, a device plan
+        ((g, st[0], "m", st[2], out), TypeError, "expected a torch tensor"),
+    ]
+    for args, exc, text in cases:
+        with pytest.raises(exc, match=text):
+            plan.step(*args, 1)
+        with pytest.raises(exc, match=text):
+            plan.step_bucket(0, *args, 1)
+    meta = torch.zeros(n, dtype=torch.bfloat16, device="meta")
+    with pytest.raises(ValueError, match="host_grads\\[0\\]: must be in host memory"):
+        plan.step_host([meta, meta], [None, None], None, None, None, None, out, 1)
+    with pytest.raises(ValueError, match="g_out: 1 elements"):
+        plan.debug_reduce(g, torch.zeros(1, dtype=torch.float32))
+    with pytest.raises(ValueError, match="out: dtype"):
+        plan.grad_sumsq(g, torch.zeros(1, dtype=torch.float32))
+    plan.close()
