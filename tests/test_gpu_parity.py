@@ -162,6 +162,31 @@ def test_large_step_numbers(t0):
             assert np.array_equal(u16(out)[mine], out_o[mine])
 
 
+def test_thirty_steps_stay_bit_exact():
+    """30 consecutive steps (fresh gradients each step, flat W = 4, ragged
+    tail): fp32 state and the bf16 buffer equal the oracle's bit for bit
+    after every step -- no drift builds up."""
+    shapes = [(50_000,), (3, 1001), (4096 + 3,)]
+    W, cap = 4, 1 << 16
+    oplan = oracle.Plan(shapes, W, 0, cap)
+    P = oplan.padded_numel
+    for r in (0, W - 1):
+        gpu = GpuRank(shapes, W, r, 0, cap, HP, seed=31)
+        orc = OracleRank(oplan, r, seed=31)
+        out_g = torch.zeros(P, dtype=torch.bfloat16, device=DEV)
+        out_o = np.zeros(P, np.uint16)
+        for t in range(1, 31):
+            gpu.fill_grads(t, 1e-3, 0.01)
+            orc.make_grads(t, 1e-3, 0.01)
+            gpu.step(out_g, t)
+            orc.step(out_o, HP, t)
+            torch.cuda.synchronize()
+            for got, want in zip(gpu.state(), (orc.master, orc.m, orc.v)):
+                assert np.array_equal(bits32(got), bits32(want)), (r, t)
+        mine = oplan.owned_global_index(r)
+        assert np.array_equal(u16(out_g)[mine], out_o[mine])
+
+
 def test_max_world_size():
     """W = 512, the ABI's maximum (the pointer array's largest instantiation):
     first, middle and last rank."""
