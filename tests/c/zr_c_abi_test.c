@@ -1,7 +1,8 @@
 /* Plain-C use of the library through include/zr.h: device buffers from
  * cudaMalloc, no Python, no torch.  Builds a plan for one rank of a small
- * flat partition, binds a workspace, runs three steps with constant
- * gradients and checks the closed form of AdamW with a constant gradient:
+ * flat partition, binds a workspace, runs four steps with constant
+ * gradients (the last in checked mode, whose status must stay clean) and
+ * checks the closed form of AdamW with a constant gradient:
  * each step moves p to p * (1 - lr * wd) - lr * g / (|g| + eps) (the bias
  * corrections cancel), within fp32 rounding.  Exit status 0 on success. */
 #include <cuda_runtime.h>
@@ -82,6 +83,16 @@ int main(void) {
 
     for (int64_t t = 1; t <= 3; ++t)
         CHECK_ZR(zr_step(plan, (const void* const*)grads, master, m, v, param_out, t, (zr_stream_t)stream));
+    /* a fourth step in checked mode: the device tables are verified first
+     * and the status stays clean */
+    CHECK_ZR(zr_plan_set_checked(plan, 1));
+    CHECK_ZR(zr_step(plan, (const void* const*)grads, master, m, v, param_out, 4, (zr_stream_t)stream));
+    zr_check_result cr;
+    CHECK_ZR(zr_plan_check_result(plan, &cr, (zr_stream_t)stream));
+    if (cr.bad_tiles != 0 || cr.first_bad != -1 || cr.hash_mismatch != 0 || cr.tables_emptied != 0) {
+        fprintf(stderr, "checked mode flagged a clean plan\n");
+        return 1;
+    }
     CHECK_CUDA(cudaStreamSynchronize(stream));
 
     float* got = (float*)malloc(sizeof(float) * owned);
@@ -92,7 +103,7 @@ int main(void) {
     for (int64_t i = 0; i < owned; ++i) {
         double want = host_p[i];
         const int is_pad = first_global + i >= total;
-        for (int t = 1; t <= 3; ++t) want = want * (1.0 - lr * wd) - (is_pad ? 0.0 : lr * g / (fabs(g) + eps));
+        for (int t = 1; t <= 4; ++t) want = want * (1.0 - lr * wd) - (is_pad ? 0.0 : lr * g / (fabs(g) + eps));
         if (fabs(got[i] - want) > 1e-6 * fmax(fabs(want), lr)) ++bad;
     }
     zr_plan_destroy(plan);
