@@ -162,7 +162,9 @@ zr_status zr_plan_set_sumsq_partials(zr_plan* plan, double* d_partials);
  *            gradient for this rank's owned elements in owned order.
  * master, m, v: fp32 device arrays of owned_numel, updated in place.
  * param_out: bf16 device array of padded_numel (global layout); only this
- *            rank's positions are written.
+ *            rank's positions are written.  (With the ZR_PARAMS_OWNED
+ *            layout, zr_plan_set_param_layout below: this rank's shard,
+ *            owned_numel elements in owned order.)
  * step: 1-based AdamW step count t (bias corrections use it).
  * Every device pointer must be 16-byte aligned.  With owned_numel == 0 it
  * returns ZR_OK and launches nothing.
@@ -223,7 +225,8 @@ zr_status zr_step_finish(const zr_plan* plan, const void* const* grad_ptrs, floa
  * (owned_numel bf16, owned order; pinned host memory for asynchronous
  * copies) into dev_grad_ptrs[w], runs the step, and copies this rank's
  * positions of param_out into host_param_out (a host buffer in the global
- * layout, padded_numel bf16).  The owned range is cut into up to 4 chunks
+ * layout, padded_numel bf16; in owned order, owned_numel bf16, with the
+ * ZR_PARAMS_OWNED layout).  The owned range is cut into up to 4 chunks
  * (1/2, 1/4, 1/8, 1/8 of it): while one chunk's gradients cross PCIe,
  * earlier chunks are stepped and their parameters copied back, on two
  * internal copy streams of the plan
@@ -350,6 +353,40 @@ zr_status zr_state_reshard(const zr_plan* target, const char* const* src_paths, 
 #define ZR_EXPORT_BF16 1
 zr_status zr_state_export_params(const zr_plan* plan, const char* const* src_paths, int32_t n_src,
                                  int32_t dtype, const char* out_path, int64_t* n_written);
+
+/* ZeRO-3 (parameters sharded too): "Scaling training to thousands of GPUs"
+ * (talk summary), section 11:24 ZeRO, and "CS336 lecture 8", section "ZeRO
+ * levels": stage 3 keeps only this rank's slice of the bf16 parameters and
+ * all-gathers each layer's full parameters just before the layer needs
+ * them, a step ahead (prefetch), freeing them after use.
+ *
+ * zr_plan_set_param_layout selects where the step writes the bf16
+ * parameters: ZR_PARAMS_GLOBAL (the default) -- param_out is the full
+ * all-gather buffer (padded_numel elements, global layout); ZR_PARAMS_OWNED
+ * -- param_out is this rank's shard, owned_numel elements in owned order
+ * (the order of master / m / v).  It applies to every step call (zr_step,
+ * zr_step_device_count, zr_step_bucket / zr_step_finish, zr_step_host,
+ * zr_step_no_alloc; zr_step_host then copies the shard back in owned
+ * order).  Changing it rebuilds the tile tables and, when a workspace is
+ * bound, uploads them on `stream` and clears checked mode's status.
+ * ZR_PARAMS_OWNED with gather targets set is ZR_ERR_UNSUPPORTED.
+ *
+ * zr_gather_params writes tensors first_tensor .. first_tensor + n_tensors
+ * - 1 (declaration order), whole and in the global layout, to dst (bf16,
+ * consecutive, row-major; 16-byte aligned), gathered from shard_ptrs[w] =
+ * rank w's bf16 shard in owned order (W device pointers, local or mapped
+ * from other GPUs, 16-byte aligned; NULL allowed for a rank that owns
+ * nothing).
+ * One kernel on `stream`, one CTA per piece of at most 16384 elements of
+ * one tensor and one owner, plain 16-byte loads and stores where source and
+ * destination share their alignment, 2-byte ones otherwise.  Issue it on a
+ * side stream a layer ahead to prefetch.  Errors: ZR_ERR_INVALID_ARG (range,
+ * NULL), ZR_ERR_ALIGNMENT (dst), ZR_ERR_NO_WORKSPACE, ZR_ERR_CUDA. */
+#define ZR_PARAMS_GLOBAL 0
+#define ZR_PARAMS_OWNED 1
+zr_status zr_plan_set_param_layout(zr_plan* plan, int32_t layout, zr_stream_t stream);
+zr_status zr_gather_params(const zr_plan* plan, int32_t first_tensor, int32_t n_tensors,
+                           const void* const* shard_ptrs, void* dst, zr_stream_t stream);
 
 /* Checked mode: a stand-in for a memory sanitizer at run time.  The plan's
  * tile tables live in the caller's workspace, so a kernel that writes there

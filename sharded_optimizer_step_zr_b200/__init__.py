@@ -45,7 +45,7 @@ EXPORTED = [
     "zr_step_finish", "zr_step_host",
     "zr_grad_sumsq", "zr_debug_reduce", "zr_step_no_alloc", "zr_state_save", "zr_state_load",
     "zr_state_reshard", "zr_state_export_params", "zr_plan_set_checked", "zr_plan_verify",
-    "zr_plan_check_result", "zr_plan_owner_offsets", "zr_plan_set_gather_targets", "zr_ipc_export",
+    "zr_plan_check_result", "zr_plan_set_param_layout", "zr_gather_params", "zr_plan_owner_offsets", "zr_plan_set_gather_targets", "zr_ipc_export",
     "zr_ipc_open", "zr_ipc_close", "zr_plan_destroy", "zr_status_string",
 ]
 ZR_NO_ALLOC_SCRATCH_BYTES = 4 << 20
@@ -94,6 +94,8 @@ _lib.zr_state_load.argtypes = [_vp, ctypes.c_char_p, _vp, _vp, _vp, _P(_i64), _v
 _lib.zr_state_reshard.argtypes = [_vp, _vp, _i32, ctypes.c_char_p]
 _lib.zr_state_export_params.argtypes = [_vp, _vp, _i32, _i32, ctypes.c_char_p, _vp]
 _lib.zr_plan_set_checked.argtypes = [_vp, _i32]
+_lib.zr_plan_set_param_layout.argtypes = [_vp, _i32, _vp]
+_lib.zr_gather_params.argtypes = [_vp, _i32, _i32, _vp, _vp, _vp]
 _lib.zr_plan_verify.argtypes = [_vp, _vp]
 _lib.zr_plan_check_result.argtypes = [_vp, _P(zr_check_result), _vp]
 _lib.zr_plan_owner_offsets.argtypes = [_vp, _vp]
@@ -292,6 +294,20 @@ def zr_state_export_params(plan: int, src_paths, dtype: int, out_path: str) -> i
     _check(_lib.zr_state_export_params(plan, arr, len(src_paths), int(dtype), os.fsencode(out_path),
                                        ctypes.byref(n)), "zr_state_export_params")
     return n.value
+
+
+ZR_PARAMS_GLOBAL = 0
+ZR_PARAMS_OWNED = 1
+
+
+def zr_plan_set_param_layout(plan: int, layout: int, stream=None) -> None:
+    _check(_lib.zr_plan_set_param_layout(plan, int(layout), _stream(stream)), "zr_plan_set_param_layout")
+
+
+def zr_gather_params(plan: int, first_tensor: int, n_tensors: int, shards, dst, stream=None) -> None:
+    arr = _ptr_array(shards)
+    _check(_lib.zr_gather_params(plan, int(first_tensor), int(n_tensors), arr, _addr(dst), _stream(stream)),
+           "zr_gather_params")
 
 
 def zr_plan_set_checked(plan: int, enable: bool) -> None:

@@ -69,6 +69,26 @@ zr_status verify_if_checked(const zr_plan* p, zr_stream_t stream) {
     return p->checked ? verify_tables(p, stream) : ZR_OK;
 }
 
+// The tile tables to the workspace on `stream`, with checked mode's
+// reference hashes and fresh status words (no failure, smallest failing
+// position all ones).
+zr_status upload_tiles(zr_plan* p, zr_stream_t stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (!p->tiles.empty()) {
+        const size_t bytes_tiles = sizeof(zr::Tile) * p->tiles.size();
+        if (cudaMemcpyAsync(p->d_tiles, p->tiles.data(), bytes_tiles, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(p->d_tiles_by_owned, p->tiles_by_owned.data(), bytes_tiles, cudaMemcpyHostToDevice, s) !=
+                cudaSuccess)
+            return ZR_ERR_CUDA;
+    }
+    p->hash_tiles = zr::table_hash(p->tiles);
+    p->hash_tiles_by_owned = zr::table_hash(p->tiles_by_owned);
+    if (cudaMemsetAsync(p->d_check, 0, sizeof(uint64_t) * zr::kCheckWords, s) != cudaSuccess ||
+        cudaMemsetAsync(p->d_check + 1, 0xFF, sizeof(uint64_t), s) != cudaSuccess)
+        return ZR_ERR_CUDA;
+    return ZR_OK;
+}
+
 zr_status check_state(const float* master, const float* m, const float* v) {
     if (!master || !m || !v) return ZR_ERR_INVALID_ARG;
     if (!aligned16(master) || !aligned16(m) || !aligned16(v)) return ZR_ERR_ALIGNMENT;
@@ -210,22 +230,51 @@ zr_status zr_plan_set_workspace(zr_plan* p, void* d_ws, uint64_t bytes, zr_strea
     p->d_check = reinterpret_cast<uint64_t*>(base + L.check);
     p->n_gather_targets = 0;
     p->d_g_scratch = p->clip_uses_scratch() ? reinterpret_cast<float*>(base + L.g_scratch) : nullptr;
+    p->d_gather_pieces = reinterpret_cast<zr::GatherPiece*>(base + L.gather_pieces);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (!p->tiles.empty()) {
-        const size_t bytes_tiles = sizeof(zr::Tile) * p->tiles.size();
-        if (cudaMemcpyAsync(p->d_tiles, p->tiles.data(), bytes_tiles, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-            cudaMemcpyAsync(p->d_tiles_by_owned, p->tiles_by_owned.data(), bytes_tiles, cudaMemcpyHostToDevice, s) !=
-                cudaSuccess)
-            return ZR_ERR_CUDA;
-    }
-    // Checked mode's reference hashes and fresh status words (no failure,
-    // smallest failing position all ones).
-    p->hash_tiles = zr::table_hash(p->tiles);
-    p->hash_tiles_by_owned = zr::table_hash(p->tiles_by_owned);
-    if (cudaMemsetAsync(p->d_check, 0, sizeof(uint64_t) * zr::kCheckWords, s) != cudaSuccess ||
-        cudaMemsetAsync(p->d_check + 1, 0xFF, sizeof(uint64_t), s) != cudaSuccess)
+    if (!p->gather_pieces.empty() &&
+        cudaMemcpyAsync(p->d_gather_pieces, p->gather_pieces.data(), sizeof(zr::GatherPiece) * p->gather_pieces.size(),
+                        cudaMemcpyHostToDevice, s) != cudaSuccess)
         return ZR_ERR_CUDA;
-    return ZR_OK;
+    return upload_tiles(p, stream);
+}
+
+zr_status zr_plan_set_param_layout(zr_plan* p, int32_t layout, zr_stream_t stream) {
+    if (!p || (layout != ZR_PARAMS_GLOBAL && layout != ZR_PARAMS_OWNED)) return ZR_ERR_INVALID_ARG;
+    if (layout == ZR_PARAMS_OWNED && p->n_gather_targets > 0) return ZR_ERR_UNSUPPORTED;
+    if (layout == p->param_layout) return ZR_OK;
+    if (p->d_workspace) {
+        const zr_status dst = check_device(p);
+        if (dst != ZR_OK) return dst;
+    }
+    p->param_layout = layout;
+    try {
+        zr::build_tiles_for_layout(*p);
+    } catch (...) {
+        return ZR_ERR_INVALID_ARG;
+    }
+    return p->d_workspace ? upload_tiles(p, stream) : ZR_OK;
+}
+
+zr_status zr_gather_params(const zr_plan* p, int32_t first_tensor, int32_t n_tensors, const void* const* shard_ptrs,
+                           void* dst, zr_stream_t stream) {
+    if (!p || !shard_ptrs || first_tensor < 0 || n_tensors < 0 || first_tensor > p->n_tensors - n_tensors)
+        return ZR_ERR_INVALID_ARG;
+    if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
+    const zr_status dst_st = check_device(p);
+    if (dst_st != ZR_OK) return dst_st;
+    const int32_t a = p->tensor_first_piece[first_tensor], b = p->tensor_first_piece[first_tensor + n_tensors];
+    if (a == b) return ZR_OK;   // only zero-element tensors
+    if (!dst) return ZR_ERR_INVALID_ARG;
+    if (!aligned16(dst)) return ZR_ERR_ALIGNMENT;
+    for (int32_t w = 0; w < p->world_size; ++w) {
+        if (p->rank_numel[w] == 0) continue;
+        if (!shard_ptrs[w]) return ZR_ERR_INVALID_ARG;
+        if (!aligned16(shard_ptrs[w])) return ZR_ERR_ALIGNMENT;
+    }
+    return cuda_status(static_cast<cudaError_t>(zr::launch_gather(p->d_gather_pieces, a, b - a, p->world_size,
+                                                                  shard_ptrs, static_cast<uint16_t*>(dst),
+                                                                  p->goff[first_tensor], stream)));
 }
 
 zr_status zr_plan_set_checked(zr_plan* p, int32_t enable) {
@@ -286,6 +335,7 @@ zr_status zr_plan_set_gather_targets(zr_plan* p, void* const* targets, zr_stream
         p->n_gather_targets = 0;
         return ZR_OK;
     }
+    if (p->param_layout == ZR_PARAMS_OWNED) return ZR_ERR_UNSUPPORTED;   // a shard is not gathered by the step
     for (int32_t w = 0; w < p->world_size; ++w) {
         if (!targets[w]) return ZR_ERR_INVALID_ARG;
         if (!aligned16(targets[w])) return ZR_ERR_ALIGNMENT;

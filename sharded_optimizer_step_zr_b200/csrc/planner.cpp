@@ -171,6 +171,34 @@ void build_tiles(zr_plan& p) {
               [](const Tile& x, const Tile& y) { return x.owned < y.owned; });
 }
 
+// The ZeRO-3 gather's pieces: every tensor's segments (all owners) in order
+// of their offset in the tensor, each cut into pieces of at most
+// kGatherPieceElems elements.
+void build_gather_pieces(zr_plan& p) {
+    p.gather_pieces.clear();
+    p.tensor_first_piece.assign(p.n_tensors + 1, 0);
+    std::vector<std::vector<const zr_segment*>> by_tensor(p.n_tensors);
+    for (const zr_segment& s : p.segments)
+        if (s.tensor >= 0) by_tensor[s.tensor].push_back(&s);
+    for (int32_t t = 0; t < p.n_tensors; ++t) {
+        p.tensor_first_piece[t] = static_cast<int32_t>(p.gather_pieces.size());
+        std::sort(by_tensor[t].begin(), by_tensor[t].end(),
+                  [](const zr_segment* a, const zr_segment* b) { return a->offset_in_tensor < b->offset_in_tensor; });
+        for (const zr_segment* s : by_tensor[t]) {
+            for (int64_t done = 0; done < s->length; done += kGatherPieceElems) {
+                GatherPiece g{};
+                g.src = s->owned_offset + done;
+                g.dst = s->global_offset + done;
+                g.len = static_cast<int32_t>(std::min<int64_t>(kGatherPieceElems, s->length - done));
+                g.owner = s->owner;
+                g.tensor = t;
+                p.gather_pieces.push_back(g);
+            }
+        }
+    }
+    p.tensor_first_piece[p.n_tensors] = static_cast<int32_t>(p.gather_pieces.size());
+}
+
 // Self-check of the tile list before anything reaches a kernel: the tiles
 // cover this rank's owned range [0, owned) exactly once, each maps owned
 // offsets to the same global offsets as the segment it came from, stays
@@ -243,7 +271,20 @@ zr_status build_plan(zr_plan& p, int32_t n_tensors, const int32_t* ndims,
     cut_segments(p);
     build_tiles(p);
     if (!tiles_are_consistent(p)) return ZR_ERR_INVALID_ARG;
+    build_gather_pieces(p);
+    if (p.gather_pieces.size() > 0x7FFFFFFFull) return ZR_ERR_UNSUPPORTED;
     return ZR_OK;
+}
+
+void build_tiles_for_layout(zr_plan& p) {
+    build_tiles(p);
+    if (p.param_layout != ZR_PARAMS_OWNED) return;
+    for (std::vector<Tile>* table : {&p.tiles, &p.tiles_by_owned}) {
+        for (Tile& t : *table) {
+            t.global = t.owned;
+            if (t.flags & kTileVector) t.flags |= kTileStoreVector;   // owned offsets of vector tiles are 8-aligned
+        }
+    }
 }
 
 static uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
@@ -267,6 +308,8 @@ WorkspaceLayout workspace_layout(const zr_plan& p) {
     off = align256(off + sizeof(AdamScalars));
     L.check = off;
     off = align256(off + sizeof(uint64_t) * kCheckWords);
+    L.gather_pieces = off;
+    off = align256(off + sizeof(GatherPiece) * std::max<size_t>(1, p.gather_pieces.size()));
     L.g_scratch = off;
     off = align256(off + (p.clip_uses_scratch() ? sizeof(float) * static_cast<uint64_t>(p.owned_numel()) : 0));
     L.total = off;

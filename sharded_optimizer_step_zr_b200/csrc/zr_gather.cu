@@ -1,0 +1,89 @@
+// ZeRO-3 parameter gather: whole tensors assembled from every rank's bf16
+// shard ("Scaling training to thousands of GPUs", talk summary, section
+// 11:24 ZeRO; "CS336 lecture 8", section "ZeRO levels": stage 3 all-gathers
+// a layer's parameters just before the layer runs).
+//
+// A pure copy, so the roofline is memory bandwidth: 2 bytes read from the
+// owner's shard and 2 written per element -- over NVLink for the elements
+// other GPUs own, when the shard pointers are peer mappings.  One CTA per
+// piece (at most 16384 elements of one tensor from one owner, a 32 KB run):
+// enough CTAs for one transformer layer to cover the 148 SMs several times,
+// and each CTA fetches its own data with plain loads (no TMA, no multicast).
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "zr_internal.hpp"
+
+namespace zr {
+namespace {
+
+template <int CAP>
+struct ShardPtrs {
+    const uint16_t* p[CAP];
+};
+
+constexpr int kGatherThreads = 256;
+constexpr int kGatherUnroll = 4;   // 16-byte vectors in flight per thread
+
+// Source and destination share their offset modulo 16 bytes: a scalar head
+// brings both to a 16-byte boundary, then 16-byte vectors (the loads of
+// kGatherUnroll of them issued before their stores), then a scalar tail.
+// Otherwise the piece is copied element by element.
+template <int CAP>
+__global__ void __launch_bounds__(kGatherThreads)
+zr_gather_kernel(const ShardPtrs<CAP> sp, const GatherPiece* __restrict__ pieces, int32_t first,
+                 uint16_t* dst, int64_t dst_base) {
+    const GatherPiece pc = pieces[first + blockIdx.x];
+    const uint16_t* src = sp.p[pc.owner] + pc.src;
+    uint16_t* out = dst + (pc.dst - dst_base);
+    const int32_t len = pc.len;
+    const uintptr_t sa = reinterpret_cast<uintptr_t>(src), da = reinterpret_cast<uintptr_t>(out);
+    if (((sa ^ da) & 15u) != 0) {
+        for (int32_t i = threadIdx.x; i < len; i += kGatherThreads) out[i] = src[i];
+        return;
+    }
+    int32_t head = static_cast<int32_t>(((16u - (da & 15u)) & 15u) >> 1);   // 0..7 elements
+    if (head > len) head = len;
+    if (static_cast<int32_t>(threadIdx.x) < head) out[threadIdx.x] = src[threadIdx.x];
+    const int32_t nvec = (len - head) >> 3;
+    const uint4* s4 = reinterpret_cast<const uint4*>(src + head);
+    uint4* d4 = reinterpret_cast<uint4*>(out + head);
+    for (int32_t v0 = threadIdx.x; v0 < nvec; v0 += kGatherThreads * kGatherUnroll) {
+        uint4 q[kGatherUnroll];
+#pragma unroll
+        for (int k = 0; k < kGatherUnroll; ++k) {
+            const int32_t v = v0 + k * kGatherThreads;
+            if (v < nvec) q[k] = s4[v];
+        }
+#pragma unroll
+        for (int k = 0; k < kGatherUnroll; ++k) {
+            const int32_t v = v0 + k * kGatherThreads;
+            if (v < nvec) d4[v] = q[k];
+        }
+    }
+    for (int32_t i = head + (nvec << 3) + threadIdx.x; i < len; i += kGatherThreads) out[i] = src[i];
+}
+
+template <int CAP>
+cudaError_t launch_gather_cap(const GatherPiece* pieces, int32_t first, int32_t n, int32_t world_size,
+                              const void* const* shard_ptrs, uint16_t* dst, int64_t dst_base, cudaStream_t s) {
+    ShardPtrs<CAP> sp;
+    for (int w = 0; w < CAP; ++w)
+        sp.p[w] = w < world_size ? static_cast<const uint16_t*>(shard_ptrs[w]) : nullptr;
+    zr_gather_kernel<CAP><<<n, kGatherThreads, 0, s>>>(sp, pieces, first, dst, dst_base);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int launch_gather(const GatherPiece* pieces, int32_t first, int32_t n, int32_t world_size,
+                  const void* const* shard_ptrs, uint16_t* dst, int64_t dst_base, void* stream_v) {
+    if (n == 0) return cudaSuccess;
+    cudaStream_t s = static_cast<cudaStream_t>(stream_v);
+    if (world_size <= 8) return launch_gather_cap<8>(pieces, first, n, world_size, shard_ptrs, dst, dst_base, s);
+    if (world_size <= 64) return launch_gather_cap<64>(pieces, first, n, world_size, shard_ptrs, dst, dst_base, s);
+    return launch_gather_cap<ZR_MAX_WORLD_SIZE>(pieces, first, n, world_size, shard_ptrs, dst, dst_base, s);
+}
+
+}  // namespace zr

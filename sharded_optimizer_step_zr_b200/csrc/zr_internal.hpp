@@ -60,6 +60,21 @@ constexpr int kTileWords = static_cast<int>(sizeof(Tile) / sizeof(uint64_t));   
 // blocks (words 3-5 are 0 between checks).
 constexpr int kCheckWords = 6;
 
+// A piece of the ZeRO-3 parameter gather: `len` consecutive elements of one
+// tensor that one rank owns, copied from that rank's bf16 shard (owned
+// order, offset `src`) to the global position `dst`.  Pieces never cross a
+// tensor or an owner boundary and hold at most kGatherPieceElems elements.
+struct GatherPiece {
+    int64_t src;
+    int64_t dst;
+    int32_t len;
+    int32_t owner;
+    int32_t tensor;
+    int32_t reserved;
+};
+static_assert(sizeof(GatherPiece) == 32, "GatherPiece is 32 bytes");
+constexpr int32_t kGatherPieceElems = 16384;   // 32 KB of bf16: one CTA's share
+
 // AdamW scalars for one step, fp64 on the host rounded once to fp32.
 struct AdamScalars {
     float beta1, beta2, one_minus_beta1, one_minus_beta2;
@@ -105,6 +120,12 @@ int launch_device_scalars(int64_t* d_step, const zr_adamw& hp, AdamScalars* out,
 int launch_clip_combine(const double* tile_partials, int32_t n_tiles, double* partials_all,
                         int32_t world_size, int32_t rank, float max_norm, float* clip_coef_out,
                         double* sumsq_out, void* stream);
+// ZeRO-3 gather: copy pieces [first, first + n) from the W shards to dst,
+// where dst holds the global range starting at dst_base.  shard_ptrs: host
+// array of W device pointers (any may be NULL for a rank owning nothing).
+int launch_gather(const GatherPiece* pieces, int32_t first, int32_t n, int32_t world_size,
+                  const void* const* shard_ptrs, uint16_t* dst, int64_t dst_base, void* stream);
+
 // Checked mode: verify both device tile tables against the tile invariants
 // and the hashes taken on the host at upload, then, if anything failed (now
 // or before), overwrite both tables with empty tiles.  One launch; `check`
@@ -155,6 +176,10 @@ struct zr_plan {
     zr::AdamScalars* d_scalars = nullptr;  // workspace: scalars computed on the device
     int32_t n_gather_targets = 0;          // 0 until zr_plan_set_gather_targets
     uint64_t* d_check = nullptr;           // workspace: checked mode's status words
+    int32_t param_layout = ZR_PARAMS_GLOBAL;   // where zr_step writes the bf16 parameters
+    std::vector<zr::GatherPiece> gather_pieces;     // all ranks, tensor by tensor
+    std::vector<int32_t> tensor_first_piece;        // n_tensors + 1 entries
+    zr::GatherPiece* d_gather_pieces = nullptr;     // workspace copy
     bool checked = false;                  // verify the tables before every launch
     uint64_t hash_tiles = 0;               // tile_word_hash sums of the two host tables
     uint64_t hash_tiles_by_owned = 0;
@@ -181,9 +206,14 @@ zr_status build_plan(zr_plan& p, int32_t n_tensors, const int32_t* ndims,
 // Workspace layout: offsets of each region, total bytes.
 struct WorkspaceLayout {
     uint64_t tiles, tiles_by_owned, tile_partials, clip_coef, own_sumsq, gather_targets, dev_scalars, check,
-        g_scratch, total;
+        gather_pieces, g_scratch, total;
 };
 WorkspaceLayout workspace_layout(const zr_plan& p);
+// Rebuilds this rank's tile tables for the plan's parameter layout: the
+// global layout as planned, or (ZR_PARAMS_OWNED) with every tile's output
+// offset moved to its owned offset, so the same kernels write the rank's
+// bf16 shard in owned order.
+void build_tiles_for_layout(zr_plan& p);
 uint64_t table_hash(const std::vector<Tile>& tiles);
 AdamScalars adam_scalars(const zr_adamw& hp, int64_t step);
 }  // namespace zr

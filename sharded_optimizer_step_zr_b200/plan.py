@@ -5,8 +5,9 @@ libzr.so's kernels through the C ABI.
 """
 from __future__ import annotations
 
-from . import (ZR_PARTITION_FLAT, zr_debug_reduce, zr_grad_sumsq, zr_plan_check_result, zr_plan_create,
-               zr_plan_destroy, zr_plan_query, zr_plan_segments, zr_plan_set_checked, zr_plan_set_sumsq_partials,
+from . import (ZR_PARAMS_GLOBAL, ZR_PARAMS_OWNED, ZR_PARTITION_FLAT, zr_debug_reduce, zr_gather_params,
+               zr_grad_sumsq, zr_plan_check_result, zr_plan_create, zr_plan_destroy, zr_plan_query,
+               zr_plan_segments, zr_plan_set_checked, zr_plan_set_param_layout, zr_plan_set_sumsq_partials,
                zr_plan_set_workspace, zr_plan_verify, zr_plan_workspace_bytes, zr_step, zr_step_bucket,
                zr_step_finish, zr_step_host)
 
@@ -58,6 +59,7 @@ class ZrPlan:
         self.n_buckets = info["n_buckets"]
         self.workspace_bytes = zr_plan_workspace_bytes(self.handle)
         self.device = None
+        self.param_layout = ZR_PARAMS_GLOBAL
         self.workspace = None
         self.partials = None
         if bind:
@@ -104,8 +106,23 @@ class ZrPlan:
             specs += [(g, f"grads[{w}]", torch.bfloat16, self.owned_numel, False) for w, g in enumerate(grads)]
         specs += [(x, name, torch.float32, self.owned_numel, False) for x, name in ((master, "master"), (m, "m"),
                                                                                       (v, "v"))]
-        specs.append((param_out, "param_out", torch.bfloat16, self.padded_numel, False))
+        specs.append((param_out, "param_out", torch.bfloat16, self.param_out_numel, False))
         return specs
+
+    @property
+    def param_out_numel(self):
+        """Elements of the buffer the step writes bf16 parameters into: the
+        full all-gather buffer, or this rank's shard (ZR_PARAMS_OWNED)."""
+        return self.owned_numel if self.param_layout == ZR_PARAMS_OWNED else self.padded_numel
+
+    def set_param_layout(self, layout, stream=None):
+        zr_plan_set_param_layout(self.handle, layout, stream)
+        self.param_layout = layout
+
+    def gather_params(self, first_tensor, n_tensors, shards, dst, stream=None):
+        """Tensors [first_tensor, first_tensor + n_tensors) whole, in the
+        global layout, into dst, from every rank's bf16 shard (owned order)."""
+        zr_gather_params(self.handle, first_tensor, n_tensors, shards, dst, stream)
 
     def step(self, grads, master, m, v, param_out, step, stream=None):
         self.check_step_buffers(grads, master, m, v, param_out)
@@ -145,7 +162,7 @@ class ZrPlan:
                 raise ValueError(f"host_grads: {len(host_grads)} buffers, the plan has W = {self.world_size}")
             specs += [(g, f"host_grads[{w}]", torch.bfloat16, self.owned_numel, True)
                       for w, g in enumerate(host_grads)]
-            specs.append((host_param_out, "host_param_out", torch.bfloat16, self.padded_numel, True))
+            specs.append((host_param_out, "host_param_out", torch.bfloat16, self.param_out_numel, True))
         _require_all(specs, self.device)
         zr_step_host(self.handle, host_grads, dev_grads, master, m, v, param_out, host_param_out,
                      step, stream)

@@ -232,3 +232,20 @@ def test_plan_rejects_wrong_buffers_before_the_library():
     with pytest.raises(ValueError, match="out: dtype"):
         plan.grad_sumsq(g, torch.zeros(1, dtype=torch.float32))
     plan.close()
+
+
+def test_zero3_calls_without_a_device():
+    """The parameter layout switch is host-side until a workspace is bound;
+    the gather rejects bad tensor ranges, then an unbound workspace."""
+    h = zr.zr_plan_create([(4096,), (0,), (100,)], 2, 0, 1, 1 << 20)
+    try:
+        zr.zr_plan_set_param_layout(h, zr.ZR_PARAMS_OWNED, 0)
+        zr.zr_plan_set_param_layout(h, zr.ZR_PARAMS_GLOBAL, 0)
+        assert zr._lib.zr_plan_set_param_layout(h, 5, None) == zr.ZR_ERR_INVALID_ARG
+        arr = zr._ptr_array([0, 0])
+        for first, n in ((-1, 1), (0, 4), (3, 1), (2, 2), (0, -1)):
+            assert zr._lib.zr_gather_params(h, first, n, arr, None, None) == zr.ZR_ERR_INVALID_ARG
+        assert zr._lib.zr_gather_params(h, 0, 3, None, None, None) == zr.ZR_ERR_INVALID_ARG
+        assert zr._lib.zr_gather_params(h, 0, 3, arr, None, None) == zr.ZR_ERR_NO_WORKSPACE
+    finally:
+        zr.zr_plan_destroy(h)
