@@ -60,6 +60,8 @@ def parse():
     ap.add_argument("--overlap", action="store_true",
                     help="exposed optimizer time behind an emulated backward pass: one zr_step "
                          "after it, against zr_step_bucket as each bucket's gradients complete")
+    ap.add_argument("--zero3", action="store_true",
+                    help="ZeRO-3 parameter gather: bandwidth, and prefetch against an emulated forward")
     ap.add_argument("--checked", action="store_true",
                     help="checked mode: the device tile tables verified before every launch")
     ap.add_argument("--sweep", action="store_true",
@@ -712,10 +714,123 @@ def run_overlap(args):
                       "exposed_ms_per_bucket": ovl_ms - back_ms}), flush=True)
 
 
+def run_zero3(args):
+    """ZeRO-3 parameter gather on the 1.3B set, flat, W = 8: every rank's
+    bf16 shard resident on this GPU (standing in for peer mappings).
+
+    Measured: (a) one zr_gather_params of the whole model and of one
+    transformer block, against the copy roofline (2 bytes read + 2 written
+    per element); (b) an emulated forward -- per block one bf16 matmul of
+    about the block's FLOPs at 8192 tokens -- run with the block's gather
+    in front of it on the same stream (in line), or with block i + 1's
+    gather issued on a side stream while block i computes (prefetch).  The
+    gather time left exposed is the difference from the forward alone.
+    Prints one JSON record."""
+    import torch
+    import synth
+    from sharded_optimizer_step_zr_b200 import ZR_PARAMS_OWNED
+    from sharded_optimizer_step_zr_b200.plan import ZrPlan
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    wl = next(w for w in synth.sweep_workloads() if w.name == "sweep_1p3b_flat_w8_cap25")
+    W = wl.world_size
+    plans = [ZrPlan(wl.shapes, W, r, wl.mode, wl.bucket_cap_bytes, *wl.hp, device=dev, bind=(r == 0))
+             for r in range(W)]
+    plan = plans[0]
+    plan.set_param_layout(ZR_PARAMS_OWNED)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(wl.seed)
+    shards = [torch.randn(p.owned_numel, device=dev, generator=gen).to(torch.bfloat16) for p in plans]
+    for p in plans[1:]:
+        p.close()
+    numels = [int(math.prod(s)) for s in wl.shapes]
+    # GPT blocks: tensors 2 + 12 i .. 2 + 12 i + 11 (wte and wpe first, ln_f last)
+    n_blocks, per_block = 24, 12
+    block_params = sum(numels[2:2 + per_block])
+    layer_buf = [torch.empty(block_params, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    full = torch.empty(sum(numels), dtype=torch.bfloat16, device=dev)
+    peak, peak_kind = measured_peak()
+
+    def timed(fn, reps, stream=None):
+        stream = stream or torch.cuda.current_stream()
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps * 1e3    # us
+
+    whole_us = timed(lambda: plan.gather_params(0, len(numels), shards, full), 20)
+    block_us = timed(lambda: plan.gather_params(2, per_block, shards, layer_buf[0]), 200)
+    gb = lambda elems, us: 4 * elems / (us * 1e-6) / 1e9
+
+    # emulated forward: per block [8192, 2048] x [2048, 24576] bf16, 2 * 8192 * 12 * 2048^2 flops --
+    # a 1.3B block's forward (12 d^2 weights) at 8192 tokens
+    x = torch.randn(8192, 2048, dtype=torch.bfloat16, device=dev)
+    w_ = torch.randn(2048, 24576, dtype=torch.bfloat16, device=dev)
+    compute, side = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def forward_only():
+        with torch.cuda.stream(compute):
+            for _ in range(n_blocks):
+                torch.matmul(x, w_)
+
+    def forward_sequential():
+        with torch.cuda.stream(compute):
+            for i in range(n_blocks):
+                plan.gather_params(2 + per_block * i, per_block, shards, layer_buf[i % 2], compute)
+                torch.matmul(x, w_)
+
+    ready = [torch.cuda.Event() for _ in range(n_blocks)]
+    done = [torch.cuda.Event() for _ in range(n_blocks)]
+
+    def forward_prefetch():
+        side.wait_stream(compute)
+        with torch.cuda.stream(side):
+            plan.gather_params(2, per_block, shards, layer_buf[0], side)
+            ready[0].record(side)
+        for i in range(n_blocks):
+            if i + 1 < n_blocks:
+                with torch.cuda.stream(side):
+                    if i >= 1:
+                        side.wait_event(done[i - 1])          # buffer (i + 1) % 2 was block i - 1's
+                    plan.gather_params(2 + per_block * (i + 1), per_block, shards, layer_buf[(i + 1) % 2], side)
+                    ready[i + 1].record(side)
+            with torch.cuda.stream(compute):
+                compute.wait_event(ready[i])
+                torch.matmul(x, w_)
+                done[i].record(compute)
+
+    t_fwd = timed(forward_only, 10, compute)
+    t_seq = timed(forward_sequential, 10, compute)
+    t_pre = timed(forward_prefetch, 10, compute)
+    line = {
+        "mode": "zero3_gather", "workload": "gpt_1p3b flat W=8, all ranks' shards on one GPU",
+        "params": sum(numels), "block_params": block_params, "unit": "us",
+        "gather_whole_model_us": whole_us, "gather_whole_model_gbs": gb(sum(numels), whole_us),
+        "gather_block_us": block_us, "gather_block_gbs": gb(block_params, block_us),
+        "roofline": {"bound": "hbm", "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
+                     "bytes_per_element": 4, "frac_whole_model": gb(sum(numels), whole_us) / peak,
+                     "frac_block": gb(block_params, block_us) / peak},
+        "forward_only_us": t_fwd, "forward_gather_in_line_us": t_seq, "forward_gather_prefetched_us": t_pre,
+        "exposed_gather_in_line_us": t_seq - t_fwd, "exposed_gather_prefetched_us": t_pre - t_fwd,
+        "blocks": n_blocks,
+    }
+    print(json.dumps(line), flush=True)
+    plan.close()
+
+
 def main():
     args = parse()
     if args.overlap:
         run_overlap(args)
+        return
+    if args.zero3:
+        run_zero3(args)
         return
     if args.sweep:
         run_sweep(args)
