@@ -772,7 +772,10 @@ def run_zero3(args):
     # a 1.3B block's forward (12 d^2 weights) at 8192 tokens
     x = torch.randn(8192, 2048, dtype=torch.bfloat16, device=dev)
     w_ = torch.randn(2048, 24576, dtype=torch.bfloat16, device=dev)
-    compute, side = torch.cuda.Stream(), torch.cuda.Stream()
+    compute = torch.cuda.Stream()
+    lo, hi = torch.cuda.Stream.priority_range() if hasattr(torch.cuda.Stream, "priority_range") else (0, -1)
+    side_streams = {"default": torch.cuda.Stream(), "high": torch.cuda.Stream(priority=hi)}
+    side = side_streams["default"]
 
     def forward_only():
         with torch.cuda.stream(compute):
@@ -788,17 +791,20 @@ def run_zero3(args):
     ready = [torch.cuda.Event() for _ in range(n_blocks)]
     done = [torch.cuda.Event() for _ in range(n_blocks)]
 
+    cap = 0
+
     def forward_prefetch():
         side.wait_stream(compute)
         with torch.cuda.stream(side):
-            plan.gather_params(2, per_block, shards, layer_buf[0], side)
+            plan.gather_params(2, per_block, shards, layer_buf[0], side, cap)
             ready[0].record(side)
         for i in range(n_blocks):
             if i + 1 < n_blocks:
                 with torch.cuda.stream(side):
                     if i >= 1:
                         side.wait_event(done[i - 1])          # buffer (i + 1) % 2 was block i - 1's
-                    plan.gather_params(2 + per_block * (i + 1), per_block, shards, layer_buf[(i + 1) % 2], side)
+                    plan.gather_params(2 + per_block * (i + 1), per_block, shards, layer_buf[(i + 1) % 2], side,
+                                       cap)
                     ready[i + 1].record(side)
             with torch.cuda.stream(compute):
                 compute.wait_event(ready[i])
@@ -807,7 +813,13 @@ def run_zero3(args):
 
     t_fwd = timed(forward_only, 10, compute)
     t_seq = timed(forward_sequential, 10, compute)
-    t_pre = timed(forward_prefetch, 10, compute)
+    t_pre = {}
+    for name, st, c in (("default", side_streams["default"], 0), ("high", side_streams["high"], 0),
+                        ("high_16_ctas", side_streams["high"], 16), ("high_32_ctas", side_streams["high"], 32)):
+        side, cap = st, c
+        t_pre[name] = timed(forward_prefetch, 10, compute)
+    capped_us = {c: timed(lambda: plan.gather_params(2, per_block, shards, layer_buf[0], None, c), 50)
+                 for c in (16, 32)}
     line = {
         "mode": "zero3_gather", "workload": "gpt_1p3b flat W=8, all ranks' shards on one GPU",
         "params": sum(numels), "block_params": block_params, "unit": "us",
@@ -816,8 +828,11 @@ def run_zero3(args):
         "roofline": {"bound": "hbm", "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
                      "bytes_per_element": 4, "frac_whole_model": gb(sum(numels), whole_us) / peak,
                      "frac_block": gb(block_params, block_us) / peak},
-        "forward_only_us": t_fwd, "forward_gather_in_line_us": t_seq, "forward_gather_prefetched_us": t_pre,
-        "exposed_gather_in_line_us": t_seq - t_fwd, "exposed_gather_prefetched_us": t_pre - t_fwd,
+        "forward_only_us": t_fwd, "forward_gather_in_line_us": t_seq,
+        "gather_block_16_ctas_us": capped_us[16], "gather_block_32_ctas_us": capped_us[32],
+        "forward_gather_prefetched_us": t_pre,
+        "exposed_gather_in_line_us": t_seq - t_fwd,
+        "exposed_gather_prefetched_us": {k: v - t_fwd for k, v in t_pre.items()},
         "blocks": n_blocks,
     }
     print(json.dumps(line), flush=True)

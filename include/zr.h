@@ -377,16 +377,19 @@ zr_status zr_state_export_params(const zr_plan* plan, const char* const* src_pat
  * rank w's bf16 shard in owned order (W device pointers, local or mapped
  * from other GPUs, 16-byte aligned; NULL allowed for a rank that owns
  * nothing).
- * One kernel on `stream`, one CTA per piece of at most 16384 elements of
- * one tensor and one owner, plain 16-byte loads and stores where source and
- * destination share their alignment, 2-byte ones otherwise.  Issue it on a
- * side stream a layer ahead to prefetch.  Errors: ZR_ERR_INVALID_ARG (range,
+ * One kernel on `stream`: pieces of at most 16384 elements of one tensor
+ * and one owner, plain 16-byte loads and stores where source and
+ * destination share their alignment, 2-byte ones otherwise, with the
+ * streaming (evict-first) cache hint; one CTA per piece when max_ctas <= 0,
+ * else at most max_ctas CTAs looping over the pieces (for a prefetch that
+ * should leave most SMs to the compute it overlaps).  Issue it on a side
+ * stream a layer ahead to prefetch.  Errors: ZR_ERR_INVALID_ARG (range,
  * NULL), ZR_ERR_ALIGNMENT (dst), ZR_ERR_NO_WORKSPACE, ZR_ERR_CUDA. */
 #define ZR_PARAMS_GLOBAL 0
 #define ZR_PARAMS_OWNED 1
 zr_status zr_plan_set_param_layout(zr_plan* plan, int32_t layout, zr_stream_t stream);
 zr_status zr_gather_params(const zr_plan* plan, int32_t first_tensor, int32_t n_tensors,
-                           const void* const* shard_ptrs, void* dst, zr_stream_t stream);
+                           const void* const* shard_ptrs, void* dst, int32_t max_ctas, zr_stream_t stream);
 
 /* Checked mode: a stand-in for a memory sanitizer at run time.  The plan's
  * tile tables live in the caller's workspace, so a kernel that writes there

@@ -95,7 +95,7 @@ _lib.zr_state_reshard.argtypes = [_vp, _vp, _i32, ctypes.c_char_p]
 _lib.zr_state_export_params.argtypes = [_vp, _vp, _i32, _i32, ctypes.c_char_p, _vp]
 _lib.zr_plan_set_checked.argtypes = [_vp, _i32]
 _lib.zr_plan_set_param_layout.argtypes = [_vp, _i32, _vp]
-_lib.zr_gather_params.argtypes = [_vp, _i32, _i32, _vp, _vp, _vp]
+_lib.zr_gather_params.argtypes = [_vp, _i32, _i32, _vp, _vp, _i32, _vp]
 _lib.zr_plan_verify.argtypes = [_vp, _vp]
 _lib.zr_plan_check_result.argtypes = [_vp, _P(zr_check_result), _vp]
 _lib.zr_plan_owner_offsets.argtypes = [_vp, _vp]
@@ -304,10 +304,11 @@ def zr_plan_set_param_layout(plan: int, layout: int, stream=None) -> None:
     _check(_lib.zr_plan_set_param_layout(plan, int(layout), _stream(stream)), "zr_plan_set_param_layout")
 
 
-def zr_gather_params(plan: int, first_tensor: int, n_tensors: int, shards, dst, stream=None) -> None:
+def zr_gather_params(plan: int, first_tensor: int, n_tensors: int, shards, dst, stream=None,
+                     max_ctas: int = 0) -> None:
     arr = _ptr_array(shards)
-    _check(_lib.zr_gather_params(plan, int(first_tensor), int(n_tensors), arr, _addr(dst), _stream(stream)),
-           "zr_gather_params")
+    _check(_lib.zr_gather_params(plan, int(first_tensor), int(n_tensors), arr, _addr(dst), int(max_ctas),
+                                 _stream(stream)), "zr_gather_params")
 
 
 def zr_plan_set_checked(plan: int, enable: bool) -> None:

@@ -257,7 +257,7 @@ zr_status zr_plan_set_param_layout(zr_plan* p, int32_t layout, zr_stream_t strea
 }
 
 zr_status zr_gather_params(const zr_plan* p, int32_t first_tensor, int32_t n_tensors, const void* const* shard_ptrs,
-                           void* dst, zr_stream_t stream) {
+                           void* dst, int32_t max_ctas, zr_stream_t stream) {
     if (!p || !shard_ptrs || first_tensor < 0 || n_tensors < 0 || first_tensor > p->n_tensors - n_tensors)
         return ZR_ERR_INVALID_ARG;
     if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
@@ -272,9 +272,10 @@ zr_status zr_gather_params(const zr_plan* p, int32_t first_tensor, int32_t n_ten
         if (!shard_ptrs[w]) return ZR_ERR_INVALID_ARG;
         if (!aligned16(shard_ptrs[w])) return ZR_ERR_ALIGNMENT;
     }
-    return cuda_status(static_cast<cudaError_t>(zr::launch_gather(p->d_gather_pieces, a, b - a, p->world_size,
-                                                                  shard_ptrs, static_cast<uint16_t*>(dst),
-                                                                  p->goff[first_tensor], stream)));
+    return cuda_status(static_cast<cudaError_t>(zr::launch_gather(p->d_gather_pieces, a, b - a, max_ctas,
+                                                                  p->world_size, shard_ptrs,
+                                                                  static_cast<uint16_t*>(dst), p->goff[first_tensor],
+                                                                  stream)));
 }
 
 zr_status zr_plan_set_checked(zr_plan* p, int32_t enable) {

@@ -9,6 +9,8 @@
 // piece (at most 16384 elements of one tensor from one owner, a 32 KB run):
 // enough CTAs for one transformer layer to cover the 148 SMs several times,
 // and each CTA fetches its own data with plain loads (no TMA, no multicast).
+// A caller prefetching under compute may cap the grid so the gather runs
+// beside the compute on a few SMs instead of taking all of them.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -26,26 +28,22 @@ struct ShardPtrs {
 constexpr int kGatherThreads = 256;
 constexpr int kGatherUnroll = 4;   // 16-byte vectors in flight per thread
 
-// Source and destination share their offset modulo 16 bytes: a scalar head
-// brings both to a 16-byte boundary, then 16-byte vectors (the loads of
-// kGatherUnroll of them issued before their stores), then a scalar tail.
-// Otherwise the piece is copied element by element.
-template <int CAP>
-__global__ void __launch_bounds__(kGatherThreads)
-zr_gather_kernel(const ShardPtrs<CAP> sp, const GatherPiece* __restrict__ pieces, int32_t first,
-                 uint16_t* dst, int64_t dst_base) {
-    const GatherPiece pc = pieces[first + blockIdx.x];
-    const uint16_t* src = sp.p[pc.owner] + pc.src;
-    uint16_t* out = dst + (pc.dst - dst_base);
-    const int32_t len = pc.len;
+// One piece: source and destination share their offset modulo 16 bytes --
+// a scalar head brings both to a 16-byte boundary, then 16-byte vectors
+// (the loads of kGatherUnroll of them issued before their stores), then a
+// scalar tail; otherwise element by element.  Loads and stores carry the
+// streaming (evict-first) hint: the gathered bytes are used once, by the
+// layer that runs next, and should not push that layer's working set out
+// of L2 while a prefetch overlaps it.
+__device__ __forceinline__ void copy_piece(const uint16_t* src, uint16_t* out, int32_t len) {
     const uintptr_t sa = reinterpret_cast<uintptr_t>(src), da = reinterpret_cast<uintptr_t>(out);
     if (((sa ^ da) & 15u) != 0) {
-        for (int32_t i = threadIdx.x; i < len; i += kGatherThreads) out[i] = src[i];
+        for (int32_t i = threadIdx.x; i < len; i += kGatherThreads) __stcs(out + i, __ldcs(src + i));
         return;
     }
     int32_t head = static_cast<int32_t>(((16u - (da & 15u)) & 15u) >> 1);   // 0..7 elements
     if (head > len) head = len;
-    if (static_cast<int32_t>(threadIdx.x) < head) out[threadIdx.x] = src[threadIdx.x];
+    if (static_cast<int32_t>(threadIdx.x) < head) __stcs(out + threadIdx.x, __ldcs(src + threadIdx.x));
     const int32_t nvec = (len - head) >> 3;
     const uint4* s4 = reinterpret_cast<const uint4*>(src + head);
     uint4* d4 = reinterpret_cast<uint4*>(out + head);
@@ -54,36 +52,52 @@ zr_gather_kernel(const ShardPtrs<CAP> sp, const GatherPiece* __restrict__ pieces
 #pragma unroll
         for (int k = 0; k < kGatherUnroll; ++k) {
             const int32_t v = v0 + k * kGatherThreads;
-            if (v < nvec) q[k] = s4[v];
+            if (v < nvec) q[k] = __ldcs(s4 + v);
         }
 #pragma unroll
         for (int k = 0; k < kGatherUnroll; ++k) {
             const int32_t v = v0 + k * kGatherThreads;
-            if (v < nvec) d4[v] = q[k];
+            if (v < nvec) __stcs(d4 + v, q[k]);
         }
     }
-    for (int32_t i = head + (nvec << 3) + threadIdx.x; i < len; i += kGatherThreads) out[i] = src[i];
+    for (int32_t i = head + (nvec << 3) + threadIdx.x; i < len; i += kGatherThreads)
+        __stcs(out + i, __ldcs(src + i));
+}
+
+// CTA b copies pieces b, b + gridDim.x, ...: one CTA per piece at full
+// speed, or a capped grid that leaves the other SMs to concurrent work.
+template <int CAP>
+__global__ void __launch_bounds__(kGatherThreads)
+zr_gather_kernel(const ShardPtrs<CAP> sp, const GatherPiece* __restrict__ pieces, int32_t first, int32_t n,
+                 uint16_t* dst, int64_t dst_base) {
+    for (int32_t k = blockIdx.x; k < n; k += gridDim.x) {
+        const GatherPiece pc = pieces[first + k];
+        copy_piece(sp.p[pc.owner] + pc.src, dst + (pc.dst - dst_base), pc.len);
+    }
 }
 
 template <int CAP>
-cudaError_t launch_gather_cap(const GatherPiece* pieces, int32_t first, int32_t n, int32_t world_size,
+cudaError_t launch_gather_cap(const GatherPiece* pieces, int32_t first, int32_t n, int32_t ctas, int32_t world_size,
                               const void* const* shard_ptrs, uint16_t* dst, int64_t dst_base, cudaStream_t s) {
     ShardPtrs<CAP> sp;
     for (int w = 0; w < CAP; ++w)
         sp.p[w] = w < world_size ? static_cast<const uint16_t*>(shard_ptrs[w]) : nullptr;
-    zr_gather_kernel<CAP><<<n, kGatherThreads, 0, s>>>(sp, pieces, first, dst, dst_base);
+    zr_gather_kernel<CAP><<<ctas, kGatherThreads, 0, s>>>(sp, pieces, first, n, dst, dst_base);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-int launch_gather(const GatherPiece* pieces, int32_t first, int32_t n, int32_t world_size,
+int launch_gather(const GatherPiece* pieces, int32_t first, int32_t n, int32_t max_ctas, int32_t world_size,
                   const void* const* shard_ptrs, uint16_t* dst, int64_t dst_base, void* stream_v) {
     if (n == 0) return cudaSuccess;
     cudaStream_t s = static_cast<cudaStream_t>(stream_v);
-    if (world_size <= 8) return launch_gather_cap<8>(pieces, first, n, world_size, shard_ptrs, dst, dst_base, s);
-    if (world_size <= 64) return launch_gather_cap<64>(pieces, first, n, world_size, shard_ptrs, dst, dst_base, s);
-    return launch_gather_cap<ZR_MAX_WORLD_SIZE>(pieces, first, n, world_size, shard_ptrs, dst, dst_base, s);
+    const int32_t ctas = (max_ctas > 0 && max_ctas < n) ? max_ctas : n;
+    if (world_size <= 8)
+        return launch_gather_cap<8>(pieces, first, n, ctas, world_size, shard_ptrs, dst, dst_base, s);
+    if (world_size <= 64)
+        return launch_gather_cap<64>(pieces, first, n, ctas, world_size, shard_ptrs, dst, dst_base, s);
+    return launch_gather_cap<ZR_MAX_WORLD_SIZE>(pieces, first, n, ctas, world_size, shard_ptrs, dst, dst_base, s);
 }
 
 }  // namespace zr

@@ -121,9 +121,10 @@ int launch_clip_combine(const double* tile_partials, int32_t n_tiles, double* pa
                         int32_t world_size, int32_t rank, float max_norm, float* clip_coef_out,
                         double* sumsq_out, void* stream);
 // ZeRO-3 gather: copy pieces [first, first + n) from the W shards to dst,
-// where dst holds the global range starting at dst_base.  shard_ptrs: host
+// where dst holds the global range starting at dst_base, on at most
+// max_ctas CTAs (<= 0: one per piece).  shard_ptrs: host
 // array of W device pointers (any may be NULL for a rank owning nothing).
-int launch_gather(const GatherPiece* pieces, int32_t first, int32_t n, int32_t world_size,
+int launch_gather(const GatherPiece* pieces, int32_t first, int32_t n, int32_t max_ctas, int32_t world_size,
                   const void* const* shard_ptrs, uint16_t* dst, int64_t dst_base, void* stream);
 
 // Checked mode: verify both device tile tables against the tile invariants

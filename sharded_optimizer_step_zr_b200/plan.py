@@ -119,10 +119,11 @@ class ZrPlan:
         zr_plan_set_param_layout(self.handle, layout, stream)
         self.param_layout = layout
 
-    def gather_params(self, first_tensor, n_tensors, shards, dst, stream=None):
+    def gather_params(self, first_tensor, n_tensors, shards, dst, stream=None, max_ctas=0):
         """Tensors [first_tensor, first_tensor + n_tensors) whole, in the
-        global layout, into dst, from every rank's bf16 shard (owned order)."""
-        zr_gather_params(self.handle, first_tensor, n_tensors, shards, dst, stream)
+        global layout, into dst, from every rank's bf16 shard (owned order);
+        max_ctas > 0 caps the grid (a prefetch beside compute)."""
+        zr_gather_params(self.handle, first_tensor, n_tensors, shards, dst, stream, max_ctas)
 
     def step(self, grads, master, m, v, param_out, step, stream=None):
         self.check_step_buffers(grads, master, m, v, param_out)

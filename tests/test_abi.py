@@ -244,8 +244,8 @@ def test_zero3_calls_without_a_device():
         assert zr._lib.zr_plan_set_param_layout(h, 5, None) == zr.ZR_ERR_INVALID_ARG
         arr = zr._ptr_array([0, 0])
         for first, n in ((-1, 1), (0, 4), (3, 1), (2, 2), (0, -1)):
-            assert zr._lib.zr_gather_params(h, first, n, arr, None, None) == zr.ZR_ERR_INVALID_ARG
-        assert zr._lib.zr_gather_params(h, 0, 3, None, None, None) == zr.ZR_ERR_INVALID_ARG
-        assert zr._lib.zr_gather_params(h, 0, 3, arr, None, None) == zr.ZR_ERR_NO_WORKSPACE
+            assert zr._lib.zr_gather_params(h, first, n, arr, None, 0, None) == zr.ZR_ERR_INVALID_ARG
+        assert zr._lib.zr_gather_params(h, 0, 3, None, None, 0, None) == zr.ZR_ERR_INVALID_ARG
+        assert zr._lib.zr_gather_params(h, 0, 3, arr, None, 0, None) == zr.ZR_ERR_NO_WORKSPACE
     finally:
         zr.zr_plan_destroy(h)
