@@ -10,12 +10,16 @@ the per-rank sums of squares.
 
 Every replica keeps its full gradient in the plan's owner-major layout
 (``grad_view(t)`` is tensor t's slice of it, for the backward pass to write
-into); ``param_buffer`` holds the full bf16 parameters in the global layout.
+into).  Stages 1 and 2: ``param_buffer`` holds the full bf16 parameters in
+the global layout, written by every rank's step.  Stage 3: each rank keeps
+only ``param_shard``, its bf16 parameters in owned order, and ``gather``
+assembles whole tensors (one layer, ahead of its use) from every rank's
+shard through the same peer mappings.
 """
 from __future__ import annotations
 
-from . import (ZR_PARTITION_FLAT, zr_ipc_close, zr_ipc_export, zr_ipc_open, zr_plan_owner_offsets,
-               zr_plan_set_gather_targets, zr_step)
+from . import (ZR_PARAMS_OWNED, ZR_PARTITION_FLAT, zr_gather_params, zr_ipc_close, zr_ipc_export, zr_ipc_open,
+               zr_plan_owner_offsets, zr_plan_set_gather_targets, zr_step)
 from .plan import ZrPlan
 
 
@@ -38,10 +42,13 @@ def sync_point(dist, group, phase, step):
 
 class PeerZero:
     def __init__(self, group, shapes, mode=ZR_PARTITION_FLAT, bucket_cap_bytes=25 << 20, lr=3e-4,
-                 beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.1, max_grad_norm=0.0, device=None):
+                 beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.1, max_grad_norm=0.0, device=None,
+                 stage=2):
         import torch
         import torch.distributed as dist
-        self.dist, self.group = dist, group
+        if stage not in (1, 2, 3):
+            raise ValueError("stage is 1, 2 or 3")
+        self.dist, self.group, self.stage = dist, group, stage
         self.world_size = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
         device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
@@ -52,24 +59,33 @@ class PeerZero:
         P = self.plan.padded_numel
         # One allocation holds both shared buffers, so each peer maps one
         # IPC handle per rank: the gradient buffer, then (256-byte aligned)
-        # the parameter buffer.
-        half = max(128, (max(P, self.offsets[-1]) + 127) // 128 * 128)
-        self._shared = torch.zeros(2 * half, dtype=torch.bfloat16, device=device)
+        # the full parameter buffer (stages 1, 2) or this rank's parameter
+        # shard (stage 3).  The gradient part has the same size on every
+        # rank, so the second part starts at the same offset everywhere.
+        round128 = lambda x: max(128, (x + 127) // 128 * 128)
+        half = round128(max(P, self.offsets[-1]))
+        second = round128(self.plan.owned_numel) if stage == 3 else half
+        self._shared = torch.zeros(half + second, dtype=torch.bfloat16, device=device)
         self.grad_buffer = self._shared[:half]
-        self.param_buffer = self._shared[half:]
         everyone = [None] * self.world_size
         dist.all_gather_object(everyone, zr_ipc_export(self._shared), group=group)
         self._opened = []
-        grad_bases, param_bases = [], []
+        grad_bases, second_bases = [], []
         for w, handle in enumerate(everyone):
             base = self._shared.data_ptr() if w == self.rank else zr_ipc_open(handle)
             if w != self.rank:
                 self._opened.append(base)
             grad_bases.append(base)
-            param_bases.append(base + 2 * half)
+            second_bases.append(base + 2 * half)
         start = 2 * self.offsets[self.rank]                 # bytes: bf16 elements
         self.grad_ptrs = [b + start for b in grad_bases]
-        zr_plan_set_gather_targets(self.plan.handle, param_bases)
+        if stage == 3:
+            self.param_shard = self._shared[half:half + self.plan.owned_numel]
+            self.shard_ptrs = second_bases
+            self.plan.set_param_layout(ZR_PARAMS_OWNED)
+        else:
+            self.param_buffer = self._shared[half:]
+            zr_plan_set_gather_targets(self.plan.handle, second_bases)
         self._segments = self.plan.segments()
         dist.barrier(group)
 
@@ -116,9 +132,20 @@ class PeerZero:
         sync_point(self.dist, self.group, "gradients ready", step)   # ... and every other replica's
         if self.plan.max_grad_norm > 0:
             self._exchange_sumsq()
-        zr_step(self.plan.handle, self.grad_ptrs, master, m, v, None, step)
+        out = self.param_shard if self.stage == 3 else None
+        zr_step(self.plan.handle, self.grad_ptrs, master, m, v, out, step)
         torch.cuda.current_stream().synchronize()
-        sync_point(self.dist, self.group, "parameters gathered", step)   # every slice is in every buffer
+        sync_point(self.dist, self.group, "parameters written", step)   # every slice / shard is written
+
+    def gather(self, first_tensor, n_tensors, dst, stream=None, max_ctas=0):
+        """Stage 3: tensors [first_tensor, first_tensor + n_tensors) whole,
+        in the global layout, into dst (bf16, on this GPU), read from every
+        rank's shard through the peer mappings.  Valid after a step (whose
+        last phase boundary every rank has passed); asynchronous on
+        `stream`, so it can run a layer ahead of use (prefetch)."""
+        if self.stage != 3:
+            raise ValueError("gather is the stage-3 parameter all-gather")
+        zr_gather_params(self.plan.handle, first_tensor, n_tensors, self.shard_ptrs, dst, stream, max_ctas)
 
     def close(self):
         if self._opened:

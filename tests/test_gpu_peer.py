@@ -102,3 +102,84 @@ def test_two_processes_share_one_gpu(shapes, mode, max_norm):
         if max_norm == 0:
             assert same_state and same_out, r
     assert all(p.exitcode == 0 for p in procs)
+
+
+def _rank_main_stage3(rank, world, port, shapes, mode, q):
+    """Stage 3 over IPC: each rank writes only its bf16 shard; after the
+    step every rank gathers whole tensors from both shards (one through a
+    peer mapping)."""
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    import torch
+    import torch.distributed as dist
+    import oracle
+    import synth
+    from sharded_optimizer_step_zr_b200.peer import PeerZero
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=90))
+    try:
+        hp = (3e-4, 0.9, 0.999, 1e-8, 0.1, 0.0)
+        pz = PeerZero(dist.group.WORLD, shapes, mode, 4096, *hp, stage=3)
+        segs = pz.plan.segments()
+        N, P = pz.plan.total_numel, pz.plan.padded_numel
+        runs_of = [synth.rank_runs(segs, r) for r in range(world)]
+        n = pz.plan.owned_numel
+        master = torch.empty(max(n, 8), dtype=torch.float32, device="cuda:0")
+        synth.fill_owned_master(master, runs_of[rank], 6, n_valid=N)
+        m, v = torch.zeros_like(master), torch.zeros_like(master)
+        idx_all = torch.arange(P, dtype=torch.int64)
+        o_master = synth.master_f32(6, idx_all, n_valid=N).numpy().copy()
+        o_m, o_v = np.zeros(P, np.float32), np.zeros(P, np.float32)
+        o_out = np.zeros(P, np.uint16)
+        for t in (1, 2):
+            for r in range(world):
+                a, b = pz.offsets[r], pz.offsets[r + 1]
+                synth.fill_owned_grad(pz.grad_buffer[a:b], runs_of[r], 6, t, rank, 1e-2, 0.01, n_valid=N)
+            pz.step(master, m, v, t)
+            reps = [synth.grad_bf16(6, t, w, idx_all, 1e-2, 0.01, n_valid=N).view(torch.int16).numpy()
+                    .view(np.uint16).copy() for w in range(world)]
+            oracle.ddp_step(reps, o_master, o_m, o_v, o_out, hp, t)
+        full = torch.full((max(N, 8),), -1, dtype=torch.int16, device="cuda:0")
+        pz.gather(0, len(shapes), full.view(torch.bfloat16))
+        numels = [int(np.prod(s)) for s in shapes]
+        goff = np.concatenate([[0], np.cumsum(numels)])
+        one = torch.zeros(max(numels[2], 8), dtype=torch.bfloat16, device="cuda:0")
+        pz.gather(2, 1, one, max_ctas=4)
+        torch.cuda.synchronize()
+        got = full[:N].cpu().numpy().view(np.uint16)
+        got_one = one[:numels[2]].cpu().view(torch.int16).numpy().view(np.uint16)
+        gi = oracle.Plan(shapes, world, mode, 4096).owned_global_index(rank)
+        shard = pz.param_shard.cpu().view(torch.int16).numpy().view(np.uint16)
+        q.put((rank, bool(np.array_equal(got, o_out[:N])),
+               bool(np.array_equal(got_one, o_out[goff[2]:goff[3]])),
+               bool(np.array_equal(shard, o_out[gi]))))
+        dist.barrier()                       # nobody unmaps a shard another rank still reads
+        pz.close()
+    except Exception as e:
+        q.put((rank, "error", repr(e), None))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("shapes, mode", [
+    ([(300, 7), (1001,), (64, 64), (4099,)], 0),
+    ([(300, 7), (1001,), (64, 64), (4099,), (17,)], 1),
+])
+def test_two_processes_stage3_gather(shapes, mode):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _port()
+    procs = [ctx.Process(target=_rank_main_stage3, args=(r, 2, port, shapes, mode, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=240) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=60)
+    for r in results:
+        assert r[1] != "error", r
+        assert r[1] and r[2] and r[3], r
+    assert all(p.exitcode == 0 for p in procs)
