@@ -398,28 +398,33 @@ zr_status zr_gather_params(const zr_plan* plan, int32_t first_tensor, int32_t n_
  * it follows from this library's caller-owned workspace.
  *
  * zr_plan_verify enqueues on `stream` one kernel that tests every tile of
- * both device tables against the invariants the planner guarantees (length
- * 1..2048, owned and global ranges inside the rank's owned count and
- * padded_numel, 16-byte vector flags only where the alignment holds, bucket
- * and index in range, each bucket-order tile at its own index) and compare
- * an order-independent 64-bit hash of each table with the one taken on the
- * host when zr_plan_set_workspace uploaded it.  If anything fails, now or at
- * an earlier check, both tables are overwritten with empty tiles, so the
- * steps queued after it update nothing and write nothing (their results
- * are then missing, not wrong); zr_plan_set_workspace re-uploads the tables
- * and clears the status.  Nothing waits on anything; a check is one small
+ * both device tile tables against the invariants the planner guarantees
+ * (length 1..2048, owned and output ranges inside the rank's owned count
+ * and the output buffer, 16-byte vector flags only where the alignment
+ * holds, bucket and index in range, each bucket-order tile at its own
+ * index) and every entry of the ZeRO-3 gather piece table (length
+ * 1..16384, owner and tensor in range, destination inside total_numel),
+ * and compares an order-independent 64-bit hash of each table with the one
+ * taken on the host when it was uploaded.  If anything fails, now or at an
+ * earlier check, all three tables are overwritten with empty entries, so
+ * the steps and gathers queued after it update and write nothing (their
+ * results are then missing, not wrong); zr_plan_set_workspace re-uploads
+ * the tables and clears the status.  Nothing waits on anything; a check is one small
  * launch reading 64 bytes per tile.
- * zr_plan_set_checked(plan, 1) makes every call that launches the tile
- * kernels (zr_step, zr_step_device_count, zr_step_bucket, zr_step_finish,
- * zr_step_host, zr_grad_sumsq, zr_debug_reduce) run that check first on its
- * stream; 0 (the default) turns it off.  zr_step_no_alloc uploads its own
+ * zr_plan_set_checked(plan, 1) makes every call that launches kernels
+ * reading those tables (zr_step, zr_step_device_count, zr_step_bucket,
+ * zr_step_finish, zr_step_host, zr_grad_sumsq, zr_debug_reduce,
+ * zr_gather_params) run that check first on its stream; 0 (the default)
+ * turns it off.  zr_step_no_alloc uploads its own
  * table on every call and is not affected.
  * zr_plan_check_result synchronises `stream` and reads the status:
- * bad_tiles = tiles that failed an invariant (both tables, counted at every
+ * bad_tiles = entries that failed an invariant (all tables, counted at every
  * check since the workspace was bound), first_bad = the smallest failing
- * position (i for the bucket-order table, n_tiles + i for the owned-order
- * one) or -1, hash_mismatch = bit 0 for the bucket-order table, bit 1 for
- * the owned-order one, tables_emptied = 1 once a failure has emptied them.
+ * position (i for the bucket-order tile table, n_tiles + i for the
+ * owned-order one, 2 n_tiles + i for the gather pieces) or -1,
+ * hash_mismatch = bit 0 for the bucket-order table, bit 1 for the
+ * owned-order one, bit 2 for the gather pieces, tables_emptied = 1 once a
+ * failure has emptied them.
  * Errors: ZR_ERR_INVALID_ARG, ZR_ERR_NO_WORKSPACE, ZR_ERR_CUDA. */
 typedef struct {
     uint64_t bad_tiles;

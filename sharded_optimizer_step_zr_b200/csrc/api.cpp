@@ -58,21 +58,33 @@ zr_status check_device(const zr_plan* p) {
 // Checked mode: verify the device tile tables before a launch that reads
 // them (one kernel on the caller's stream).
 zr_status verify_tables(const zr_plan* p, zr_stream_t stream) {
-    if (p->tiles.empty()) return ZR_OK;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return cuda_status(static_cast<cudaError_t>(zr::launch_verify_tables(
-        p->d_tiles, p->d_tiles_by_owned, static_cast<int32_t>(p->tiles.size()), p->owned_numel(), p->padded_numel,
-        p->n_buckets, p->hash_tiles, p->hash_tiles_by_owned, p->d_check, s)));
+    zr::VerifyArgs a{};
+    a.tiles = p->d_tiles;
+    a.tiles_by_owned = p->d_tiles_by_owned;
+    a.n_tiles = static_cast<int32_t>(p->tiles.size());
+    a.n_buckets = p->n_buckets;
+    a.n_owned = p->owned_numel();
+    a.n_out = p->param_layout == ZR_PARAMS_OWNED ? p->owned_numel() : p->padded_numel;
+    a.pieces = p->d_gather_pieces;
+    a.n_pieces = static_cast<int32_t>(p->gather_pieces.size());
+    a.world_size = p->world_size;
+    a.total_numel = p->total_numel;
+    a.n_tensors = p->n_tensors;
+    a.hash_tiles = p->hash_tiles;
+    a.hash_by_owned = p->hash_tiles_by_owned;
+    a.hash_pieces = p->hash_gather_pieces;
+    a.check = p->d_check;
+    return cuda_status(static_cast<cudaError_t>(zr::launch_verify_tables(a, stream)));
 }
 
 zr_status verify_if_checked(const zr_plan* p, zr_stream_t stream) {
     return p->checked ? verify_tables(p, stream) : ZR_OK;
 }
 
-// The tile tables to the workspace on `stream`, with checked mode's
-// reference hashes and fresh status words (no failure, smallest failing
-// position all ones).
-zr_status upload_tiles(zr_plan* p, zr_stream_t stream) {
+// The tile tables and the gather piece table to the workspace on `stream`,
+// with checked mode's reference hashes and fresh status words (no failure,
+// smallest failing position all ones).
+zr_status upload_tables(zr_plan* p, zr_stream_t stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (!p->tiles.empty()) {
         const size_t bytes_tiles = sizeof(zr::Tile) * p->tiles.size();
@@ -81,8 +93,13 @@ zr_status upload_tiles(zr_plan* p, zr_stream_t stream) {
                 cudaSuccess)
             return ZR_ERR_CUDA;
     }
+    if (!p->gather_pieces.empty() &&
+        cudaMemcpyAsync(p->d_gather_pieces, p->gather_pieces.data(), sizeof(zr::GatherPiece) * p->gather_pieces.size(),
+                        cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return ZR_ERR_CUDA;
     p->hash_tiles = zr::table_hash(p->tiles);
     p->hash_tiles_by_owned = zr::table_hash(p->tiles_by_owned);
+    p->hash_gather_pieces = zr::table_hash(p->gather_pieces);
     if (cudaMemsetAsync(p->d_check, 0, sizeof(uint64_t) * zr::kCheckWords, s) != cudaSuccess ||
         cudaMemsetAsync(p->d_check + 1, 0xFF, sizeof(uint64_t), s) != cudaSuccess)
         return ZR_ERR_CUDA;
@@ -231,12 +248,7 @@ zr_status zr_plan_set_workspace(zr_plan* p, void* d_ws, uint64_t bytes, zr_strea
     p->n_gather_targets = 0;
     p->d_g_scratch = p->clip_uses_scratch() ? reinterpret_cast<float*>(base + L.g_scratch) : nullptr;
     p->d_gather_pieces = reinterpret_cast<zr::GatherPiece*>(base + L.gather_pieces);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (!p->gather_pieces.empty() &&
-        cudaMemcpyAsync(p->d_gather_pieces, p->gather_pieces.data(), sizeof(zr::GatherPiece) * p->gather_pieces.size(),
-                        cudaMemcpyHostToDevice, s) != cudaSuccess)
-        return ZR_ERR_CUDA;
-    return upload_tiles(p, stream);
+    return upload_tables(p, stream);
 }
 
 zr_status zr_plan_set_param_layout(zr_plan* p, int32_t layout, zr_stream_t stream) {
@@ -253,7 +265,7 @@ zr_status zr_plan_set_param_layout(zr_plan* p, int32_t layout, zr_stream_t strea
     } catch (...) {
         return ZR_ERR_INVALID_ARG;
     }
-    return p->d_workspace ? upload_tiles(p, stream) : ZR_OK;
+    return p->d_workspace ? upload_tables(p, stream) : ZR_OK;
 }
 
 zr_status zr_gather_params(const zr_plan* p, int32_t first_tensor, int32_t n_tensors, const void* const* shard_ptrs,
@@ -265,6 +277,10 @@ zr_status zr_gather_params(const zr_plan* p, int32_t first_tensor, int32_t n_ten
     if (dst_st != ZR_OK) return dst_st;
     const int32_t a = p->tensor_first_piece[first_tensor], b = p->tensor_first_piece[first_tensor + n_tensors];
     if (a == b) return ZR_OK;   // only zero-element tensors
+    {
+        const zr_status cs = verify_if_checked(p, stream);
+        if (cs != ZR_OK) return cs;
+    }
     if (!dst) return ZR_ERR_INVALID_ARG;
     if (!aligned16(dst)) return ZR_ERR_ALIGNMENT;
     for (int32_t w = 0; w < p->world_size; ++w) {

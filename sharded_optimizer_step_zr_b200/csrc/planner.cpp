@@ -316,15 +316,20 @@ WorkspaceLayout workspace_layout(const zr_plan& p) {
     return L;
 }
 
-uint64_t table_hash(const std::vector<Tile>& tiles) {
+template <typename Entry>
+static uint64_t hash_entries(const std::vector<Entry>& table) {
+    static_assert(sizeof(Entry) == sizeof(uint64_t) * kTileWords, "4-word entries");
     uint64_t h = 0;
-    for (size_t i = 0; i < tiles.size(); ++i) {
+    for (size_t i = 0; i < table.size(); ++i) {
         uint64_t w[kTileWords];
-        std::memcpy(w, &tiles[i], sizeof(Tile));
+        std::memcpy(w, &table[i], sizeof(Entry));
         for (int j = 0; j < kTileWords; ++j) h += tile_word_hash(w[j], kTileWords * i + j);
     }
     return h;
 }
+
+uint64_t table_hash(const std::vector<Tile>& tiles) { return hash_entries(tiles); }
+uint64_t table_hash(const std::vector<GatherPiece>& pieces) { return hash_entries(pieces); }
 
 AdamScalars adam_scalars(const zr_adamw& hp, int64_t step) {
     const double b1 = hp.beta1, b2 = hp.beta2, lr = hp.lr, t = static_cast<double>(step);

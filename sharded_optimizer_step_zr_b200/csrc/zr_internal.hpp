@@ -57,8 +57,9 @@ constexpr int kTileWords = static_cast<int>(sizeof(Tile) / sizeof(uint64_t));   
 // table i, owned-order table n_tiles + i; all ones when none), [2] hash
 // mismatch bits (1: bucket-order table, 2: owned-order table), [3], [4] the
 // two tables' hash sums while a check runs, [5] the count of its finished
-// blocks (words 3-5 are 0 between checks).
-constexpr int kCheckWords = 6;
+// blocks, [6] the gather pieces' hash sum (words 3-6 are 0 between checks;
+// mismatch bit 4: the gather piece table).
+constexpr int kCheckWords = 7;
 
 // A piece of the ZeRO-3 parameter gather: `len` consecutive elements of one
 // tensor that one rank owns, copied from that rank's bf16 shard (owned
@@ -127,14 +128,27 @@ int launch_clip_combine(const double* tile_partials, int32_t n_tiles, double* pa
 int launch_gather(const GatherPiece* pieces, int32_t first, int32_t n, int32_t max_ctas, int32_t world_size,
                   const void* const* shard_ptrs, uint16_t* dst, int64_t dst_base, void* stream);
 
-// Checked mode: verify both device tile tables against the tile invariants
-// and the hashes taken on the host at upload, then, if anything failed (now
-// or before), overwrite both tables with empty tiles.  One launch; `check`
-// holds kCheckWords words, zeroed (word 1 all ones) when the workspace is
-// bound.
-int launch_verify_tables(Tile* tiles, Tile* tiles_by_owned, int32_t n_tiles, int64_t n_owned, int64_t n_out,
-                         int32_t n_buckets, uint64_t hash_tiles, uint64_t hash_by_owned, uint64_t* check,
-                         void* stream);
+// Checked mode: verify both device tile tables and the gather piece table
+// against their invariants and the hashes taken on the host at upload,
+// then, if anything failed (now or before), overwrite all three with empty
+// entries.  One launch; `check` holds kCheckWords words, zeroed (word 1 all
+// ones) when the workspace is bound.
+struct VerifyArgs {
+    Tile* tiles;
+    Tile* tiles_by_owned;
+    int32_t n_tiles;
+    int32_t n_buckets;
+    int64_t n_owned;       // this rank's owned elements
+    int64_t n_out;         // elements of the buffer the step writes
+    GatherPiece* pieces;
+    int32_t n_pieces;
+    int32_t world_size;
+    int64_t total_numel;
+    int32_t n_tensors;
+    uint64_t hash_tiles, hash_by_owned, hash_pieces;
+    uint64_t* check;
+};
+int launch_verify_tables(const VerifyArgs& args, void* stream);
 
 }  // namespace zr
 
@@ -182,8 +196,9 @@ struct zr_plan {
     std::vector<int32_t> tensor_first_piece;        // n_tensors + 1 entries
     zr::GatherPiece* d_gather_pieces = nullptr;     // workspace copy
     bool checked = false;                  // verify the tables before every launch
-    uint64_t hash_tiles = 0;               // tile_word_hash sums of the two host tables
+    uint64_t hash_tiles = 0;               // tile_word_hash sums of the host tables
     uint64_t hash_tiles_by_owned = 0;
+    uint64_t hash_gather_pieces = 0;
 
     // zr_step_host's copy streams and events, created on its first call
     // (host-side resources, not part of the plan's observable state).
@@ -216,5 +231,6 @@ WorkspaceLayout workspace_layout(const zr_plan& p);
 // bf16 shard in owned order.
 void build_tiles_for_layout(zr_plan& p);
 uint64_t table_hash(const std::vector<Tile>& tiles);
+uint64_t table_hash(const std::vector<GatherPiece>& pieces);
 AdamScalars adam_scalars(const zr_adamw& hp, int64_t step);
 }  // namespace zr

@@ -1,11 +1,13 @@
 """Checked mode on the GPU: a clean plan verifies clean and steps bit for bit
-like an unchecked one; a corrupted device tile table is found (by an
-invariant or by its hash) and emptied before a step can use it.
+like an unchecked one; a corrupted device tile table or gather piece table
+is found (by an invariant or by its hash) and emptied before a step or a
+gather can use it.
 
-No test here runs a step on a table that could send it out of bounds: the
-out-of-range corruption is only verified (then the tables are re-uploaded),
-and the corruption that is stepped under checked mode keeps every tile in
-bounds (two tiles of equal length swap their owned offsets)."""
+No test here runs a step or a gather on a table that could send it out of
+bounds: out-of-range corruptions are only verified (then the tables are
+re-uploaded), and the corruptions run under checked mode keep every entry
+in bounds (two tiles of equal length swap their owned offsets; a piece
+reads an earlier part of the same shard)."""
 import numpy as np
 import pytest
 import torch
@@ -130,3 +132,70 @@ def test_in_bounds_swap_caught_by_the_hash_before_the_step():
     for a, b in zip(g.state(), before):
         assert np.array_equal(bits32(a), bits32(b))
     assert bool(torch.all(out == sentinel))
+
+
+def _layout_no_clip(n_tiles, n_pieces, W):
+    """Byte offsets of the workspace regions of a plan without clipping
+    (each region 256-byte aligned, in this order): tile table, owned-order
+    tile table, clip partials (empty), clip coefficient, own sum of squares,
+    gather targets, device scalars, checked-mode status, gather pieces."""
+    up = lambda x: (x + 255) // 256 * 256
+    off = {"tiles": 0}
+    off["by_owned"] = up(32 * max(1, n_tiles))
+    partials = up(off["by_owned"] + 32 * max(1, n_tiles))
+    clip_coef = partials
+    own = up(clip_coef + 4)
+    targets = up(own + 8)
+    scalars = up(targets + 8 * W)
+    check = up(scalars + 32)
+    off["pieces"] = up(check + 8 * 7)
+    off["total"] = up(off["pieces"] + 32 * max(1, n_pieces))
+    return off
+
+
+PIECE = np.dtype([("src", "<i8"), ("dst", "<i8"), ("len", "<i4"), ("owner", "<i4"), ("tensor", "<i4"),
+                  ("reserved", "<i4")])
+
+
+def test_gather_pieces_checked():
+    """The gather piece table under checked mode: an out-of-range piece is
+    found and the table emptied (only verified, never gathered from); an
+    in-bounds change is caught by the hash and the checked gather writes
+    nothing; a re-upload restores a clean gather."""
+    shapes = [(2048 * 10,)]
+    g = GpuRank(shapes, 1, 0, 0, 1 << 30, HP, seed=9)
+    off = _layout_no_clip(10, 2, 1)
+    assert g.plan.workspace_bytes == off["total"]
+    ws = g.plan.workspace
+    pieces = ws[off["pieces"]:off["pieces"] + 64].cpu().numpy().view(PIECE).copy()
+    assert list(pieces["len"]) == [16384, 4096] and list(pieces["src"]) == [0, 16384]
+    shard = torch.randn(2048 * 10, device=DEV).to(torch.bfloat16)
+    g.plan.set_checked(True)
+    dst = torch.zeros(2048 * 10, dtype=torch.bfloat16, device=DEV)
+    g.plan.gather_params(0, 1, [shard], dst)
+    torch.cuda.synchronize()
+    assert torch.equal(dst.view(torch.int16), shard.view(torch.int16)) and g.plan.check_result() == CLEAN
+    # out of range: verified only
+    bad = pieces.copy()
+    bad["len"][1] = 40000
+    ws[off["pieces"]:off["pieces"] + 64].copy_(torch.from_numpy(bad.view(np.uint8)).to(DEV))
+    g.plan.verify()
+    assert g.plan.check_result() == {"bad_tiles": 1, "first_bad": 2 * 10 + 1, "hash_mismatch": 4,
+                                     "tables_emptied": 1}
+    emptied = ws[off["pieces"]:off["pieces"] + 64].cpu().numpy().view(PIECE)
+    assert np.all(emptied["len"] == 0)
+    rebind(g.plan)
+    # in bounds (piece 1 now reads the shard's first 4096 elements): the hash
+    moved = pieces.copy()
+    moved["src"][1] = 0
+    ws[off["pieces"]:off["pieces"] + 64].copy_(torch.from_numpy(moved.view(np.uint8)).to(DEV))
+    sentinel = torch.full((2048 * 10,), -16447, dtype=torch.int16, device=DEV)
+    g.plan.gather_params(0, 1, [shard], sentinel.view(torch.bfloat16))
+    torch.cuda.synchronize()
+    assert g.plan.check_result() == {"bad_tiles": 0, "first_bad": -1, "hash_mismatch": 4, "tables_emptied": 1}
+    assert bool(torch.all(sentinel == -16447))
+    rebind(g.plan)
+    dst.zero_()
+    g.plan.gather_params(0, 1, [shard], dst)
+    torch.cuda.synchronize()
+    assert torch.equal(dst.view(torch.int16), shard.view(torch.int16)) and g.plan.check_result() == CLEAN
