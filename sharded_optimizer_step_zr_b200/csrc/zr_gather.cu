@@ -26,7 +26,7 @@ struct ShardPtrs {
 };
 
 constexpr int kGatherThreads = 256;
-constexpr int kGatherUnroll = 4;   // 16-byte vectors in flight per thread
+constexpr int kGatherUnroll = 8;   // 16-byte vectors in flight per thread (4: 0.97, 16: 0.96 of the copy peak)
 
 // One piece: source and destination share their offset modulo 16 bytes --
 // a scalar head brings both to a 16-byte boundary, then 16-byte vectors
