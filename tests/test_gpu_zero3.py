@@ -147,3 +147,43 @@ def test_owned_layout_through_buckets_and_host_copies():
     for o in outs[1:]:
         assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
     assert torch.equal(host_out.view(torch.int16), outs[0].cpu().view(torch.int16))
+
+
+@pytest.mark.parametrize("seed", range(30))
+def test_gather_random_sets(seed):
+    """Random tensor sets (zero-element and odd sizes included), W 1..70,
+    both partitions, random tensor ranges and grid caps: the gather equals
+    the shards placed at their global positions by the oracle's owned ->
+    global map, and writes nothing outside its range."""
+    from sharded_optimizer_step_zr_b200.plan import ZrPlan
+    rng = np.random.default_rng(seed)
+    shapes = []
+    for _ in range(int(rng.integers(1, 12))):
+        k = rng.random()
+        shapes.append(() if k < 0.1 else (0,) if k < 0.2 else
+                      (int(rng.integers(1, 40000)),) if k < 0.6 else tuple(int(x) for x in rng.integers(1, 200, 2)))
+    W = int(rng.choice([1, 2, 3, 5, 8, 13, 64, 70]))
+    mode = int(rng.integers(0, 2))
+    oplan = oracle.Plan(shapes, W, mode, 1 << 20)
+    plan = ZrPlan(shapes, W, 0, mode, 1 << 20, *HP, device=DEV)
+    owned = [int(x) for x in oplan.owned_numel]
+    shards = [torch.randint(-32768, 32767, (max(n, 8),), dtype=torch.int16, device=DEV) for n in owned]
+    placed = np.zeros(max(oplan.padded_numel, 8), np.uint16)
+    for r in range(W):
+        idx = oplan.owned_global_index(r)
+        placed[idx] = shards[r][: idx.size].cpu().numpy().view(np.uint16)
+    numels = [int(np.prod(s)) for s in shapes]
+    goff = np.concatenate([[0], np.cumsum(numels)])
+    for _ in range(4):
+        first = int(rng.integers(0, len(shapes)))
+        count = int(rng.integers(0, len(shapes) - first + 1))
+        cap = int(rng.choice([0, 0, 1, 7, 64]))
+        lo, hi = int(goff[first]), int(goff[first + count])
+        dst = torch.full((hi - lo + 16,), -1, dtype=torch.int16, device=DEV)
+        plan.gather_params(first, count, [s.view(torch.bfloat16) for s in shards], dst.view(torch.bfloat16),
+                           max_ctas=cap)
+        torch.cuda.synchronize()
+        got = dst.cpu().numpy().view(np.uint16)
+        assert np.array_equal(got[: hi - lo], placed[lo:hi]), (seed, first, count, cap)
+        assert np.all(got[hi - lo:] == 0xFFFF)
+    plan.close()
