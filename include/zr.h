@@ -148,6 +148,16 @@ zr_status zr_plan_workspace_bytes(const zr_plan* plan, uint64_t* bytes);
 zr_status zr_plan_set_workspace(zr_plan* plan, void* d_workspace, uint64_t bytes,
                                 zr_stream_t stream);
 
+/* New AdamW hyperparameters for the calls that follow (a learning-rate
+ * schedule changes lr every step; the pages' lr of 3e-4 is one constant
+ * point of it).  Host-side: every step call computes its scalars from the
+ * plan's current values, except that zr_step_device_count passes them by
+ * value to its scalars kernel, so a CUDA graph that captured it keeps the
+ * values current at capture.  Turning clipping on or off (max_grad_norm
+ * crossing 0) changes what the workspace holds: ZR_ERR_UNSUPPORTED, make a
+ * new plan.  Errors: ZR_ERR_INVALID_ARG (NULL), ZR_ERR_UNSUPPORTED. */
+zr_status zr_plan_set_adamw(zr_plan* plan, const zr_adamw* hp);
+
 /* Clipping only.  d_partials: device array of world_size doubles, entry w =
  * rank w's sum of squares S_w of its averaged owned gradient.  zr_step
  * writes this rank's entry itself; the other entries must hold the other

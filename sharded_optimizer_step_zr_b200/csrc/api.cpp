@@ -325,6 +325,14 @@ zr_status zr_plan_check_result(const zr_plan* p, zr_check_result* out, zr_stream
     return ZR_OK;
 }
 
+zr_status zr_plan_set_adamw(zr_plan* p, const zr_adamw* hp) {
+    if (!p || !hp) return ZR_ERR_INVALID_ARG;
+    // Clipping on or off changes what the workspace must hold.
+    if ((hp->max_grad_norm > 0.0f) != p->clip_enabled()) return ZR_ERR_UNSUPPORTED;
+    p->hp = *hp;
+    return ZR_OK;
+}
+
 zr_status zr_plan_set_sumsq_partials(zr_plan* p, double* d_partials) {
     if (!p || !d_partials) return ZR_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(d_partials) & 7u) != 0) return ZR_ERR_ALIGNMENT;

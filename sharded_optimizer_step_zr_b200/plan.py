@@ -7,7 +7,8 @@ from __future__ import annotations
 
 from . import (ZR_PARAMS_GLOBAL, ZR_PARAMS_OWNED, ZR_PARTITION_FLAT, zr_debug_reduce, zr_gather_params,
                zr_grad_sumsq, zr_plan_check_result, zr_plan_create, zr_plan_destroy, zr_plan_query,
-               zr_plan_segments, zr_plan_set_checked, zr_plan_set_param_layout, zr_plan_set_sumsq_partials,
+               zr_plan_segments, zr_plan_set_adamw, zr_plan_set_checked, zr_plan_set_param_layout,
+               zr_plan_set_sumsq_partials,
                zr_plan_set_workspace, zr_plan_verify, zr_plan_workspace_bytes, zr_step, zr_step_bucket,
                zr_step_finish, zr_step_host)
 
@@ -179,6 +180,11 @@ class ZrPlan:
         specs = [(g, f"grads[{w}]", torch.bfloat16, self.owned_numel, False) for w, g in enumerate(grads)]
         _require_all(specs + [(g_out, "g_out", torch.float32, self.owned_numel, False)], self.device)
         zr_debug_reduce(self.handle, grads, g_out, stream)
+
+    def set_adamw(self, lr=3e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.1, max_grad_norm=0.0):
+        """Hyperparameters for the following steps (e.g. this step's lr)."""
+        zr_plan_set_adamw(self.handle, lr, beta1, beta2, eps, weight_decay, max_grad_norm)
+        self.max_grad_norm = max_grad_norm
 
     def set_checked(self, enable=True):
         zr_plan_set_checked(self.handle, enable)

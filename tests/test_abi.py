@@ -249,3 +249,19 @@ def test_zero3_calls_without_a_device():
         assert zr._lib.zr_gather_params(h, 0, 3, arr, None, 0, None) == zr.ZR_ERR_NO_WORKSPACE
     finally:
         zr.zr_plan_destroy(h)
+
+
+def test_set_adamw_refuses_turning_clipping_on_or_off():
+    h = zr.zr_plan_create([(4096,)], 2, 0, 0, 1 << 20)                     # no clipping
+    hc = zr.zr_plan_create([(4096,)], 2, 0, 0, 1 << 20, max_grad_norm=1.0)
+    try:
+        zr.zr_plan_set_adamw(h, lr=1e-3, weight_decay=0.0)
+        zr.zr_plan_set_adamw(hc, lr=1e-3, max_grad_norm=0.5)
+        for plan, mgn in ((h, 1.0), (hc, 0.0)):
+            with pytest.raises(zr.ZrError) as e:
+                zr.zr_plan_set_adamw(plan, max_grad_norm=mgn)
+            assert e.value.status == zr.ZR_ERR_UNSUPPORTED
+        assert zr._lib.zr_plan_set_adamw(h, None) == zr.ZR_ERR_INVALID_ARG
+    finally:
+        zr.zr_plan_destroy(h)
+        zr.zr_plan_destroy(hc)

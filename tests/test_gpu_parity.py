@@ -187,6 +187,52 @@ def test_thirty_steps_stay_bit_exact():
         assert np.array_equal(u16(out_g)[mine], out_o[mine])
 
 
+@pytest.mark.parametrize("clip", [0.0, 1.0])
+def test_learning_rate_schedule(clip):
+    """zr_plan_set_adamw between steps: a warmup-then-cosine lr over five
+    steps (and, with clipping, a changing max_grad_norm), both ranks of a
+    flat W = 2 partition, against the oracle stepping with the same
+    per-step hyperparameters."""
+    import math
+    shapes = [(4096 * 3 + 5,), (300,)]
+    W = 2
+    oplan = oracle.Plan(shapes, W, 0, 1 << 20)
+    P = oplan.padded_numel
+    ranks = [GpuRank(shapes, W, r, 0, 1 << 20, HP, seed=13, max_grad_norm=clip) for r in range(W)]
+    orcs = [OracleRank(oplan, r, seed=13) for r in range(W)]
+    out_g = torch.zeros(P, dtype=torch.bfloat16, device=DEV)
+    out_o = np.zeros(P, np.uint16)
+    for t in range(1, 6):
+        lr = 1e-3 * min(1.0, t / 2) * 0.5 * (1 + math.cos(math.pi * t / 6))
+        mgn = clip * (1.0 + 0.5 * t) if clip > 0 else 0.0
+        hp = (lr, 0.9, 0.999, 1e-8, 0.1, mgn)
+        S_parts = []
+        for g, o in zip(ranks, orcs):
+            g.fill_grads(t, 1e-2, 0.01)
+            o.make_grads(t, 1e-2, 0.01)
+            S_parts.append(oracle.sumsq(oracle.reduce(o.grads)))
+        c = None
+        if clip > 0:
+            S = 0.0
+            for x in S_parts:
+                S += x
+            c = oracle.clip_coef(S, mgn)
+            for g in ranks:
+                g.plan.partials.copy_(torch.tensor(S_parts, dtype=torch.float64))
+        for g, o in zip(ranks, orcs):
+            g.plan.set_adamw(*hp)
+            g.step(out_g, t)
+            o.step(out_o, hp, t, clip=c)
+        torch.cuda.synchronize()
+        for g, o in zip(ranks, orcs):
+            for got, want in zip(g.state(), (o.master, o.m, o.v)):
+                if clip == 0:
+                    assert np.array_equal(bits32(got), bits32(want)), t
+                else:
+                    assert_state_close(got, want, f"step {t}")
+        assert bf16_ulp_distance(u16(out_g), out_o).max() <= 1
+
+
 def test_max_world_size():
     """W = 512, the ABI's maximum (the pointer array's largest instantiation):
     first, middle and last rank."""
