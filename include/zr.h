@@ -158,6 +158,14 @@ zr_status zr_plan_set_workspace(zr_plan* plan, void* d_workspace, uint64_t bytes
  * new plan.  Errors: ZR_ERR_INVALID_ARG (NULL), ZR_ERR_UNSUPPORTED. */
 zr_status zr_plan_set_adamw(zr_plan* plan, const zr_adamw* hp);
 
+/* A learning rate in device memory for zr_step_device_count: its scalars
+ * kernel reads *d_lr (one fp32, caller-owned, 4-byte aligned) at every
+ * launch instead of the plan's lr, so a captured graph follows a schedule
+ * that the caller's own device work updates between replays.  NULL (the
+ * default) goes back to the plan's lr.  The other hyperparameters stay
+ * those current at capture.  Errors: ZR_ERR_INVALID_ARG, ZR_ERR_ALIGNMENT. */
+zr_status zr_plan_set_device_lr(zr_plan* plan, const float* d_lr);
+
 /* Clipping only.  d_partials: device array of world_size doubles, entry w =
  * rank w's sum of squares S_w of its averaged owned gradient.  zr_step
  * writes this rank's entry itself; the other entries must hold the other

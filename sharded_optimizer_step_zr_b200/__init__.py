@@ -40,7 +40,7 @@ ZR_MAX_WORLD_SIZE = 512
 
 EXPORTED = [
     "zr_plan_create", "zr_plan_query", "zr_plan_segments", "zr_plan_workspace_bytes",
-    "zr_plan_set_workspace", "zr_plan_set_adamw", "zr_plan_set_sumsq_partials", "zr_step", "zr_step_device_count",
+    "zr_plan_set_workspace", "zr_plan_set_adamw", "zr_plan_set_device_lr", "zr_plan_set_sumsq_partials", "zr_step", "zr_step_device_count",
     "zr_step_bucket",
     "zr_step_finish", "zr_step_host",
     "zr_grad_sumsq", "zr_debug_reduce", "zr_step_no_alloc", "zr_state_save", "zr_state_load",
@@ -95,6 +95,7 @@ _lib.zr_state_reshard.argtypes = [_vp, _vp, _i32, ctypes.c_char_p]
 _lib.zr_state_export_params.argtypes = [_vp, _vp, _i32, _i32, ctypes.c_char_p, _vp]
 _lib.zr_plan_set_checked.argtypes = [_vp, _i32]
 _lib.zr_plan_set_adamw.argtypes = [_vp, _P(zr_adamw)]
+_lib.zr_plan_set_device_lr.argtypes = [_vp, _vp]
 _lib.zr_plan_set_param_layout.argtypes = [_vp, _i32, _vp]
 _lib.zr_gather_params.argtypes = [_vp, _i32, _i32, _vp, _vp, _i32, _vp]
 _lib.zr_plan_verify.argtypes = [_vp, _vp]
@@ -301,6 +302,11 @@ def zr_plan_set_adamw(plan: int, lr=3e-4, beta1=0.9, beta2=0.999, eps=1e-8, weig
                       max_grad_norm=0.0) -> None:
     hp = zr_adamw(lr, beta1, beta2, eps, weight_decay, max_grad_norm)
     _check(_lib.zr_plan_set_adamw(plan, ctypes.byref(hp)), "zr_plan_set_adamw")
+
+
+def zr_plan_set_device_lr(plan: int, d_lr) -> None:
+    """d_lr: a one-element fp32 device tensor (or address), or None."""
+    _check(_lib.zr_plan_set_device_lr(plan, _addr(d_lr)), "zr_plan_set_device_lr")
 
 
 ZR_PARAMS_GLOBAL = 0

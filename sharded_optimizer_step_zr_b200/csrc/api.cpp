@@ -333,6 +333,13 @@ zr_status zr_plan_set_adamw(zr_plan* p, const zr_adamw* hp) {
     return ZR_OK;
 }
 
+zr_status zr_plan_set_device_lr(zr_plan* p, const float* d_lr) {
+    if (!p) return ZR_ERR_INVALID_ARG;
+    if (d_lr && (reinterpret_cast<uintptr_t>(d_lr) & 3u) != 0) return ZR_ERR_ALIGNMENT;
+    p->d_lr = d_lr;
+    return ZR_OK;
+}
+
 zr_status zr_plan_set_sumsq_partials(zr_plan* p, double* d_partials) {
     if (!p || !d_partials) return ZR_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(d_partials) & 7u) != 0) return ZR_ERR_ALIGNMENT;
@@ -400,7 +407,7 @@ static zr_status step_impl(const zr_plan* p, const void* const* grad_ptrs, float
         // Nothing to update, but a device step count still advances, so it
         // stays equal on every rank.
         if (d_step)
-            return cuda_status(static_cast<cudaError_t>(zr::launch_device_scalars(d_step, p->hp, p->d_scalars, stream)));
+            return cuda_status(static_cast<cudaError_t>(zr::launch_device_scalars(d_step, p->hp, p->d_lr, p->d_scalars, stream)));
         return ZR_OK;
     }
     zr_status st = check_grads(p, grad_ptrs);
@@ -422,7 +429,7 @@ static zr_status step_impl(const zr_plan* p, const void* const* grad_ptrs, float
     if (d_step) {
         // The count and the scalars live in device memory, so a captured
         // graph of this call replays as the next step each time.
-        if (zr::launch_device_scalars(d_step, p->hp, p->d_scalars, s) != cudaSuccess) return ZR_ERR_CUDA;
+        if (zr::launch_device_scalars(d_step, p->hp, p->d_lr, p->d_scalars, s) != cudaSuccess) return ZR_ERR_CUDA;
         a.dev_scalars = p->d_scalars;
     }
     if (!p->clip_enabled())

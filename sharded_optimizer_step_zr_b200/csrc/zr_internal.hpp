@@ -117,7 +117,7 @@ struct LaunchArgs {
 // pointers.  Return cudaError_t as int.
 int launch_tiles(Pass pass, const LaunchArgs& a, const void* const* grad_ptrs, bool g_from_scratch,
                  bool write_g_scratch, void* stream);
-int launch_device_scalars(int64_t* d_step, const zr_adamw& hp, AdamScalars* out, void* stream);
+int launch_device_scalars(int64_t* d_step, const zr_adamw& hp, const float* d_lr, AdamScalars* out, void* stream);
 int launch_clip_combine(const double* tile_partials, int32_t n_tiles, double* partials_all,
                         int32_t world_size, int32_t rank, float max_norm, float* clip_coef_out,
                         double* sumsq_out, void* stream);
@@ -189,6 +189,7 @@ struct zr_plan {
     double* d_sumsq_partials = nullptr;   // caller-owned, world_size doubles
     uint16_t** d_gather_targets = nullptr; // workspace: world_size parameter buffers
     zr::AdamScalars* d_scalars = nullptr;  // workspace: scalars computed on the device
+    const float* d_lr = nullptr;           // caller-owned learning rate for zr_step_device_count
     int32_t n_gather_targets = 0;          // 0 until zr_plan_set_gather_targets
     uint64_t* d_check = nullptr;           // workspace: checked mode's status words
     int32_t param_layout = ZR_PARAMS_GLOBAL;   // where zr_step writes the bf16 parameters

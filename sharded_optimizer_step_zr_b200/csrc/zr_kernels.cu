@@ -296,26 +296,6 @@ zr_tile_kernel(const GradPtrs<CAP> gp, const LaunchArgs a) {
     }
 }
 
-// One thread: advance the device step count and compute the AdamW scalars
-// for the new step, in fp64 from the fp32 hyperparameters and rounded once
-// to fp32 -- the same expressions as the host computes for zr_step.
-__global__ void zr_device_scalars_kernel(int64_t* d_step, const zr_adamw hp, AdamScalars* out) {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
-    const int64_t step = *d_step + 1;
-    *d_step = step;
-    const double b1 = hp.beta1, b2 = hp.beta2, lr = hp.lr, t = static_cast<double>(step);
-    AdamScalars s;
-    s.beta1 = hp.beta1;
-    s.beta2 = hp.beta2;
-    s.one_minus_beta1 = static_cast<float>(1.0 - b1);
-    s.one_minus_beta2 = static_cast<float>(1.0 - b2);
-    s.step_size = static_cast<float>(lr / (1.0 - pow(b1, t)));
-    s.bc2_sqrt = static_cast<float>(sqrt(1.0 - pow(b2, t)));
-    s.decay = static_cast<float>(1.0 - lr * static_cast<double>(hp.weight_decay));
-    s.eps = hp.eps;
-    *out = s;
-}
-
 // One block: S_r = sum of the per-tile partials in a fixed order, stored as
 // this rank's entry of the partials array (or to sumsq_out alone); then the
 // clip coefficient from all ranks' entries, summed in rank order.
@@ -411,11 +391,6 @@ int launch_tiles(Pass pass, const LaunchArgs& a, const void* const* grad_ptrs, b
                                   : dispatch_update<Pass::kStepClip, false>(a, grad_ptrs, s);
     }
     return cudaErrorInvalidValue;
-}
-
-int launch_device_scalars(int64_t* d_step, const zr_adamw& hp, AdamScalars* out, void* stream_v) {
-    zr_device_scalars_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream_v)>>>(d_step, hp, out);
-    return cudaGetLastError();
 }
 
 int launch_clip_combine(const double* tile_partials, int32_t n_tiles, double* partials_all,

@@ -265,3 +265,13 @@ def test_set_adamw_refuses_turning_clipping_on_or_off():
     finally:
         zr.zr_plan_destroy(h)
         zr.zr_plan_destroy(hc)
+
+
+def test_set_device_lr_arguments():
+    h = zr.zr_plan_create([(4096,)], 2, 0, 0, 1 << 20)
+    try:
+        assert zr._lib.zr_plan_set_device_lr(None, None) == zr.ZR_ERR_INVALID_ARG
+        assert zr._lib.zr_plan_set_device_lr(h, 2) == zr.ZR_ERR_ALIGNMENT
+        zr.zr_plan_set_device_lr(h, None)
+    finally:
+        zr.zr_plan_destroy(h)
