@@ -119,3 +119,14 @@ def test_recorded_traffic_is_close_to_the_algorithmic_bytes():
         alg = plan.owned_numel * bench.bytes_per_owned_param(wl.world_size, clip)
         plan.close()
         assert 0.9 * alg <= t <= 1.02 * alg, (name, t, alg)
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    """Under torchrun (N > 1) only rank 0 runs and prints the reference
+    arm; the other ranks exit 0 without work or output."""
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                          "--steps", "2", "--warmup", "1"], capture_output=True, text=True, timeout=300,
+                         cwd=ROOT, env=env)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert out.stdout.strip() == ""
