@@ -394,7 +394,7 @@ zr_status zr_state_export_params(const zr_plan* plan, const char* const* src_pat
  * consecutive, row-major; 16-byte aligned), gathered from shard_ptrs[w] =
  * rank w's bf16 shard in owned order (W device pointers, local or mapped
  * from other GPUs, 16-byte aligned; NULL allowed for a rank that owns
- * nothing).
+ * nothing).  dst must not overlap any shard.
  * One kernel on `stream`: pieces of at most 16384 elements of one tensor
  * and one owner, plain 16-byte loads and stores where source and
  * destination share their alignment, 2-byte ones otherwise, with the
