@@ -1,8 +1,11 @@
 // C ABI of the fused sharded optimizer step (declared in include/zr.h).
 //
 // This layer validates arguments, holds the host-side plan, binds the
-// caller's device workspace and enqueues the kernels; it never allocates
-// device memory and never synchronises.
+// caller's device workspace and enqueues the kernels.  It never allocates
+// device memory, and the step, gather and check calls never synchronise;
+// zr_plan_set_gather_targets and zr_plan_check_result synchronise their
+// stream (documented in the header), and zr_step_host creates its two copy
+// streams and events on first use.
 #include <cuda_runtime.h>
 
 #include <algorithm>
