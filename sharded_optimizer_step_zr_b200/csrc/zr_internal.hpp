@@ -52,13 +52,13 @@ ZR_HOST_DEVICE inline uint64_t tile_word_hash(uint64_t w, uint64_t k) {
 }
 constexpr int kTileWords = static_cast<int>(sizeof(Tile) / sizeof(uint64_t));   // 4
 
-// Checked mode's status words in the workspace: [0] tiles failing a check
-// (both tables, cumulative), [1] the smallest failing position (bucket-order
-// table i, owned-order table n_tiles + i; all ones when none), [2] hash
-// mismatch bits (1: bucket-order table, 2: owned-order table), [3], [4] the
-// two tables' hash sums while a check runs, [5] the count of its finished
-// blocks, [6] the gather pieces' hash sum (words 3-6 are 0 between checks;
-// mismatch bit 4: the gather piece table).
+// Checked mode's status words in the workspace: [0] entries failing a
+// check (all three tables, cumulative), [1] the smallest failing position
+// (bucket-order tile table i, owned-order tile table n_tiles + i, gather
+// pieces 2 n_tiles + i; all ones when none), [2] hash mismatch bits (1:
+// bucket-order tiles, 2: owned-order tiles, 4: gather pieces), [3], [4] the
+// tile tables' hash sums while a check runs, [5] the count of its finished
+// blocks, [6] the gather pieces' hash sum (words 3-6 are 0 between checks).
 constexpr int kCheckWords = 7;
 
 // A piece of the ZeRO-3 parameter gather: `len` consecutive elements of one
