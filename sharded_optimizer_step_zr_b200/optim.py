@@ -1,0 +1,136 @@
+"""ZeroAdamW: the sharded step behind a torch-optimizer-style interface.
+
+    opt = ZeroAdamW(model.parameters(), group=None, lr=3e-4)     # or a process group
+    loss.backward(); opt.step(); opt.zero_grad()
+
+The model's bf16 parameters become views of the full bf16 parameter buffer
+that every rank's step writes (the all-gather), and their .grad tensors
+views of the replica's gradient buffer in the plan's owner-major layout, so
+autograd accumulates straight into it ("DDP -> ZeRO" blog, section 2.1:
+gradients are written into flat buckets as the backward pass produces
+them).  Each rank holds only its owned slice of the fp32 master weights and
+Adam moments (ZeRO stage 1/2).  With one rank the plan's own buffers are
+used; with a process group of several ranks the buffers are shared between
+the processes over CUDA IPC (PeerZero), and the step reads the other
+replicas' gradients and writes every rank's parameters through peer memory.
+
+Only the buffer plumbing lives here: the step itself runs in libzr.so.
+"""
+from __future__ import annotations
+
+from . import ZR_PARTITION_FLAT, ZR_PARTITION_WHOLE_TENSOR
+
+
+class ZeroAdamW:
+    def __init__(self, params, group=None, lr=3e-4, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.1,
+                 max_grad_norm=0.0, partition="flat", bucket_cap_mb=25):
+        import torch
+        self.params = [p for p in params]
+        if not self.params:
+            raise ValueError("no parameters")
+        dev = self.params[0].device
+        for p in self.params:
+            if p.dtype != torch.bfloat16 or p.device != dev:
+                raise ValueError("parameters must be bf16 tensors on one CUDA device")
+        mode = {"flat": ZR_PARTITION_FLAT, "whole": ZR_PARTITION_WHOLE_TENSOR}[partition]
+        shapes = [tuple(p.shape) for p in self.params]
+        self.hp = dict(lr=lr, beta1=betas[0], beta2=betas[1], eps=eps, weight_decay=weight_decay,
+                       max_grad_norm=max_grad_norm)
+        hp = tuple(self.hp.values())
+        cap = int(bucket_cap_mb * (1 << 20))
+        world = 1
+        if group is not None:
+            import torch.distributed as dist
+            world = dist.get_world_size(group)
+        if world > 1:
+            from .peer import PeerZero
+            self.peer = PeerZero(group, shapes, mode, cap, *hp, device=dev)
+            self.plan = self.peer.plan
+            self.grad_buffer = self.peer.grad_buffer
+            self.param_buffer = self.peer.param_buffer
+            self.offsets = self.peer.offsets
+        else:
+            from .plan import ZrPlan
+            self.peer = None
+            self.plan = ZrPlan(shapes, 1, 0, mode, cap, *hp, device=dev)
+            self.offsets = [0, self.plan.padded_numel]
+            self.grad_buffer = torch.zeros(max(self.plan.padded_numel, 8), dtype=torch.bfloat16, device=dev)
+            self.param_buffer = torch.zeros(max(self.plan.padded_numel, 8), dtype=torch.bfloat16, device=dev)
+        segs = self.plan.segments()
+        goff = [0]
+        for p in self.params:
+            goff.append(goff[-1] + p.numel())
+        # parameters: views of the full bf16 buffer (global layout), current values kept
+        with torch.no_grad():
+            for t, p in enumerate(self.params):
+                view = self.param_buffer[goff[t]:goff[t + 1]].view(p.shape)
+                view.copy_(p)
+                p.data = view
+        # gradients: views of the owner-major buffer where a tensor is one run there
+        self._copy_in = []
+        self._bound = []
+        for t, p in enumerate(self.params):
+            pieces = sorted((s["offset_in_tensor"], s["owner"], s["owned_offset"], s["length"])
+                            for s in segs if s["tensor"] == t)
+            starts = [self.offsets[r] + o for _, r, o, _ in pieces]
+            contiguous = all(starts[i] + pieces[i][3] == starts[i + 1] for i in range(len(pieces) - 1))
+            if pieces and contiguous:
+                p.grad = self.grad_buffer[starts[0]:starts[0] + p.numel()].view(p.shape)
+                self._bound.append((p, starts[0]))
+            else:
+                p.grad = torch.zeros_like(p)
+                self._copy_in.append((p, [(off, self.offsets[r] + o, n) for off, r, o, n in pieces]))
+        # this rank's fp32 master weights (from the bf16 parameters), moments at zero
+        rank = self.plan.rank
+        n = self.plan.owned_numel
+        self.master = torch.zeros(max(n, 8), dtype=torch.float32, device=dev)
+        flat = self.param_buffer
+        for owned, glob, length in self.plan.runs():
+            self.master[owned:owned + length] = flat[glob:glob + length].float()
+        self.m = torch.zeros_like(self.master)
+        self.v = torch.zeros_like(self.master)
+        self.rank, self.step_count = rank, 0
+        self._grads = [self.grad_buffer[self.offsets[rank]:]]
+
+    def zero_grad(self, set_to_none=False):
+        """Zeroes the gradient buffer; the .grad views stay bound (set_to_none
+        is ignored: releasing them would detach autograd from the buffer)."""
+        self.grad_buffer.zero_()
+        for p, _ in self._copy_in:
+            p.grad.zero_()
+
+    def set_lr(self, lr):
+        self.hp["lr"] = lr
+        self.plan.set_adamw(*self.hp.values())
+
+    def step(self):
+        """One optimizer step: this rank's slice of the averaged gradient,
+        AdamW on its fp32 state, the bf16 result into every rank's
+        parameters.  With several ranks, every rank calls it together."""
+        flat_grad = self.grad_buffer.view(-1)
+        # autograd accumulates into a bound .grad in place; should anything
+        # have replaced it with a new tensor, copy that in and bind again
+        for p, start in self._bound:
+            view = flat_grad[start:start + p.numel()]
+            if p.grad is None or p.grad.data_ptr() != view.data_ptr():
+                if p.grad is not None:
+                    view.copy_(p.grad.reshape(-1))
+                else:
+                    view.zero_()
+                p.grad = view.view(p.shape)
+        for p, pieces in self._copy_in:
+            g = p.grad.reshape(-1)
+            for off, start, n in pieces:
+                flat_grad[start:start + n].copy_(g[off:off + n])
+        self.step_count += 1
+        if self.peer is not None:
+            self.peer.step(self.master, self.m, self.v, self.step_count)
+        else:
+            self.plan.step(self._grads, self.master, self.m, self.v, self.param_buffer, self.step_count)
+        return None
+
+    def close(self):
+        if self.peer is not None:
+            self.peer.close()
+        else:
+            self.plan.close()

@@ -1,0 +1,62 @@
+"""ZeroAdamW on a small bf16 model: autograd writes into the plan's gradient
+buffer through the .grad views, the step writes the model's parameters
+through the parameter buffer, and three steps equal the oracle's step on
+the same gradients (fp32 state bit for bit, bf16 parameters within 1 ulp)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_harness import DEV, bf16_ulp_distance, bits32
+from sharded_optimizer_step_zr_b200.optim import ZeroAdamW
+
+pytestmark = pytest.mark.gpu
+
+
+def make_model(seed):
+    torch.manual_seed(seed)
+    return torch.nn.Sequential(torch.nn.Linear(64, 128), torch.nn.GELU(), torch.nn.Linear(128, 24),
+                               torch.nn.LayerNorm(24)).to(DEV).to(torch.bfloat16)
+
+
+def flat_u16(tensors):
+    return torch.cat([t.detach().reshape(-1) for t in tensors]).cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("partition, clip", [("flat", 0.0), ("whole", 1.0)])
+def test_zero_adamw_one_rank_matches_the_oracle(partition, clip):
+    model = make_model(5)
+    params = list(model.parameters())
+    hp = (1e-3, 0.9, 0.999, 1e-8, 0.1, clip)
+    init = flat_u16(params)
+    opt = ZeroAdamW(params, lr=hp[0], betas=hp[1:3], eps=hp[3], weight_decay=hp[4], max_grad_norm=clip,
+                    partition=partition, bucket_cap_mb=0.01)
+    assert np.array_equal(flat_u16(params), init)          # rebinding kept the values
+    N = init.size
+    o_master = (init.astype(np.uint32) << 16).view(np.float32)      # bf16 -> fp32 is exact
+    o_m, o_v = np.zeros(N, np.float32), np.zeros(N, np.float32)
+    o_out = np.zeros(N, np.uint16)
+    gen = torch.Generator(device=DEV).manual_seed(11)
+    lo, hi = opt.grad_buffer.data_ptr(), opt.grad_buffer.data_ptr() + 2 * opt.grad_buffer.numel()
+    for t in (1, 2, 3):
+        x = torch.randn(32, 64, device=DEV, generator=gen).to(torch.bfloat16)
+        loss = model(x).float().pow(2).mean()
+        loss.backward()
+        for p in params:                                      # autograd wrote into the buffer
+            assert lo <= p.grad.data_ptr() < hi
+        grads = flat_u16([p.grad for p in params])
+        c = None
+        if clip > 0:
+            g = oracle.reduce([grads])
+            c = oracle.clip_coef(oracle.sumsq(g), clip)
+        oracle.ddp_step([grads], o_master, o_m, o_v, o_out, hp, t, clip=c)
+        opt.step()
+        opt.zero_grad()
+        torch.cuda.synchronize()
+        got = flat_u16(params)
+        assert bf16_ulp_distance(got, o_out).max() <= 1, t
+        if clip == 0:
+            assert np.array_equal(got, o_out), t
+            # one rank: owned order is the global order
+            assert np.array_equal(bits32(opt.master[:N].cpu().numpy()), bits32(o_master))
+    opt.close()

@@ -183,3 +183,70 @@ def test_two_processes_stage3_gather(shapes, mode):
         assert r[1] != "error", r
         assert r[1] and r[2] and r[3], r
     assert all(p.exitcode == 0 for p in procs)
+
+
+def _rank_main_optim(rank, world, port, q):
+    """ZeroAdamW over a two-process group: the same bf16 model on both
+    ranks, different data; after each step both models equal the oracle's
+    unsharded step on the two replicas' gradients."""
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    import torch
+    import torch.distributed as dist
+    import oracle
+    from sharded_optimizer_step_zr_b200.optim import ZeroAdamW
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=90))
+    try:
+        torch.manual_seed(5)
+        model = torch.nn.Sequential(torch.nn.Linear(64, 128), torch.nn.GELU(), torch.nn.Linear(128, 24),
+                                    torch.nn.LayerNorm(24)).to("cuda:0").to(torch.bfloat16)
+        params = list(model.parameters())
+        flat = lambda ts: torch.cat([t.detach().reshape(-1) for t in ts]).cpu().view(torch.int16).numpy() \
+            .view(np.uint16).copy()
+        init = flat(params)
+        hp = (1e-3, 0.9, 0.999, 1e-8, 0.1, 0.0)
+        opt = ZeroAdamW(params, group=dist.group.WORLD, lr=hp[0], weight_decay=hp[4], bucket_cap_mb=0.01)
+        N = init.size
+        o_master = (init.astype(np.uint32) << 16).view(np.float32).copy()
+        o_m, o_v, o_out = np.zeros(N, np.float32), np.zeros(N, np.float32), np.zeros(N, np.uint16)
+        gen = torch.Generator(device="cuda:0").manual_seed(100 + rank)
+        ok = True
+        for t in (1, 2, 3):
+            x = torch.randn(16, 64, device="cuda:0", generator=gen).to(torch.bfloat16)
+            model(x).float().pow(2).mean().backward()
+            torch.cuda.synchronize()
+            mine = flat([p.grad for p in params])
+            reps = [None] * world
+            dist.all_gather_object(reps, mine)
+            oracle.ddp_step(reps, o_master, o_m, o_v, o_out, hp, t)
+            opt.step()
+            opt.zero_grad()
+            torch.cuda.synchronize()
+            ok = ok and bool(np.array_equal(flat(params), o_out))
+        q.put((rank, ok, len(opt._copy_in)))
+        dist.barrier()
+        opt.close()
+    except Exception as e:
+        q.put((rank, "error", repr(e)))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+def test_zero_adamw_two_processes():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _port()
+    procs = [ctx.Process(target=_rank_main_optim, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=240) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=60)
+    for r in results:
+        assert r[1] is True, r
+    assert all(p.exitcode == 0 for p in procs)
