@@ -129,6 +129,22 @@ class ZeroAdamW:
             self.plan.step(self._grads, self.master, self.m, self.v, self.param_buffer, self.step_count)
         return None
 
+    def save(self, path):
+        """This rank's fp32 master / m / v and the step count to `path` (one
+        file per rank; zr_state_export_params turns a complete set into a
+        whole-model file)."""
+        from . import zr_state_save
+        zr_state_save(self.plan.handle, path, self.master, self.m, self.v, self.step_count)
+
+    def load(self, path):
+        """Restores this rank's state and step count from `path` (a shard of
+        the same partition and rank) and writes the restored master weights,
+        rounded to bf16, into this rank's parameters."""
+        from . import zr_state_load
+        self.step_count = zr_state_load(self.plan.handle, path, self.master, self.m, self.v)
+        for owned, glob, length in self.plan.runs():
+            self.param_buffer[glob:glob + length] = self.master[owned:owned + length].to(self.param_buffer.dtype)
+
     def close(self):
         if self.peer is not None:
             self.peer.close()

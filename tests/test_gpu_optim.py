@@ -60,3 +60,41 @@ def test_zero_adamw_one_rank_matches_the_oracle(partition, clip):
             # one rank: owned order is the global order
             assert np.array_equal(bits32(opt.master[:N].cpu().numpy()), bits32(o_master))
     opt.close()
+
+
+def test_zero_adamw_save_and_resume(tmp_path):
+    """Two steps, save, a fresh model and optimizer loaded from the shard,
+    a third step: equal to three uninterrupted steps bit for bit."""
+    import os
+
+    def batches():
+        gen = torch.Generator(device=DEV).manual_seed(7)
+        return [torch.randn(32, 64, device=DEV, generator=gen).to(torch.bfloat16) for _ in range(3)]
+
+    xs = batches()
+    ref_model = make_model(3)
+    ref = ZeroAdamW(list(ref_model.parameters()), lr=1e-3)
+    for x in xs:
+        ref_model(x).float().pow(2).mean().backward()
+        ref.step()
+        ref.zero_grad()
+    model = make_model(3)
+    opt = ZeroAdamW(list(model.parameters()), lr=1e-3)
+    for x in xs[:2]:
+        model(x).float().pow(2).mean().backward()
+        opt.step()
+        opt.zero_grad()
+    path = os.path.join(str(tmp_path), "rank0.zrs")
+    opt.save(path)
+    model2 = make_model(99)                                   # other initial weights: replaced by the load
+    opt2 = ZeroAdamW(list(model2.parameters()), lr=1e-3)
+    opt2.load(path)
+    assert opt2.step_count == 2
+    model2(xs[2]).float().pow(2).mean().backward()
+    opt2.step()
+    torch.cuda.synchronize()
+    assert np.array_equal(flat_u16(model2.parameters()), flat_u16(ref_model.parameters()))
+    for a, b in ((opt2.master, ref.master), (opt2.m, ref.m), (opt2.v, ref.v)):
+        assert np.array_equal(bits32(a.cpu().numpy()), bits32(b.cpu().numpy()))
+    for o in (ref, opt, opt2):
+        o.close()
