@@ -386,7 +386,8 @@ zr_status zr_state_export_params(const zr_plan* plan, const char* const* src_pat
  * zr_step_device_count, zr_step_bucket / zr_step_finish, zr_step_host,
  * zr_step_no_alloc; zr_step_host then copies the shard back in owned
  * order).  Changing it rebuilds the tile tables and, when a workspace is
- * bound, uploads them on `stream` and clears checked mode's status.
+ * bound, uploads them on `stream` and clears checked mode's status; work
+ * queued on other streams that reads the tables must be ordered before it.
  * ZR_PARAMS_OWNED with gather targets set is ZR_ERR_UNSUPPORTED.
  *
  * zr_gather_params writes tensors first_tensor .. first_tensor + n_tensors
