@@ -62,6 +62,8 @@ def parse():
                          "after it, against zr_step_bucket as each bucket's gradients complete")
     ap.add_argument("--zero3", action="store_true",
                     help="ZeRO-3 parameter gather: bandwidth, and prefetch against an emulated forward")
+    ap.add_argument("--zero3-set", default="1p3b", choices=["1p3b", "gpt2"],
+                    help="tensor set of --zero3 (gpt2: a small case, e.g. for profiling)")
     ap.add_argument("--checked", action="store_true",
                     help="checked mode: the device tile tables verified before every launch")
     ap.add_argument("--sweep", action="store_true",
@@ -715,8 +717,9 @@ def run_overlap(args):
 
 
 def run_zero3(args):
-    """ZeRO-3 parameter gather on the 1.3B set, flat, W = 8: every rank's
-    bf16 shard resident on this GPU (standing in for peer mappings).
+    """ZeRO-3 parameter gather on the 1.3B set (or the GPT-2 set), flat,
+    W = 8: every rank's bf16 shard resident on this GPU (standing in for
+    peer mappings).
 
     Measured: (a) one zr_gather_params of the whole model and of one
     transformer block, against the copy roofline (2 bytes read + 2 written
@@ -732,7 +735,10 @@ def run_zero3(args):
     from sharded_optimizer_step_zr_b200.plan import ZrPlan
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
-    wl = next(w for w in synth.sweep_workloads() if w.name == "sweep_1p3b_flat_w8_cap25")
+    if args.zero3_set == "gpt2":
+        wl = synth.WORKLOADS["gpt2_124m_w8"]
+    else:
+        wl = next(w for w in synth.sweep_workloads() if w.name == "sweep_1p3b_flat_w8_cap25")
     W = wl.world_size
     plans = [ZrPlan(wl.shapes, W, r, wl.mode, wl.bucket_cap_bytes, *wl.hp, device=dev, bind=(r == 0))
              for r in range(W)]
@@ -745,7 +751,9 @@ def run_zero3(args):
         p.close()
     numels = [int(math.prod(s)) for s in wl.shapes]
     # GPT blocks: tensors 2 + 12 i .. 2 + 12 i + 11 (wte and wpe first, ln_f last)
-    n_blocks, per_block = 24, 12
+    per_block = 12
+    n_blocks = (len(numels) - 4) // per_block
+    d_model = int(wl.shapes[1][1])
     block_params = sum(numels[2:2 + per_block])
     layer_buf = [torch.empty(block_params, dtype=torch.bfloat16, device=dev) for _ in range(2)]
     full = torch.empty(sum(numels), dtype=torch.bfloat16, device=dev)
@@ -768,10 +776,10 @@ def run_zero3(args):
     block_us = timed(lambda: plan.gather_params(2, per_block, shards, layer_buf[0]), 200)
     gb = lambda elems, us: 4 * elems / (us * 1e-6) / 1e9
 
-    # emulated forward: per block [8192, 2048] x [2048, 24576] bf16, 2 * 8192 * 12 * 2048^2 flops --
-    # a 1.3B block's forward (12 d^2 weights) at 8192 tokens
-    x = torch.randn(8192, 2048, dtype=torch.bfloat16, device=dev)
-    w_ = torch.randn(2048, 24576, dtype=torch.bfloat16, device=dev)
+    # emulated forward: per block [8192, d] x [d, 12 d] bf16, 2 * 8192 * 12 * d^2 flops -- a
+    # block's forward (12 d^2 weights) at 8192 tokens
+    x = torch.randn(8192, d_model, dtype=torch.bfloat16, device=dev)
+    w_ = torch.randn(d_model, 12 * d_model, dtype=torch.bfloat16, device=dev)
     compute = torch.cuda.Stream()
     lo, hi = torch.cuda.Stream.priority_range() if hasattr(torch.cuda.Stream, "priority_range") else (0, -1)
     side_streams = {"default": torch.cuda.Stream(), "high": torch.cuda.Stream(priority=hi)}
@@ -821,7 +829,7 @@ def run_zero3(args):
     capped_us = {c: timed(lambda: plan.gather_params(2, per_block, shards, layer_buf[0], None, c), 50)
                  for c in (16, 32)}
     line = {
-        "mode": "zero3_gather", "workload": "gpt_1p3b flat W=8, all ranks' shards on one GPU",
+        "mode": "zero3_gather", "workload": f"{wl.name} (flat W={W}), all ranks' shards on one GPU",
         "params": sum(numels), "block_params": block_params, "unit": "us",
         "gather_whole_model_us": whole_us, "gather_whole_model_gbs": gb(sum(numels), whole_us),
         "gather_block_us": block_us, "gather_block_gbs": gb(block_params, block_us),
