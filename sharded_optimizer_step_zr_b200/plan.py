@@ -120,6 +120,22 @@ class ZrPlan:
         zr_plan_set_param_layout(self.handle, layout, stream)
         self.param_layout = layout
 
+    def bound_gather(self, first_tensor, n_tensors, shards, dst, stream=None, max_ctas=0):
+        """A callable f() that runs zr_gather_params on fixed arguments,
+        marshalled once: a per-layer prefetch loop then pays one C call per
+        gather, not the Python argument handling."""
+        from . import _addr, _check, _lib, _ptr_array, _stream
+        arr = _ptr_array(shards)
+        args = (self.handle, int(first_tensor), int(n_tensors), arr, _addr(dst), int(max_ctas), _stream(stream))
+        fn = _lib.zr_gather_params
+
+        def gather_fn():
+            st = fn(*args)
+            if st:
+                _check(st, "zr_gather_params")
+        gather_fn._keepalive = (arr, shards, dst)
+        return gather_fn
+
     def gather_params(self, first_tensor, n_tensors, shards, dst, stream=None, max_ctas=0):
         """Tensors [first_tensor, first_tensor + n_tensors) whole, in the
         global layout, into dst, from every rank's bf16 shard (owned order);
