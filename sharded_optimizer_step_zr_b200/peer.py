@@ -147,6 +147,13 @@ class PeerZero:
             raise ValueError("gather is the stage-3 parameter all-gather")
         zr_gather_params(self.plan.handle, first_tensor, n_tensors, self.shard_ptrs, dst, stream, max_ctas)
 
+    def bound_gather(self, first_tensor, n_tensors, dst, stream=None, max_ctas=0):
+        """gather() with its arguments marshalled once: a callable for a
+        per-layer prefetch loop (see ZrPlan.bound_gather)."""
+        if self.stage != 3:
+            raise ValueError("gather is the stage-3 parameter all-gather")
+        return self.plan.bound_gather(first_tensor, n_tensors, self.shard_ptrs, dst, stream, max_ctas)
+
     def close(self):
         if self._opened:
             self.dist.barrier(self.group)

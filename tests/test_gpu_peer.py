@@ -147,7 +147,7 @@ def _rank_main_stage3(rank, world, port, shapes, mode, q):
         numels = [int(np.prod(s)) for s in shapes]
         goff = np.concatenate([[0], np.cumsum(numels)])
         one = torch.zeros(max(numels[2], 8), dtype=torch.bfloat16, device="cuda:0")
-        pz.gather(2, 1, one, max_ctas=4)
+        pz.bound_gather(2, 1, one, max_ctas=4)()
         torch.cuda.synchronize()
         got = full[:N].cpu().numpy().view(np.uint16)
         got_one = one[:numels[2]].cpu().view(torch.int16).numpy().view(np.uint16)
