@@ -30,8 +30,10 @@ class ZeroAdamW:
             raise ValueError("no parameters")
         dev = self.params[0].device
         for p in self.params:
-            if p.dtype != torch.bfloat16 or p.device != dev:
+            if p.dtype != torch.bfloat16 or p.device != dev or dev.type != "cuda":
                 raise ValueError("parameters must be bf16 tensors on one CUDA device")
+        if partition not in ("flat", "whole"):
+            raise ValueError("partition is 'flat' or 'whole'")
         mode = {"flat": ZR_PARTITION_FLAT, "whole": ZR_PARTITION_WHOLE_TENSOR}[partition]
         shapes = [tuple(p.shape) for p in self.params]
         self.hp = dict(lr=lr, beta1=betas[0], beta2=betas[1], eps=eps, weight_decay=weight_decay,

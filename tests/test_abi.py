@@ -275,3 +275,14 @@ def test_set_device_lr_arguments():
         zr.zr_plan_set_device_lr(h, None)
     finally:
         zr.zr_plan_destroy(h)
+
+
+def test_zero_adamw_rejects_parameters_it_cannot_bind():
+    import torch
+    from sharded_optimizer_step_zr_b200.optim import ZeroAdamW
+    with pytest.raises(ValueError, match="no parameters"):
+        ZeroAdamW([])
+    with pytest.raises(ValueError, match="bf16 tensors on one CUDA device"):
+        ZeroAdamW([torch.nn.Parameter(torch.zeros(4, dtype=torch.float32))])
+    with pytest.raises(ValueError, match="bf16 tensors on one CUDA device"):
+        ZeroAdamW([torch.nn.Parameter(torch.zeros(4, dtype=torch.bfloat16))])   # host memory
