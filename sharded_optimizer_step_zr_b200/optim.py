@@ -152,3 +152,198 @@ class ZeroAdamW:
             self.peer.close()
         else:
             self.plan.close()
+
+
+class Zero3:
+    """ZeRO stage 3 for a torch module ("Scaling training to thousands of
+    GPUs", talk summary, section 11:24 ZeRO; "CS336 lecture 8", section
+    "ZeRO levels"): each rank keeps only its bf16 shard of the parameters
+    (owned order) and its fp32 master / m / v slice; a module's parameters
+    are gathered from all shards just before its forward -- the next
+    module's ahead of time, on a side stream -- and again just before its
+    backward.
+
+    Every module that owns parameters directly gets one of two rotating
+    gather slots (module i: slot i mod 2), and its parameters stay views of
+    that slot, so only two modules' parameters are ever whole.  Autograd's
+    saved weights are those views: the slot is refilled with the module's
+    parameters before its backward reads them.  Gradients are bound to the
+    replica's gradient buffer as in ZeroAdamW.  The rotation assumes the
+    units run as a chain: forward in the order of module.parameters(), each
+    once, and backward in reverse (a sequential stack of layers).
+
+        z = Zero3(model, group=None, lr=3e-4)
+        loss = model(x).sum(); loss.backward(); z.step(); z.zero_grad()
+    """
+
+    def __init__(self, module, group=None, lr=3e-4, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.1,
+                 max_grad_norm=0.0, partition="flat", bucket_cap_mb=25):
+        import torch
+        from . import ZR_PARAMS_OWNED
+        self.module = module
+        params = list(module.parameters())
+        if not params:
+            raise ValueError("no parameters")
+        dev = params[0].device
+        for p in params:
+            if p.dtype != torch.bfloat16 or p.device != dev or dev.type != "cuda":
+                raise ValueError("parameters must be bf16 tensors on one CUDA device")
+        if partition not in ("flat", "whole"):
+            raise ValueError("partition is 'flat' or 'whole'")
+        # the units: modules owning parameters directly, each a run of consecutive tensors
+        index = {id(p): i for i, p in enumerate(params)}
+        self.units = []
+        for mod in module.modules():
+            own = list(mod.parameters(recurse=False))
+            if not own:
+                continue
+            ids = [index[id(p)] for p in own]
+            if ids != list(range(ids[0], ids[0] + len(ids))):
+                raise ValueError("a module's parameters must be consecutive in module.parameters()")
+            self.units.append((mod, ids[0], len(ids)))
+        self.units.sort(key=lambda u: u[1])
+        mode = {"flat": ZR_PARTITION_FLAT, "whole": ZR_PARTITION_WHOLE_TENSOR}[partition]
+        shapes = [tuple(p.shape) for p in params]
+        self.hp = dict(lr=lr, beta1=betas[0], beta2=betas[1], eps=eps, weight_decay=weight_decay,
+                       max_grad_norm=max_grad_norm)
+        hp = tuple(self.hp.values())
+        cap = int(bucket_cap_mb * (1 << 20))
+        world = 1
+        if group is not None:
+            import torch.distributed as dist
+            world = dist.get_world_size(group)
+        if world > 1:
+            from .peer import PeerZero
+            self.peer = PeerZero(group, shapes, mode, cap, *hp, device=dev, stage=3)
+            self.plan = self.peer.plan
+            self.grad_buffer = self.peer.grad_buffer
+            self.offsets = self.peer.offsets
+            self.shard = self.peer.param_shard
+            shard_ptrs = self.peer.shard_ptrs
+        else:
+            from .plan import ZrPlan
+            self.peer = None
+            self.plan = ZrPlan(shapes, 1, 0, mode, cap, *hp, device=dev)
+            self.plan.set_param_layout(ZR_PARAMS_OWNED)
+            self.offsets = [0, self.plan.padded_numel]
+            self.grad_buffer = torch.zeros(max(self.plan.padded_numel, 8), dtype=torch.bfloat16, device=dev)
+            self.shard = torch.zeros(max(self.plan.owned_numel, 8), dtype=torch.bfloat16, device=dev)
+            shard_ptrs = [self.shard]
+        # this rank's shard and fp32 state from the current (whole) parameters
+        goff = [0]
+        for p in params:
+            goff.append(goff[-1] + p.numel())
+        whole = torch.cat([p.detach().reshape(-1) for p in params])
+        n = self.plan.owned_numel
+        self.master = torch.zeros(max(n, 8), dtype=torch.float32, device=dev)
+        for owned, glob, length in self.plan.runs():
+            if glob < whole.numel():
+                k = min(length, whole.numel() - glob)
+                self.shard[owned:owned + k] = whole[glob:glob + k]
+        self.master[:n] = self.shard[:n].float()
+        self.m = torch.zeros_like(self.master)
+        self.v = torch.zeros_like(self.master)
+        del whole
+        # two slots; each unit's parameters become views of its slot
+        biggest = max(goff[a + k] - goff[a] for _, a, k in self.units)
+        self.slots = [torch.zeros(max(biggest, 8), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.side = torch.cuda.Stream(device=dev)
+        self.ready = [torch.cuda.Event() for _ in self.units]
+        for u, (mod, a, k) in enumerate(self.units):
+            slot = self.slots[u % 2]
+            with torch.no_grad():
+                for t in range(a, a + k):
+                    p = params[t]
+                    p.data = slot[goff[t] - goff[a]:goff[t + 1] - goff[a]].view(p.shape)
+            mod.register_forward_pre_hook(self._make_forward_hook(u))
+            mod.register_full_backward_pre_hook(self._make_backward_hook(u))
+        self._shard_ptrs, self._slot_of = shard_ptrs, [self.slots[u % 2] for u in range(len(self.units))]
+        self._prefetched = [False] * len(self.units)
+        # gradients: as ZeroAdamW
+        segs = self.plan.segments()
+        self.params = params
+        self._bound, self._copy_in = [], []
+        for t, p in enumerate(params):
+            pieces = sorted((s["offset_in_tensor"], s["owner"], s["owned_offset"], s["length"])
+                            for s in segs if s["tensor"] == t)
+            starts = [self.offsets[r] + o for _, r, o, _ in pieces]
+            contiguous = all(starts[i] + pieces[i][3] == starts[i + 1] for i in range(len(pieces) - 1))
+            if pieces and contiguous:
+                p.grad = self.grad_buffer[starts[0]:starts[0] + p.numel()].view(p.shape)
+                self._bound.append((p, starts[0]))
+            else:
+                p.grad = torch.zeros_like(p)
+                self._copy_in.append((p, [(off, self.offsets[r] + o, n_) for off, r, o, n_ in pieces]))
+        self.step_count = 0
+
+    def _gather(self, u, stream):
+        import torch
+        _, a, k = self.units[u]
+        self.plan.gather_params(a, k, self._shard_ptrs, self._slot_of[u], stream)
+
+    def _make_forward_hook(self, u):
+        def hook(module, inputs):
+            import torch
+            cur = torch.cuda.current_stream()
+            if self._prefetched[u]:
+                cur.wait_event(self.ready[u])             # gathered on the side stream
+                self._prefetched[u] = False
+            else:
+                self._gather(u, cur)
+            if u + 1 < len(self.units):
+                # the next unit's slot was the previous unit's: its forward is queued before this point
+                self.side.wait_stream(cur)
+                self._gather(u + 1, self.side)
+                self.ready[u + 1].record(self.side)
+                self._prefetched[u + 1] = True
+        return hook
+
+    def _make_backward_hook(self, u):
+        def hook(module, grad_output):
+            import torch
+            # the slot held later units since this unit's forward: refill it
+            self._gather(u, torch.cuda.current_stream())
+        return hook
+
+    def zero_grad(self, set_to_none=False):
+        self.grad_buffer.zero_()
+        for p, _ in self._copy_in:
+            p.grad.zero_()
+
+    def set_lr(self, lr):
+        self.hp["lr"] = lr
+        self.plan.set_adamw(*self.hp.values())
+
+    def step(self):
+        """One optimizer step (every rank together): the rank's slice of the
+        averaged gradient, AdamW, the bf16 result into the rank's shard."""
+        from . import zr_step
+        flat_grad = self.grad_buffer.view(-1)
+        for p, start in self._bound:
+            view = flat_grad[start:start + p.numel()]
+            if p.grad is None or p.grad.data_ptr() != view.data_ptr():
+                if p.grad is not None:
+                    view.copy_(p.grad.reshape(-1))
+                else:
+                    view.zero_()
+                p.grad = view.view(p.shape)
+        for p, pieces in self._copy_in:
+            g = p.grad.reshape(-1)
+            for off, start, n in pieces:
+                flat_grad[start:start + n].copy_(g[off:off + n])
+        self.step_count += 1
+        if self.peer is not None:
+            self.peer.step(self.master, self.m, self.v, self.step_count)
+        else:
+            self.plan.step([self.grad_buffer], self.master, self.m, self.v, self.shard, self.step_count)
+        self._prefetched = [False] * len(self.units)
+
+    def gather_all(self, out):
+        """The whole model, in the global layout, into `out` (bf16)."""
+        self.plan.gather_params(0, len(self.params), self._shard_ptrs, out)
+
+    def close(self):
+        if self.peer is not None:
+            self.peer.close()
+        else:
+            self.plan.close()

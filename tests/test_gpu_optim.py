@@ -98,3 +98,45 @@ def test_zero_adamw_save_and_resume(tmp_path):
         assert np.array_equal(bits32(a.cpu().numpy()), bits32(b.cpu().numpy()))
     for o in (ref, opt, opt2):
         o.close()
+
+
+def make_deep_model(seed):
+    torch.manual_seed(seed)
+    return torch.nn.Sequential(torch.nn.Linear(64, 128), torch.nn.GELU(), torch.nn.Linear(128, 128), torch.nn.GELU(),
+                               torch.nn.Linear(128, 96), torch.nn.LayerNorm(96), torch.nn.Linear(96, 24)
+                               ).to(DEV).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("partition", ["flat", "whole"])
+def test_zero3_trains_like_zero_adamw(partition):
+    """Zero3 (each module's parameters gathered from the shard before its
+    forward and again before its backward, two rotating slots) takes the
+    same steps as ZeroAdamW with every parameter resident: after each of
+    three steps the gathered model equals the other one bit for bit, and so
+    do the losses."""
+    from sharded_optimizer_step_zr_b200.optim import Zero3
+    a, b = make_deep_model(8), make_deep_model(8)
+    z2 = ZeroAdamW(list(a.parameters()), lr=1e-3, partition=partition)
+    z3 = Zero3(b, lr=1e-3, partition=partition)
+    N = sum(p.numel() for p in a.parameters())
+    big = max(sum(p.numel() for p in m.parameters(recurse=False)) for m in b.modules())
+    assert all(s.numel() == max(big, 8) for s in z3.slots)          # two slots of the largest module
+    gen = torch.Generator(device=DEV).manual_seed(21)
+    for t in (1, 2, 3):
+        x = torch.randn(32, 64, device=DEV, generator=gen).to(torch.bfloat16)
+        la = a(x).float().pow(2).mean()
+        la.backward()
+        z2.step()
+        z2.zero_grad()
+        lb = b(x).float().pow(2).mean()
+        lb.backward()
+        z3.step()
+        z3.zero_grad()
+        torch.cuda.synchronize()
+        assert la.item() == lb.item(), t
+        full = torch.empty(N, dtype=torch.bfloat16, device=DEV)
+        z3.gather_all(full)
+        torch.cuda.synchronize()
+        assert np.array_equal(full.cpu().view(torch.int16).numpy(), flat_u16(a.parameters()).view(np.int16)), t
+    z2.close()
+    z3.close()
