@@ -250,3 +250,72 @@ def test_zero_adamw_two_processes():
     for r in results:
         assert r[1] is True, r
     assert all(p.exitcode == 0 for p in procs)
+
+
+def _rank_main_zero3(rank, world, port, q):
+    """Zero3 over a two-process group: parameters gathered from both ranks'
+    shards (one through IPC) before each module's forward and backward;
+    after every step the gathered model equals the oracle's unsharded step
+    on the two replicas' gradients."""
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    import torch
+    import torch.distributed as dist
+    import oracle
+    from sharded_optimizer_step_zr_b200.optim import Zero3
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=90))
+    try:
+        torch.manual_seed(6)
+        model = torch.nn.Sequential(torch.nn.Linear(64, 128), torch.nn.GELU(), torch.nn.Linear(128, 96),
+                                    torch.nn.LayerNorm(96), torch.nn.Linear(96, 24)).to("cuda:0").to(torch.bfloat16)
+        flat = lambda ts: torch.cat([t.detach().reshape(-1) for t in ts]).cpu().view(torch.int16).numpy() \
+            .view(np.uint16).copy()
+        init = flat(model.parameters())
+        hp = (1e-3, 0.9, 0.999, 1e-8, 0.1, 0.0)
+        z = Zero3(model, group=dist.group.WORLD, lr=hp[0], weight_decay=hp[4], bucket_cap_mb=0.01)
+        N = init.size
+        o_master = (init.astype(np.uint32) << 16).view(np.float32).copy()
+        o_m, o_v, o_out = np.zeros(N, np.float32), np.zeros(N, np.float32), np.zeros(N, np.uint16)
+        gen = torch.Generator(device="cuda:0").manual_seed(300 + rank)
+        ok = True
+        full = torch.empty(N, dtype=torch.bfloat16, device="cuda:0")
+        for t in (1, 2, 3):
+            x = torch.randn(16, 64, device="cuda:0", generator=gen).to(torch.bfloat16)
+            model(x).float().pow(2).mean().backward()
+            torch.cuda.synchronize()
+            mine = flat([p.grad for p in z.params])
+            reps = [None] * world
+            dist.all_gather_object(reps, mine)
+            oracle.ddp_step(reps, o_master, o_m, o_v, o_out, hp, t)
+            z.step()
+            z.zero_grad()
+            z.gather_all(full)
+            torch.cuda.synchronize()
+            ok = ok and bool(np.array_equal(full.cpu().view(torch.int16).numpy().view(np.uint16), o_out))
+        q.put((rank, ok))
+        dist.barrier()
+        z.close()
+    except Exception as e:
+        q.put((rank, "error", repr(e)))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+def test_zero3_module_two_processes():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _port()
+    procs = [ctx.Process(target=_rank_main_zero3, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=240) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=60)
+    for r in results:
+        assert r[1] is True, r
+    assert all(p.exitcode == 0 for p in procs)
