@@ -170,7 +170,9 @@ class Zero3:
     parameters before its backward reads them.  Gradients are bound to the
     replica's gradient buffer as in ZeroAdamW.  The rotation assumes the
     units run as a chain: forward in the order of module.parameters(), each
-    once, and backward in reverse (a sequential stack of layers).
+    once, and backward in reverse (a sequential stack of layers); a
+    parameter used by a module other than its owner (tied weights) is not
+    supported, since that module would read whatever the slot holds.
 
         z = Zero3(model, group=None, lr=3e-4)
         loss = model(x).sum(); loss.backward(); z.step(); z.zero_grad()
