@@ -62,6 +62,8 @@ def parse():
                          "after it, against zr_step_bucket as each bucket's gradients complete")
     ap.add_argument("--zero3", action="store_true",
                     help="ZeRO-3 parameter gather: bandwidth, and prefetch against an emulated forward")
+    ap.add_argument("--zero3-train", action="store_true",
+                    help="training steps of an MLP stack: ZeroAdamW against Zero3 (the layer loop's cost)")
     ap.add_argument("--zero3-set", default="1p3b", choices=["1p3b", "gpt2"],
                     help="tensor set of --zero3 (gpt2: a small case, e.g. for profiling)")
     ap.add_argument("--checked", action="store_true",
@@ -851,8 +853,71 @@ def run_zero3(args):
     plan.close()
 
 
+def run_zero3_train(args):
+    """Training steps of a stack of MLP blocks (12 x [Linear(d, 4d), GELU,
+    Linear(4d, d)], d = 2048: 403 M bf16 parameters; 4096 tokens) with
+    ZeroAdamW (every parameter resident) and with Zero3 (each layer
+    gathered from the shard before its forward and again before its
+    backward, the next layer's forward gather prefetched), one rank.  Both
+    take the same steps (checked); the difference in step time is what the
+    layer loop costs on one GPU.  Prints one JSON record."""
+    import torch
+    from sharded_optimizer_step_zr_b200.optim import Zero3, ZeroAdamW
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    d, n_blocks, tokens = 2048, 12, 4096
+
+    def model(seed):
+        torch.manual_seed(seed)
+        layers = []
+        for _ in range(n_blocks):
+            layers += [torch.nn.Linear(d, 4 * d), torch.nn.GELU(), torch.nn.Linear(4 * d, d)]
+        return torch.nn.Sequential(*layers).to(dev).to(torch.bfloat16)
+
+    a, b = model(1), model(1)
+    n_params = sum(p.numel() for p in a.parameters())
+    z2 = ZeroAdamW(list(a.parameters()), lr=1e-4)
+    z3 = Zero3(b, lr=1e-4)
+    x = torch.randn(tokens, d, device=dev, dtype=torch.bfloat16)
+
+    def step(m, opt):
+        m(x).float().pow(2).mean().backward()
+        opt.step()
+        opt.zero_grad()
+
+    def timed(m, opt, reps):
+        for _ in range(2):
+            step(m, opt)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            step(m, opt)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    t2 = timed(a, z2, 5)
+    t3 = timed(b, z3, 5)
+    full = torch.empty(n_params, dtype=torch.bfloat16, device=dev)
+    z3.gather_all(full)
+    resident = torch.cat([p.detach().reshape(-1) for p in a.parameters()])
+    same = bool(torch.equal(full.view(torch.int16), resident.view(torch.int16)))
+    flops = 6 * tokens * n_params
+    line = {"mode": "zero3_train", "params": n_params, "tokens": tokens, "blocks": n_blocks, "unit": "ms",
+            "zero_adamw_step_ms": t2, "zero3_step_ms": t3, "layer_loop_overhead_ms": t3 - t2,
+            "gathers_per_step": 2 * len(z3.units), "gathered_bytes_per_step": 2 * 2 * n_params,
+            "model_tflops_zero_adamw": flops / (t2 * 1e-3) / 1e12, "same_parameters": same}
+    print(json.dumps(line), flush=True)
+    z2.close()
+    z3.close()
+
+
 def main():
     args = parse()
+    if args.zero3_train:
+        run_zero3_train(args)
+        return
     if args.overlap:
         run_overlap(args)
         return
