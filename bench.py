@@ -874,10 +874,11 @@ def run_zero3_train(args):
             layers += [torch.nn.Linear(d, 4 * d), torch.nn.GELU(), torch.nn.Linear(4 * d, d)]
         return torch.nn.Sequential(*layers).to(dev).to(torch.bfloat16)
 
-    a, b = model(1), model(1)
+    a, b, c = model(1), model(1), model(1)
     n_params = sum(p.numel() for p in a.parameters())
     z2 = ZeroAdamW(list(a.parameters()), lr=1e-4)
     z3 = Zero3(b, lr=1e-4)
+    z3_fwd_only = Zero3(c, lr=1e-4, backward_prefetch=False)
     x = torch.randn(tokens, d, device=dev, dtype=torch.bfloat16)
 
     def step(m, opt):
@@ -899,6 +900,7 @@ def run_zero3_train(args):
 
     t2 = timed(a, z2, 5)
     t3 = timed(b, z3, 5)
+    t3f = timed(c, z3_fwd_only, 5)
     full = torch.empty(n_params, dtype=torch.bfloat16, device=dev)
     z3.gather_all(full)
     resident = torch.cat([p.detach().reshape(-1) for p in a.parameters()])
@@ -906,11 +908,13 @@ def run_zero3_train(args):
     flops = 6 * tokens * n_params
     line = {"mode": "zero3_train", "params": n_params, "tokens": tokens, "blocks": n_blocks, "unit": "ms",
             "zero_adamw_step_ms": t2, "zero3_step_ms": t3, "layer_loop_overhead_ms": t3 - t2,
+            "zero3_forward_prefetch_only_step_ms": t3f,
             "gathers_per_step": 2 * len(z3.units), "gathered_bytes_per_step": 2 * 2 * n_params,
             "model_tflops_zero_adamw": flops / (t2 * 1e-3) / 1e12, "same_parameters": same}
     print(json.dumps(line), flush=True)
     z2.close()
     z3.close()
+    z3_fwd_only.close()
 
 
 def main():

@@ -159,9 +159,9 @@ class Zero3:
     GPUs", talk summary, section 11:24 ZeRO; "CS336 lecture 8", section
     "ZeRO levels"): each rank keeps only its bf16 shard of the parameters
     (owned order) and its fp32 master / m / v slice; a module's parameters
-    are gathered from all shards just before its forward -- the next
-    module's ahead of time, on a side stream -- and again just before its
-    backward.
+    are gathered from all shards just before its forward and again just
+    before its backward -- in both passes the next module's ahead of time,
+    on a side stream (backward_prefetch=False keeps the backward's in line).
 
     Every module that owns parameters directly gets one of two rotating
     gather slots (module i: slot i mod 2), and its parameters stay views of
@@ -179,7 +179,7 @@ class Zero3:
     """
 
     def __init__(self, module, group=None, lr=3e-4, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.1,
-                 max_grad_norm=0.0, partition="flat", bucket_cap_mb=25):
+                 max_grad_norm=0.0, partition="flat", bucket_cap_mb=25, backward_prefetch=True):
         import torch
         from . import ZR_PARAMS_OWNED
         self.module = module
@@ -261,6 +261,9 @@ class Zero3:
             mod.register_full_backward_pre_hook(self._make_backward_hook(u))
         self._shard_ptrs, self._slot_of = shard_ptrs, [self.slots[u % 2] for u in range(len(self.units))]
         self._prefetched = [False] * len(self.units)
+        self.back_ready = [torch.cuda.Event() for _ in self.units]
+        self._back_prefetched = [False] * len(self.units)
+        self.backward_prefetch = backward_prefetch
         # gradients: as ZeroAdamW
         segs = self.plan.segments()
         self.params = params
@@ -303,8 +306,20 @@ class Zero3:
     def _make_backward_hook(self, u):
         def hook(module, grad_output):
             import torch
+            cur = torch.cuda.current_stream()
             # the slot held later units since this unit's forward: refill it
-            self._gather(u, torch.cuda.current_stream())
+            # (prefetched during the next unit's backward, or now)
+            if self._back_prefetched[u]:
+                cur.wait_event(self.back_ready[u])
+                self._back_prefetched[u] = False
+            else:
+                self._gather(u, cur)
+            if self.backward_prefetch and u >= 1:
+                # unit u - 1's slot last held unit u + 1, whose backward is queued before this point
+                self.side.wait_stream(cur)
+                self._gather(u - 1, self.side)
+                self.back_ready[u - 1].record(self.side)
+                self._back_prefetched[u - 1] = True
         return hook
 
     def zero_grad(self, set_to_none=False):
@@ -339,6 +354,7 @@ class Zero3:
         else:
             self.plan.step([self.grad_buffer], self.master, self.m, self.v, self.shard, self.step_count)
         self._prefetched = [False] * len(self.units)
+        self._back_prefetched = [False] * len(self.units)
 
     def gather_all(self, out):
         """The whole model, in the global layout, into `out` (bf16)."""
