@@ -356,6 +356,21 @@ class Zero3:
         self._prefetched = [False] * len(self.units)
         self._back_prefetched = [False] * len(self.units)
 
+    def save(self, path):
+        """This rank's fp32 master / m / v and the step count to `path`."""
+        from . import zr_state_save
+        zr_state_save(self.plan.handle, path, self.master, self.m, self.v, self.step_count)
+
+    def load(self, path):
+        """Restores this rank's state and step count; its bf16 shard becomes
+        the restored master weights rounded to bf16 (what the step writes)."""
+        from . import zr_state_load
+        self.step_count = zr_state_load(self.plan.handle, path, self.master, self.m, self.v)
+        n = self.plan.owned_numel
+        self.shard[:n] = self.master[:n].to(self.shard.dtype)
+        self._prefetched = [False] * len(self.units)
+        self._back_prefetched = [False] * len(self.units)
+
     def gather_all(self, out):
         """The whole model, in the global layout, into `out` (bf16)."""
         self.plan.gather_params(0, len(self.params), self._shard_ptrs, out)

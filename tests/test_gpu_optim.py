@@ -140,3 +140,38 @@ def test_zero3_trains_like_zero_adamw(partition):
         assert np.array_equal(full.cpu().view(torch.int16).numpy(), flat_u16(a.parameters()).view(np.int16)), t
     z2.close()
     z3.close()
+
+
+def test_zero3_save_and_resume(tmp_path):
+    import os
+    from sharded_optimizer_step_zr_b200.optim import Zero3
+    gen = torch.Generator(device=DEV).manual_seed(9)
+    xs = [torch.randn(32, 64, device=DEV, generator=gen).to(torch.bfloat16) for _ in range(3)]
+    ref_model = make_deep_model(4)
+    ref = Zero3(ref_model, lr=1e-3)
+    for x in xs:
+        ref_model(x).float().pow(2).mean().backward()
+        ref.step()
+        ref.zero_grad()
+    model = make_deep_model(4)
+    z = Zero3(model, lr=1e-3)
+    for x in xs[:2]:
+        model(x).float().pow(2).mean().backward()
+        z.step()
+        z.zero_grad()
+    path = os.path.join(str(tmp_path), "z3_rank0.zrs")
+    z.save(path)
+    model2 = make_deep_model(77)
+    z2 = Zero3(model2, lr=1e-3)
+    z2.load(path)
+    model2(xs[2]).float().pow(2).mean().backward()
+    z2.step()
+    N = sum(p.numel() for p in ref_model.parameters())
+    a = torch.empty(N, dtype=torch.bfloat16, device=DEV)
+    b = torch.empty(N, dtype=torch.bfloat16, device=DEV)
+    ref.gather_all(a)
+    z2.gather_all(b)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    for o in (ref, z, z2):
+        o.close()
