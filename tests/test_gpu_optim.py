@@ -175,3 +175,32 @@ def test_zero3_save_and_resume(tmp_path):
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
     for o in (ref, z, z2):
         o.close()
+
+
+def test_zero3_accumulation_and_evaluation():
+    """Two forward / backward passes per step (gradient accumulation) and a
+    no-grad evaluation forward between steps: Zero3's hooks gather for every
+    pass, and the steps equal ZeroAdamW's bit for bit."""
+    from sharded_optimizer_step_zr_b200.optim import Zero3
+    a, b = make_deep_model(12), make_deep_model(12)
+    z2 = ZeroAdamW(list(a.parameters()), lr=1e-3)
+    z3 = Zero3(b, lr=1e-3)
+    gen = torch.Generator(device=DEV).manual_seed(5)
+    N = sum(p.numel() for p in a.parameters())
+    for t in (1, 2):
+        xs = [torch.randn(16, 64, device=DEV, generator=gen).to(torch.bfloat16) for _ in range(3)]
+        for m, opt in ((a, z2), (b, z3)):
+            for x in xs[:2]:
+                m(x).float().pow(2).mean().backward()
+            opt.step()
+            opt.zero_grad()
+        with torch.no_grad():
+            ea, eb = a(xs[2]), b(xs[2])
+        torch.cuda.synchronize()
+        assert torch.equal(ea.view(torch.int16), eb.view(torch.int16)), t
+        full = torch.empty(N, dtype=torch.bfloat16, device=DEV)
+        z3.gather_all(full)
+        torch.cuda.synchronize()
+        assert np.array_equal(full.cpu().view(torch.int16).numpy(), flat_u16(a.parameters()).view(np.int16)), t
+    z2.close()
+    z3.close()
