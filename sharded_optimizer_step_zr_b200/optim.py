@@ -172,7 +172,9 @@ class Zero3:
     units run as a chain: forward in the order of module.parameters(), each
     once, and backward in reverse (a sequential stack of layers); a
     parameter used by a module other than its owner (tied weights) is not
-    supported, since that module would read whatever the slot holds.
+    supported, since that module would read whatever the slot holds.  With
+    a process group, every rank's module must start from the same
+    parameters (each rank's shard is cut from its own copy).
 
         z = Zero3(model, group=None, lr=3e-4)
         loss = model(x).sum(); loss.backward(); z.step(); z.zero_grad()
@@ -251,14 +253,15 @@ class Zero3:
         self.slots = [torch.zeros(max(biggest, 8), dtype=torch.bfloat16, device=dev) for _ in range(2)]
         self.side = torch.cuda.Stream(device=dev)
         self.ready = [torch.cuda.Event() for _ in self.units]
+        self._hooks = []
         for u, (mod, a, k) in enumerate(self.units):
             slot = self.slots[u % 2]
             with torch.no_grad():
                 for t in range(a, a + k):
                     p = params[t]
                     p.data = slot[goff[t] - goff[a]:goff[t + 1] - goff[a]].view(p.shape)
-            mod.register_forward_pre_hook(self._make_forward_hook(u))
-            mod.register_full_backward_pre_hook(self._make_backward_hook(u))
+            self._hooks.append(mod.register_forward_pre_hook(self._make_forward_hook(u)))
+            self._hooks.append(mod.register_full_backward_pre_hook(self._make_backward_hook(u)))
         self._shard_ptrs, self._slot_of = shard_ptrs, [self.slots[u % 2] for u in range(len(self.units))]
         self._prefetched = [False] * len(self.units)
         self.back_ready = [torch.cuda.Event() for _ in self.units]
@@ -376,6 +379,11 @@ class Zero3:
         self.plan.gather_params(0, len(self.params), self._shard_ptrs, out)
 
     def close(self):
+        """Removes the hooks (the module keeps the parameters last gathered
+        into its slots) and releases the plan."""
+        for h in self._hooks:
+            h.remove()
+        self._hooks = []
         if self.peer is not None:
             self.peer.close()
         else:
