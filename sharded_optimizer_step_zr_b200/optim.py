@@ -12,7 +12,9 @@ them).  Each rank holds only its owned slice of the fp32 master weights and
 Adam moments (ZeRO stage 1/2).  With one rank the plan's own buffers are
 used; with a process group of several ranks the buffers are shared between
 the processes over CUDA IPC (PeerZero), and the step reads the other
-replicas' gradients and writes every rank's parameters through peer memory.
+replicas' gradients and writes every rank's parameters through peer memory;
+every rank's model must then start from the same parameters (each rank's
+fp32 master slice is taken from its own copy).
 
 Only the buffer plumbing lives here: the step itself runs in libzr.so.
 """
