@@ -62,6 +62,8 @@ def parse():
                          "after it, against zr_step_bucket as each bucket's gradients complete")
     ap.add_argument("--zero3", action="store_true",
                     help="ZeRO-3 parameter gather: bandwidth, and prefetch against an emulated forward")
+    ap.add_argument("--vs-torch", action="store_true",
+                    help="the optimizer step against torch's fused AdamW mixed-precision recipe (context)")
     ap.add_argument("--zero3-train", action="store_true",
                     help="training steps of an MLP stack: ZeroAdamW against Zero3 (the layer loop's cost)")
     ap.add_argument("--zero3-set", default="1p3b", choices=["1p3b", "gpt2"],
@@ -917,8 +919,64 @@ def run_zero3_train(args):
     z3_fwd_only.close()
 
 
+def run_vs_torch(args):
+    """The optimizer step alone, one rank, on the 403 M-parameter MLP stack
+    of --zero3-train, against PyTorch's own mixed-precision recipe: fused
+    torch.optim.AdamW on fp32 master parameters (gradients cast from the
+    bf16 ones), then the masters copied back into the bf16 model.  Context,
+    not a target: both are memory-bound, and the fused step moves fewer
+    bytes (2 gradient + 24 state + 2 parameter per element at W = 1).
+    Prints one JSON record."""
+    import torch
+    from sharded_optimizer_step_zr_b200.optim import ZeroAdamW
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    d, n_blocks = 2048, 12
+    shapes = [(4 * d, d), (4 * d,), (d, 4 * d), (d,)] * n_blocks
+    torch.manual_seed(0)
+    model = [torch.nn.Parameter(torch.randn(s, device=dev).mul_(0.02).to(torch.bfloat16)) for s in shapes]
+    grads = [torch.randn(s, device=dev).mul_(1e-3).to(torch.bfloat16) for s in shapes]
+    n = sum(p.numel() for p in model)
+    z = ZeroAdamW(model, lr=1e-4)
+    for p, g in zip(model, grads):
+        p.grad.copy_(g)
+    masters = [torch.nn.Parameter(p.detach().float()) for p in model]
+    opt = torch.optim.AdamW(masters, lr=1e-4, weight_decay=0.1, fused=True)
+
+    def torch_step():
+        for mp, g in zip(masters, grads):
+            mp.grad = g.float()
+        opt.step()
+        with torch.no_grad():
+            for p, mp in zip(model, masters):
+                p.copy_(mp)
+
+    def timed(fn, reps=20):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    t_zr = timed(z.step)
+    t_torch = timed(torch_step)
+    line = {"mode": "vs_torch_adamw", "params": n, "unit": "ms", "zr_step_ms": t_zr,
+            "torch_fused_adamw_step_ms": t_torch, "speedup": t_torch / t_zr,
+            "zr_gbs_algorithmic": 28 * n / (t_zr * 1e-3) / 1e9}
+    print(json.dumps(line), flush=True)
+    z.close()
+
+
 def main():
     args = parse()
+    if args.vs_torch:
+        run_vs_torch(args)
+        return
     if args.zero3_train:
         run_zero3_train(args)
         return
