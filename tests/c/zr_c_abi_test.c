@@ -2,9 +2,10 @@
  * cudaMalloc, no Python, no torch.  Builds a plan for one rank of a small
  * flat partition, binds a workspace, runs four steps with constant
  * gradients (the last in checked mode, whose status must stay clean) and
- * checks the closed form of AdamW with a constant gradient:
- * each step moves p to p * (1 - lr * wd) - lr * g / (|g| + eps) (the bias
- * corrections cancel), within fp32 rounding.  Exit status 0 on success. */
+ * checks the closed form of AdamW with a constant gradient: each step moves
+ * p to p * (1 - lr * wd) - lr * g / (|g| + eps) (the bias corrections
+ * cancel), within fp32 rounding.  Then the ZeRO-3 calls (see below).  Exit
+ * status 0 on success. */
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -107,6 +108,63 @@ int main(void) {
         if (fabs(got[i] - want) > 1e-6 * fmax(fabs(want), lr)) ++bad;
     }
     zr_plan_destroy(plan);
-    printf("owned %lld, mismatches %lld\n", (long long)owned, (long long)bad);
-    return bad == 0 ? 0 : 1;
+
+    /* ZeRO-3 calls from C: a one-rank plan of the same tensors steps once
+     * in the global layout and once (on its own copy of the state) in the
+     * owned-order layout; zr_gather_params then reassembles the tensors
+     * from the shard, which must equal the global-layout result. */
+    int64_t mism3 = 0;
+    {
+        const zr_adamw hp1 = {3e-4f, 0.9f, 0.999f, 1e-8f, 0.1f, 0.0f};
+        zr_plan *g1 = NULL, *s1 = NULL;
+        CHECK_ZR(zr_plan_create(3, ndims, shapes, 1, 0, ZR_PARTITION_FLAT, 4096, &hp1, &g1));
+        CHECK_ZR(zr_plan_create(3, ndims, shapes, 1, 0, ZR_PARTITION_FLAT, 4096, &hp1, &s1));
+        uint64_t b1 = 0, b2 = 0;
+        CHECK_ZR(zr_plan_workspace_bytes(g1, &b1));
+        CHECK_ZR(zr_plan_workspace_bytes(s1, &b2));
+        void *w1, *w2;
+        CHECK_CUDA(cudaMalloc(&w1, b1));
+        CHECK_CUDA(cudaMalloc(&w2, b2));
+        CHECK_ZR(zr_plan_set_workspace(g1, w1, b1, (zr_stream_t)stream));
+        CHECK_ZR(zr_plan_set_workspace(s1, w2, b2, (zr_stream_t)stream));
+        CHECK_ZR(zr_plan_set_param_layout(s1, ZR_PARAMS_OWNED, (zr_stream_t)stream));
+        const int64_t N = total;
+        uint16_t* hg = (uint16_t*)malloc(sizeof(uint16_t) * N);
+        float* hp0 = (float*)malloc(sizeof(float) * N);
+        for (int64_t i = 0; i < N; ++i) {
+            hg[i] = bf16_of((float)((i % 7) - 3) / 8.0f);
+            hp0[i] = 0.01f * (float)((i % 13) - 6);
+        }
+        void *grad1, *out_g, *shard, *gathered;
+        float *ms[2], *mm[2], *vv[2];
+        CHECK_CUDA(cudaMalloc(&grad1, sizeof(uint16_t) * N));
+        CHECK_CUDA(cudaMemcpy(grad1, hg, sizeof(uint16_t) * N, cudaMemcpyHostToDevice));
+        for (int k = 0; k < 2; ++k) {
+            CHECK_CUDA(cudaMalloc((void**)&ms[k], sizeof(float) * N));
+            CHECK_CUDA(cudaMalloc((void**)&mm[k], sizeof(float) * N));
+            CHECK_CUDA(cudaMalloc((void**)&vv[k], sizeof(float) * N));
+            CHECK_CUDA(cudaMemcpy(ms[k], hp0, sizeof(float) * N, cudaMemcpyHostToDevice));
+            CHECK_CUDA(cudaMemset(mm[k], 0, sizeof(float) * N));
+            CHECK_CUDA(cudaMemset(vv[k], 0, sizeof(float) * N));
+        }
+        CHECK_CUDA(cudaMalloc(&out_g, sizeof(uint16_t) * N));
+        CHECK_CUDA(cudaMalloc(&shard, sizeof(uint16_t) * N));
+        CHECK_CUDA(cudaMalloc(&gathered, sizeof(uint16_t) * N));
+        const void* one_grad[1] = {grad1};
+        CHECK_ZR(zr_step(g1, one_grad, ms[0], mm[0], vv[0], out_g, 1, (zr_stream_t)stream));
+        CHECK_ZR(zr_step(s1, one_grad, ms[1], mm[1], vv[1], shard, 1, (zr_stream_t)stream));
+        const void* shards[1] = {shard};
+        CHECK_ZR(zr_gather_params(s1, 0, 3, shards, gathered, 0, (zr_stream_t)stream));
+        CHECK_CUDA(cudaStreamSynchronize(stream));
+        uint16_t* a = (uint16_t*)malloc(sizeof(uint16_t) * N);
+        uint16_t* b = (uint16_t*)malloc(sizeof(uint16_t) * N);
+        CHECK_CUDA(cudaMemcpy(a, out_g, sizeof(uint16_t) * N, cudaMemcpyDeviceToHost));
+        CHECK_CUDA(cudaMemcpy(b, gathered, sizeof(uint16_t) * N, cudaMemcpyDeviceToHost));
+        for (int64_t i = 0; i < N; ++i) mism3 += a[i] != b[i];
+        zr_plan_destroy(g1);
+        zr_plan_destroy(s1);
+    }
+    printf("owned %lld, mismatches %lld, zero-3 mismatches %lld\n", (long long)owned, (long long)bad,
+           (long long)mism3);
+    return (bad == 0 && mism3 == 0) ? 0 : 1;
 }
