@@ -1,6 +1,6 @@
 /*
- * zr.h -- C ABI of the fused ZeRO-1/2 sharded optimizer step for NVIDIA B200
- * (sm_100a).
+ * zr.h -- C ABI of the fused ZeRO sharded optimizer step for NVIDIA B200
+ * (sm_100a): stages 1 and 2, and the parameter side of stage 3.
  *
  * One step of data-parallel training with sharded optimizer state, for the
  * slice of parameters that one rank owns:
@@ -27,8 +27,10 @@
  *               ("CS336", ZeRO-1 sketch, update-then-gather).
  *
  * The four stages run as one fused, memory-bound GPU pass (two passes and a
- * tiny combine kernel when clipping).  All W replicas' gradients live in the
- * memory of the one GPU the call runs on; there is no collective.
+ * tiny combine kernel when clipping).  The W replicas' gradients live in
+ * memory the GPU can load from: its own, or other GPUs' buffers mapped with
+ * CUDA IPC (zr_ipc_*).  There is no collective: the reduce-scatter and the
+ * all-gather are the kernel's own loads and stores.
  *
  * Partitioning ("Scaling training to thousands of GPUs", 11:24 ZeRO, FSDP1
  * vs FSDP2):
@@ -135,13 +137,16 @@ zr_status zr_plan_query(const zr_plan* plan, int64_t* total_numel, int64_t* padd
  * ZR_ERR_BUFFER_TOO_SMALL is returned (call with cap 0 to size). */
 zr_status zr_plan_segments(const zr_plan* plan, zr_segment* out, int64_t cap, int64_t* n);
 
-/* Device workspace the plan needs: the tile table, the clip partial sums and
- * (when clipping with W > 4) an fp32 scratch copy of the reduced gradient. */
+/* Device workspace the plan needs: the tile tables, the clip partial sums,
+ * a few scalars and status words, the ZeRO-3 gather piece table (32 bytes
+ * per piece of at most 16384 elements, all ranks) and (when clipping with
+ * W > 4) an fp32 scratch copy of the reduced gradient. */
 zr_status zr_plan_workspace_bytes(const zr_plan* plan, uint64_t* bytes);
 
 /* Bind a device workspace (>= zr_plan_workspace_bytes, 256-byte aligned,
  * owned by the caller, kept alive while the plan is used) and upload the
- * tile table into it with an asynchronous copy on `stream`.  Selects the
+ * tile tables and the gather piece table into it with asynchronous copies
+ * on `stream` (clearing checked mode's status).  Selects the
  * current CUDA device as the plan's device.  Errors: ZR_ERR_NO_WORKSPACE
  * (too small), ZR_ERR_ALIGNMENT, ZR_ERR_UNSUPPORTED (the current device is
  * not compute capability 10.x), ZR_ERR_CUDA. */
