@@ -299,12 +299,14 @@ zr_status zr_debug_reduce(const zr_plan* plan, const void* const* grad_ptrs, flo
  * grad_ptrs[w].  offsets: world_size + 1 entries. */
 zr_status zr_plan_owner_offsets(const zr_plan* plan, int64_t* offsets);
 
-/* Make zr_step, zr_step_bucket and zr_step_finish store each bf16 result in
- * targets[0..world_size) (rank w's parameter buffer, global layout, local
- * or peer-mapped, 16-byte aligned) instead of param_out, which may then be
- * NULL.  The pointer array is copied into the workspace (synchronising
- * `stream`); targets == NULL goes back to param_out.  zr_step_host refuses a
- * plan with gather targets (ZR_ERR_UNSUPPORTED).  Needs a bound workspace. */
+/* Make zr_step, zr_step_device_count, zr_step_bucket and zr_step_finish
+ * store each bf16 result in targets[0..world_size) (rank w's parameter
+ * buffer, global layout, local or peer-mapped, 16-byte aligned) instead of
+ * param_out, which may then be NULL.  The pointer array is copied into the
+ * workspace (synchronising `stream`); targets == NULL goes back to
+ * param_out.  zr_step_host refuses a plan with gather targets
+ * (ZR_ERR_UNSUPPORTED); zr_step_no_alloc always writes param_out alone.
+ * Needs a bound workspace. */
 zr_status zr_plan_set_gather_targets(zr_plan* plan, void* const* targets, zr_stream_t stream);
 
 /* A device buffer as another process can map it: the CUDA IPC handle of the
