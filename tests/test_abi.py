@@ -286,3 +286,48 @@ def test_zero_adamw_rejects_parameters_it_cannot_bind():
         ZeroAdamW([torch.nn.Parameter(torch.zeros(4, dtype=torch.float32))])
     with pytest.raises(ValueError, match="bf16 tensors on one CUDA device"):
         ZeroAdamW([torch.nn.Parameter(torch.zeros(4, dtype=torch.bfloat16))])   # host memory
+
+
+def test_early_argument_errors_of_every_launching_call():
+    """Each call that launches work rejects a missing plan, a bad step or
+    an unbound workspace before any CUDA call (so these run without a GPU),
+    and the IPC calls reject NULL arguments."""
+    import ctypes
+    L = zr._lib
+    h = zr.zr_plan_create([(4096,), (100,)], 2, 0, 0, 1 << 20)
+    try:
+        g = zr._ptr_array([16, 16])
+        step_like = [
+            lambda p, t: L.zr_step(p, g, 16, 16, 16, 16, t, None),
+            lambda p, t: L.zr_step_bucket(p, 0, g, 16, 16, 16, 16, t, None),
+            lambda p, t: L.zr_step_finish(p, g, 16, 16, 16, 16, t, None),
+            lambda p, t: L.zr_step_host(p, g, g, 16, 16, 16, 16, 16, t, None),
+        ]
+        for call in step_like:
+            assert call(None, 1) == zr.ZR_ERR_INVALID_ARG
+            assert call(h, 0) == zr.ZR_ERR_INVALID_ARG            # steps are 1-based
+            assert call(h, 1) == zr.ZR_ERR_NO_WORKSPACE
+        assert L.zr_step_device_count(h, g, 16, 16, 16, 16, None, None) == zr.ZR_ERR_INVALID_ARG
+        assert L.zr_step_device_count(h, g, 16, 16, 16, 16, 4, None) == zr.ZR_ERR_ALIGNMENT
+        assert L.zr_step_device_count(h, g, 16, 16, 16, 16, 16, None) == zr.ZR_ERR_NO_WORKSPACE
+        assert L.zr_grad_sumsq(None, g, 16, None) == zr.ZR_ERR_INVALID_ARG
+        assert L.zr_debug_reduce(None, g, 16, None) == zr.ZR_ERR_INVALID_ARG
+        assert L.zr_step_no_alloc(None, g, 16, 16, 16, 16, None, 1, None) == zr.ZR_ERR_INVALID_ARG
+        assert L.zr_step_no_alloc(h, None, 16, 16, 16, 16, None, 1, None) == zr.ZR_ERR_INVALID_ARG
+        assert L.zr_step_no_alloc(h, zr._ptr_array([16, 8]), 16, 16, 16, 16, None, 1, None) == zr.ZR_ERR_ALIGNMENT
+        assert L.zr_plan_set_gather_targets(None, None, None) == zr.ZR_ERR_INVALID_ARG
+        assert L.zr_plan_set_gather_targets(h, g, None) == zr.ZR_ERR_NO_WORKSPACE
+        assert L.zr_plan_owner_offsets(h, None) == zr.ZR_ERR_INVALID_ARG
+        assert L.zr_ipc_export(None, None) == zr.ZR_ERR_INVALID_ARG
+        assert L.zr_ipc_open(None, None) == zr.ZR_ERR_INVALID_ARG
+        bad = zr.zr_ipc_handle()
+        bad.offset, bad.allocation_bytes = 10, 10                # offset outside the allocation
+        out = ctypes.c_void_p()
+        assert L.zr_ipc_open(ctypes.byref(bad), ctypes.byref(out)) == zr.ZR_ERR_INVALID_ARG
+        assert L.zr_ipc_close(None) == zr.ZR_ERR_INVALID_ARG
+        assert L.zr_state_save(None, b"x", 16, 16, 16, 1, None) == zr.ZR_ERR_INVALID_ARG
+        assert L.zr_state_load(h, None, 16, 16, 16, None, None) == zr.ZR_ERR_INVALID_ARG
+        assert L.zr_state_reshard(h, None, 0, b"x") == zr.ZR_ERR_INVALID_ARG
+        assert L.zr_state_export_params(h, None, 1, 1, b"x", None) == zr.ZR_ERR_INVALID_ARG
+    finally:
+        zr.zr_plan_destroy(h)
