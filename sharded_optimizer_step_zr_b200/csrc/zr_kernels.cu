@@ -306,22 +306,19 @@ zr_clip_combine_kernel(const double* __restrict__ tile_partials, int32_t n_tiles
     __shared__ double part[1024];
     // Thread t adds partials t, t + B, t + 2B, ... in that order (B = block
     // size); the loads of 16 of them are issued before their additions so
-    // the block is not bound by one memory round trip per partial.  Past
-    // the last partial a batch adds +0.0, which leaves the (non-negative)
-    // sum unchanged, so a short tail costs one round trip too.
+    // the block is not bound by one memory round trip per partial.
     constexpr int kBatch = 16;
-    const int64_t B = blockDim.x;
+    const int32_t B = static_cast<int32_t>(blockDim.x);
     double x = 0.0;
-    for (int64_t i = threadIdx.x; i < n_tiles; i += kBatch * B) {
+    int32_t i = threadIdx.x;
+    for (; i + (kBatch - 1) * B < n_tiles; i += kBatch * B) {
         double v[kBatch];
 #pragma unroll
-        for (int k = 0; k < kBatch; ++k) {
-            const int64_t j = i + k * B;
-            v[k] = j < n_tiles ? tile_partials[j] : 0.0;
-        }
+        for (int k = 0; k < kBatch; ++k) v[k] = tile_partials[i + k * B];
 #pragma unroll
         for (int k = 0; k < kBatch; ++k) x += v[k];
     }
+    for (; i < n_tiles; i += B) x += tile_partials[i];
     part[threadIdx.x] = x;
     __syncthreads();
     for (int stride = blockDim.x / 2; stride >= 1; stride >>= 1) {
