@@ -24,6 +24,9 @@ from . import ZR_PARTITION_FLAT, ZR_PARTITION_WHOLE_TENSOR
 
 
 class ZeroAdamW:
+    """ZeRO stage 1/2 AdamW with a torch-optimizer interface (see the module
+    docstring): step(), zero_grad(), set_lr(), save() / load(), close()."""
+
     def __init__(self, params, group=None, lr=3e-4, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.1,
                  max_grad_norm=0.0, partition="flat", bucket_cap_mb=25):
         import torch
@@ -104,6 +107,7 @@ class ZeroAdamW:
             p.grad.zero_()
 
     def set_lr(self, lr):
+        """The learning rate for the following steps (a schedule)."""
         self.hp["lr"] = lr
         self.plan.set_adamw(*self.hp.values())
 
@@ -328,11 +332,13 @@ class Zero3:
         return hook
 
     def zero_grad(self, set_to_none=False):
+        """Zeroes the gradient buffer (the .grad views stay bound)."""
         self.grad_buffer.zero_()
         for p, _ in self._copy_in:
             p.grad.zero_()
 
     def set_lr(self, lr):
+        """The learning rate for the following steps (a schedule)."""
         self.hp["lr"] = lr
         self.plan.set_adamw(*self.hp.values())
 

@@ -41,6 +41,12 @@ def sync_point(dist, group, phase, step):
 
 
 class PeerZero:
+    """One rank of a ZeRO job across processes (one per GPU) over CUDA IPC:
+    the shared gradient buffer (owner-major), and either every rank's full
+    parameter buffer (stages 1, 2: the step's stores are the all-gather) or
+    this rank's parameter shard (stage 3: gather() assembles layers).
+    Every rank constructs it, steps and closes it together."""
+
     def __init__(self, group, shapes, mode=ZR_PARTITION_FLAT, bucket_cap_bytes=25 << 20, lr=3e-4,
                  beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.1, max_grad_norm=0.0, device=None,
                  stage=2):
@@ -155,6 +161,8 @@ class PeerZero:
         return self.plan.bound_gather(first_tensor, n_tensors, self.shard_ptrs, dst, stream, max_ctas)
 
     def close(self):
+        """Unmaps the peers' buffers (after a barrier: no rank still reads
+        them) and destroys the plan."""
         if self._opened:
             self.dist.barrier(self.group)
             for addr in self._opened:

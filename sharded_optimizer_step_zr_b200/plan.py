@@ -44,6 +44,12 @@ def _require_all(specs, device):
 
 
 class ZrPlan:
+    """One rank's plan (zr_plan_create) with a torch-allocated device
+    workspace (bound at construction unless bind=False) and, with clipping,
+    the W-entry partials array.  Tensor arguments of the step calls are
+    checked against the plan before their addresses reach the library;
+    plain integers pass through as raw addresses."""
+
     def __init__(self, shapes, world_size, rank, mode=ZR_PARTITION_FLAT, bucket_cap_bytes=25 << 20,
                  lr=3e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.1, max_grad_norm=0.0,
                  device=None, stream=None, bind=True):
@@ -67,6 +73,8 @@ class ZrPlan:
             self.bind(device, stream)
 
     def bind(self, device=None, stream=None):
+        """Allocates the workspace on `device` and binds it (tables uploaded
+        on `stream`); with clipping, also the partials array."""
         import torch
         device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
         device = torch.device(device)
@@ -81,6 +89,7 @@ class ZrPlan:
             zr_plan_set_sumsq_partials(self.handle, self.partials)
 
     def segments(self):
+        """All ranks' segments as dictionaries (zr_plan_segments)."""
         return zr_plan_segments(self.handle)
 
     def runs(self):
@@ -117,6 +126,8 @@ class ZrPlan:
         return self.owned_numel if self.param_layout == ZR_PARAMS_OWNED else self.padded_numel
 
     def set_param_layout(self, layout, stream=None):
+        """ZR_PARAMS_GLOBAL (param_out: the full buffer) or ZR_PARAMS_OWNED
+        (param_out: this rank's shard, owned order)."""
         zr_plan_set_param_layout(self.handle, layout, stream)
         self.param_layout = layout
 
@@ -143,14 +154,17 @@ class ZrPlan:
         zr_gather_params(self.handle, first_tensor, n_tensors, shards, dst, stream, max_ctas)
 
     def step(self, grads, master, m, v, param_out, step, stream=None):
+        """zr_step: the whole step for this rank, asynchronous on `stream`."""
         self.check_step_buffers(grads, master, m, v, param_out)
         zr_step(self.handle, grads, master, m, v, param_out, step, stream)
 
     def step_bucket(self, bucket, grads, master, m, v, param_out, step, stream=None):
+        """zr_step_bucket: this rank's part of one bucket."""
         self.check_step_buffers(grads, master, m, v, param_out)
         zr_step_bucket(self.handle, bucket, grads, master, m, v, param_out, step, stream)
 
     def step_finish(self, grads, master, m, v, param_out, step, stream=None):
+        """zr_step_finish: the clip's second half after every bucket."""
         self.check_step_buffers(grads, master, m, v, param_out)
         zr_step_finish(self.handle, grads, master, m, v, param_out, step, stream)
 
@@ -173,6 +187,7 @@ class ZrPlan:
 
     def step_host(self, host_grads, dev_grads, master, m, v, param_out, host_param_out, step,
                   stream=None):
+        """zr_step_host: gradients from host memory, the result copied back."""
         import torch
         specs = self._step_specs(dev_grads, master, m, v, param_out)
         if self.owned_numel > 0:
@@ -186,12 +201,14 @@ class ZrPlan:
                      step, stream)
 
     def grad_sumsq(self, grads, out, stream=None):
+        """zr_grad_sumsq: this rank's sum of squares into out[0] (fp64)."""
         import torch
         specs = [(g, f"grads[{w}]", torch.bfloat16, self.owned_numel, False) for w, g in enumerate(grads)]
         _require_all(specs + [(out, "out", torch.float64, 1, False)], self.device)
         zr_grad_sumsq(self.handle, grads, out, stream)
 
     def debug_reduce(self, grads, g_out, stream=None):
+        """zr_debug_reduce: the averaged fp32 gradient, owned order."""
         import torch
         specs = [(g, f"grads[{w}]", torch.bfloat16, self.owned_numel, False) for w, g in enumerate(grads)]
         _require_all(specs + [(g_out, "g_out", torch.float32, self.owned_numel, False)], self.device)
@@ -203,15 +220,19 @@ class ZrPlan:
         self.max_grad_norm = max_grad_norm
 
     def set_checked(self, enable=True):
+        """Checked mode: verify the device tables before every launch."""
         zr_plan_set_checked(self.handle, enable)
 
     def verify(self, stream=None):
+        """zr_plan_verify: one verification of the device tables now."""
         zr_plan_verify(self.handle, stream)
 
     def check_result(self, stream=None):
+        """zr_plan_check_result: the checked-mode status (synchronises)."""
         return zr_plan_check_result(self.handle, stream)
 
     def close(self):
+        """Destroys the plan (the workspace tensor is freed with this object)."""
         if self.handle:
             zr_plan_destroy(self.handle)
             self.handle = 0
