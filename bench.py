@@ -62,6 +62,8 @@ def parse():
                          "after it, against zr_step_bucket as each bucket's gradients complete")
     ap.add_argument("--zero3", action="store_true",
                     help="ZeRO-3 parameter gather: bandwidth, and prefetch against an emulated forward")
+    ap.add_argument("--plan-info", action="store_true",
+                    help="the workload's plan and per-rank device footprint (host only, no GPU)")
     ap.add_argument("--vs-torch", action="store_true",
                     help="the optimizer step against torch's fused AdamW mixed-precision recipe (context)")
     ap.add_argument("--zero3-train", action="store_true",
@@ -972,8 +974,30 @@ def run_vs_torch(args):
     z.close()
 
 
+def plan_info(name):
+    """A workload's plan and this rank's device footprint, host only (no
+    GPU): element counts, buckets, tiles, the workspace and the buffers the
+    step reads and writes."""
+    from sharded_optimizer_step_zr_b200.plan import ZrPlan
+    wl = workload(name)
+    plan = ZrPlan(wl.shapes, wl.world_size, wl.ranks[0], wl.mode, wl.bucket_cap_bytes, *wl.hp, bind=False)
+    n, W = plan.owned_numel, wl.world_size
+    info = {"workload": wl.name, "W": W, "rank": wl.ranks[0], "partition": "flat" if wl.mode == 0 else "whole_tensor",
+            "tensors": len(wl.shapes), "total_numel": plan.total_numel, "padded_numel": plan.padded_numel,
+            "owned_numel": n, "buckets": plan.n_buckets, "segments": len(plan.segments()),
+            "bytes": {"gradients": 2 * W * n, "master_m_v": 12 * n, "param_out": 2 * plan.padded_numel,
+                      "workspace": plan.workspace_bytes},
+            "bytes_per_owned_param": bytes_per_owned_param(W, wl.max_grad_norm > 0)}
+    info["bytes"]["total"] = sum(info["bytes"].values())
+    plan.close()
+    return info
+
+
 def main():
     args = parse()
+    if args.plan_info:
+        print(json.dumps(plan_info(args.config)), flush=True)
+        return
     if args.vs_torch:
         run_vs_torch(args)
         return

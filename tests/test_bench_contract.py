@@ -130,3 +130,18 @@ def test_reference_arm_other_ranks_exit_quietly():
                          cwd=ROOT, env=env)
     assert out.returncode == 0, out.stderr[-2000:]
     assert out.stdout.strip() == ""
+
+
+def test_plan_info_footprints():
+    """--plan-info on the host: the footprints stated for the GPT-2 and
+    Llama-7B workloads (249 MB of gradients and 187 MB of state at W = 8;
+    about 28 GB in all at W = 64)."""
+    g = bench.plan_info("gpt2_124m_w8")
+    assert g["owned_numel"] == 15554976 and g["bytes"]["gradients"] == 248879616
+    assert g["bytes"]["master_m_v"] == 186659712 and g["bytes_per_owned_param"] == 42
+    ll = bench.plan_info("llama_7b_w64")
+    assert ll["owned_numel"] == 105287744 and ll["total_numel"] == 6738415616
+    assert 27e9 < ll["bytes"]["total"] < 29e9
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--plan-info", "--config", "tiny"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 0 and json.loads(out.stdout)["total_numel"] == 1441792
