@@ -269,6 +269,7 @@ class Zero3:
             self._hooks.append(mod.register_forward_pre_hook(self._make_forward_hook(u)))
             self._hooks.append(mod.register_full_backward_pre_hook(self._make_backward_hook(u)))
         self._shard_ptrs, self._slot_of = shard_ptrs, [self.slots[u % 2] for u in range(len(self.units))]
+        self._bound_gathers = {}
         self._prefetched = [False] * len(self.units)
         self.back_ready = [torch.cuda.Event() for _ in self.units]
         self._back_prefetched = [False] * len(self.units)
@@ -291,9 +292,13 @@ class Zero3:
         self.step_count = 0
 
     def _gather(self, u, stream):
-        import torch
-        _, a, k = self.units[u]
-        self.plan.gather_params(a, k, self._shard_ptrs, self._slot_of[u], stream)
+        # one bound call per (unit, stream): the arguments are marshalled once
+        key = (u, stream.cuda_stream)
+        fn = self._bound_gathers.get(key)
+        if fn is None:
+            _, a, k = self.units[u]
+            fn = self._bound_gathers[key] = self.plan.bound_gather(a, k, self._shard_ptrs, self._slot_of[u], stream)
+        fn()
 
     def _make_forward_hook(self, u):
         def hook(module, inputs):
