@@ -177,7 +177,13 @@ zr_status zr_plan_set_device_lr(zr_plan* plan, const float* d_lr);
  * ranks' S_w (from zr_grad_sumsq, or from a scalar all-gather across GPUs)
  * before zr_step runs on the stream.  The clip norm is
  * sqrt(S_0 + S_1 + ... + S_{W-1}), summed in rank order in fp64, so every
- * rank derives the same coefficient. */
+ * rank derives the same coefficient.
+ * This array takes the place of a single pre-summed "other ranks' S"
+ * scalar (a zr_plan_set_peer_sumsq(plan, d_peer_sumsq) form): with one such
+ * scalar each rank would add its own S_r at a different position of the
+ * sum, fp64 addition is not associative, and the ranks could clip by
+ * coefficients that differ in the last bit.  With all W entries in one
+ * array every rank forms the identical sum. */
 zr_status zr_plan_set_sumsq_partials(zr_plan* plan, double* d_partials);
 
 /* The optimizer step for this rank (stages 1-4 above).
