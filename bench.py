@@ -1,7 +1,7 @@
 """Benchmark of the fused ZeRO-1/2 sharded optimizer step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl zr|reference]
-                    [--config NAME] [--no-cpu-baseline]
+                    [--config NAME] [--no-cpu-baseline] [--no-companions]
 
 One step = one zr_step() call on one rank's owned shard: the W-replica bf16
 gradient reduce, (the global-norm clip when the workload has it), AdamW on
@@ -9,9 +9,19 @@ the fp32 master / m / v, and the bf16 write into the all-gather buffer.
 Inputs are seeded synthetic data resident in HBM before the timed region;
 each step's bytes exceed the 126 MB L2, so no flush is needed between steps.
 
+The headline is the Llama-7B-shaped shard at W = 64 (105 M owned params,
+154 B each); the GPT-2-small flat W = 8 shard and the 1.3B whole-tensor
+clipped W = 8 shard are timed after it in the same run, each reported in
+`per_config` with its own roofline, clocks and CPU baseline.
+
 N > 1 (torchrun, one process per GPU): process i runs ZeRO rank (r0 + i) mod
-W of the same workload (r0: the workload's timed rank) on its own GPU -- independent shards, no data-path
-collective (weak scaling); the step time is the max over processes.
+W of the same workloads (r0: the workload's timed rank) on its own GPU --
+independent shards, no data-path collective (weak scaling); the step time is
+the max over processes.  The same run then times the real ZeRO step across
+the processes (`peer`): W = N ranks of the workload's parameter set, each
+reading its slice of every replica's gradient through peer loads and storing
+its bf16 results into every rank's parameter buffer, beside NCCL's
+reduce-scatter + local step + all-gather on the same parameters.
 
 --impl reference times the oracle (plain C on the host, unchanged) on a
 bounded sample of the same workload, split into disjoint slices stepped by
@@ -37,7 +47,9 @@ if ROOT not in sys.path:
 
 METRIC = "owned Gparams/s of fused reduce+AdamW step; achieved HBM GB/s vs B200 peak"
 UNIT = "Gparams/s"
-DEFAULT_CONFIG = "gpt2_124m_w8"
+DEFAULT_CONFIG = "llama_7b_w64"
+# timed in the same run after the headline workload, each with its own roofline, clocks and CPU baseline
+COMPANIONS = ("gpt2_124m_w8", "gpt_1p3b_w8_whole_clip")
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCE = os.path.join(ROOT, "sharded_optimizer_step_zr_b200", "csrc", "zr_kernels.cu")
 PROFILES = os.path.join(ROOT, "profiles")
@@ -74,6 +86,17 @@ def parse():
                     help="checked mode: the device tile tables verified before every launch")
     ap.add_argument("--sweep", action="store_true",
                     help="1.3B set: bucket cap x W x partition; one JSON record per point")
+    ap.add_argument("--no-companions", action="store_true",
+                    help="time the --config workload alone (no per_config entries)")
+    ap.add_argument("--no-peer", action="store_true",
+                    help="N > 1: skip the ZeRO step across the processes over peer memory")
+    ap.add_argument("--peer-set", default=None, choices=sorted(__import__("synth").PARAM_SETS),
+                    help="parameter set of the N > 1 peer step (default: the --config workload's)")
+    ap.add_argument("--peer-steps", type=int, default=20, help="timed steps of the N > 1 peer step")
+    ap.add_argument("--backend", default="nccl", choices=["nccl", "gloo"],
+                    help="process-group backend for N > 1 (gloo: tests of several processes on one GPU)")
+    ap.add_argument("--same-gpu", action="store_true",
+                    help="N > 1: every process on cuda:0 (a test on a one-GPU machine)")
     args = ap.parse_args()
     if args.cpu_threads <= 0:
         args.cpu_threads = host_threads()
@@ -136,22 +159,31 @@ def kernel_source_hash():
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def recorded_traffic(workload_name, clip):
+def recorded_traffic(workload_name, clip, owned_params):
     """dram__bytes_read.sum + dram__bytes_write.sum from the committed ncu
-    record of the workload, if it was taken on the current kernel source,
-    else None: per launch of zr_tile_kernel for a step without clipping, per
-    step (its three launches) with clipping -- the same unit as the line's
-    `achieved`."""
+    record of the workload, if it was taken on the current kernel source:
+    per launch of zr_tile_kernel for a step without clipping, per step (all
+    of its launches) with clipping -- the same unit as the line's
+    `achieved`.  A record taken on a smaller case of the same kernels gives
+    bytes per owned parameter, scaled here to `owned_params`.  Returns
+    (bytes or None, a note on where they come from)."""
     name = f"zr_clip_step_{workload_name}" if clip else f"zr_tile_kernel_{workload_name}"
     try:
         with open(os.path.join(PROFILES, f"{name}_traffic.json")) as f:
             d = json.load(f)
-        e = d.get(workload_name)
-        if e and e.get("kernel_source_sha256_16") == kernel_source_hash():
-            return float(e["bytes_per_step"] if clip else e["bytes_per_launch"])
-    except Exception:
-        pass
-    return None
+    except (OSError, ValueError):
+        return None, "no ncu record for this workload"
+    e = d.get(workload_name)
+    if not e:
+        return None, "no ncu record for this workload"
+    if e.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None, "ncu record taken on an older kernel source"
+    if "bytes_per_owned_param" in e:
+        small = e["small_case"]
+        return (float(e["bytes_per_owned_param"]) * owned_params,
+                f"ncu capture of {small['workload']} ({small['owned_params']} owned params), "
+                f"scaled by owned params")
+    return float(e["bytes_per_step"] if clip else e["bytes_per_launch"]), "ncu capture of this workload"
 
 
 class ClockSampler:
@@ -393,27 +425,66 @@ def bound_bucket_steps(plan, buckets, grads, master, m, v, param_out, stream):
     return step_fn
 
 
-def run_zr(args):
+class ProcessContext:
+    """This process's place in the run: the process group (None for one
+    process), its ranks and its device."""
+
+    def __init__(self, args, use_cuda=True):
+        import torch
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.grank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.dist = None
+        self.backend = None
+        if use_cuda:
+            # --same-gpu: every process on cuda:0 (a multi-process test on a
+            # one-GPU machine; the kernels never wait on another process)
+            torch.cuda.set_device(0 if (self.world == 1 or args.same_gpu) else self.local)
+            self.dev = torch.device("cuda", torch.cuda.current_device())
+        else:
+            self.dev = torch.device("cpu")     # host-side logic only (gloo tests)
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            self.backend = args.backend
+            kw = {"device_id": self.dev} if (self.backend == "nccl" and use_cuda) else {}
+            dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=120), **kw)
+            self.dist = dist
+
+    def barrier(self):
+        if self.dist is not None:
+            if self.backend == "nccl":
+                self.dist.barrier(device_ids=[self.dev.index])
+            else:
+                self.dist.barrier()
+
+    def reduce(self, elapsed_ms, owned_done):
+        """(max of elapsed_ms, sum of owned_done) over the processes."""
+        if self.dist is None:
+            return elapsed_ms, owned_done
+        import torch
+        d = self.dev if self.backend == "nccl" else torch.device("cpu")
+        return reduce_timing(self.dist, elapsed_ms, owned_done, d)
+
+    def close(self):
+        if self.dist is not None:
+            self.barrier()
+            self.dist.destroy_process_group()
+
+
+def measure_local(args, ctx, wl, with_e2e, with_cpu):
+    """K timed steps of workload `wl` on this process's shard (ZeRO rank
+    shard_rank(wl, ...)): the step time (max over processes), the roofline
+    of the step's kernels, the clocks, and optionally the end-to-end rate
+    through zr_step_host and the oracle's CPU rate.  Returns the entry as
+    rank 0 reports it (identical keys on every process)."""
     import torch
     import synth
     from sharded_optimizer_step_zr_b200.plan import ZrPlan
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    grank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    else:
-        torch.cuda.set_device(0)
-    dev = torch.device("cuda", torch.cuda.current_device())
-
-    wl = workload(args.config)
+    dev = ctx.dev
     W = wl.world_size
-    zr_rank = shard_rank(wl, grank, world)
+    zr_rank = shard_rank(wl, ctx.grank, ctx.world)
     clip = wl.max_grad_norm > 0
     plan = ZrPlan(wl.shapes, W, zr_rank, wl.mode, wl.bucket_cap_bytes, *wl.hp, device=dev)
     n = plan.owned_numel
@@ -452,8 +523,7 @@ def run_zr(args):
 
     K = args.steps
     sampler = ClockSampler(dev.index)
-    if dist:
-        dist.barrier(device_ids=[local])
+    ctx.barrier()
     torch.cuda.synchronize()
     with sampler:
         t_start = torch.cuda.Event(enable_timing=True)
@@ -464,27 +534,52 @@ def run_zr(args):
             run_step(step_no)
         t_end.record(stream)
         torch.cuda.synchronize()
-    if dist:
-        dist.barrier(device_ids=[local])
+    ctx.barrier()
     local_ms = t_start.elapsed_time(t_end)
-    total_ms, owned_total = reduce_timing(dist, local_ms, n * K, dev)
+    total_ms, owned_total = ctx.reduce(local_ms, n * K)
     value = owned_total / (total_ms * 1e-3) / 1e9
     ms_per_step = total_ms / K
 
     # roofline: without clipping the step is one launch of zr_tile_kernel, so
     # its average launch duration is this process's timed region / K; with
-    # clipping the three launches of the step are taken together.
+    # clipping the step's launches are taken together.
     bpp = bytes_per_owned_param(W, clip)
     alg_bytes = n * bpp
     avg_ms = local_ms / K
     achieved = alg_bytes / (avg_ms * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
     # (bucket-by-bucket or checked steps launch more kernels: no per-launch record)
-    traffic = None if (args.per_bucket or args.checked) else recorded_traffic(wl.name, clip)
+    traffic = None
+    traffic_note = None
+    if not (args.per_bucket or args.checked):
+        traffic, traffic_note = recorded_traffic(wl.name, clip, n)
+
+    # the ceiling at this size: a plain device copy (torch) moving the step's
+    # algorithmic bytes (half read, half written), timed the same way
+    copy_ref = None
+    if not (args.per_bucket or args.checked):
+        half = (alg_bytes // 2) // 16 * 16
+        src = torch.empty(half, dtype=torch.uint8, device=dev)
+        dst = torch.empty(half, dtype=torch.uint8, device=dev)
+        reps = max(3, min(K, 200))
+        for _ in range(3):
+            dst.copy_(src)
+        torch.cuda.synchronize()
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(reps):
+            dst.copy_(src)
+        c1.record(stream)
+        torch.cuda.synchronize()
+        copy_ms = c0.elapsed_time(c1) / reps
+        copy_ref = {"bytes": 2 * half, "ms": copy_ms, "gbs": 2 * half / (copy_ms * 1e-3) / 1e9, "reps": reps,
+                    "step_speed_vs_copy": copy_ms / avg_ms}
+        del src, dst
+        torch.cuda.empty_cache()
 
     # end to end through zr_step_host: pinned host gradients in, result out
     e2e = None
-    if not args.no_e2e:
+    if with_e2e:
         host_grads = [g.cpu().pin_memory() for g in grads]
         host_out = torch.empty(plan.padded_numel, dtype=torch.bfloat16).pin_memory()
         for _ in range(3):
@@ -493,8 +588,7 @@ def run_zr(args):
         torch.cuda.synchronize()
         K2 = max(3, min(K, 50))
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if dist:
-            dist.barrier(device_ids=[local])
+        ctx.barrier()
         torch.cuda.synchronize()
         a.record(stream)
         for _ in range(K2):
@@ -502,29 +596,24 @@ def run_zr(args):
             plan.step_host(host_grads, grads, master, m, v, param_out, host_out, step_no, stream)
         b.record(stream)
         torch.cuda.synchronize()
-        e2e_ms, e2e_owned = reduce_timing(dist, a.elapsed_time(b), n * K2, dev)
+        e2e_ms, e2e_owned = ctx.reduce(a.elapsed_time(b), n * K2)
         e2e = {"value": e2e_owned / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
                "h2d_bytes_per_step": 2 * W * n, "d2h_bytes_per_step": 2 * n,
                "steps": K2, "api": "zr_step_host"}
+        del host_grads, host_out
 
     cpu = None
-    if grank == 0 and world == 1 and not args.no_cpu_baseline:
+    if with_cpu and ctx.grank == 0 and ctx.world == 1:
         cpu = cpu_baseline(wl, zr_rank, args.cpu_seconds, args.cpu_threads)
 
-    if dist:
-        dist.barrier(device_ids=[local])
-        dist.destroy_process_group()
-    if grank != 0:
-        return
-    launches_per_step = 3 if clip else 1
+    launches_per_step = launches_per_clip_step() if clip else 1
     if args.per_bucket:
+        # pass 1 per bucket with clipping; zr_step_finish: the coefficient, then pass 2
         launches_per_step = len(my_buckets) + (2 if clip else 0)
     if args.checked:
         launches_per_step += (len(my_buckets) + (1 if clip else 0)) if args.per_bucket else 1
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+    entry = {
+        "workload": wl.name, "value": value, "unit": UNIT, "ms_per_step": ms_per_step, "steps": K,
         "config": {"workload": wl.name, "W": W, "rank": zr_rank,
                    "partition": "flat" if wl.mode == 0 else "whole_tensor",
                    "bucket_cap_mb": wl.bucket_cap_mb, "clip": clip, "owned_params": n,
@@ -534,13 +623,173 @@ def run_zr(args):
                    "l2": f"no flush: each step touches {alg_bytes / 1e6:.0f} MB > 126 MB L2"},
         "hbm_gbs": achieved,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
-                     "kernel": "zr_tile_kernel" if not clip else "zr_step (3 kernels)"},
+                     "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_note,
+                     "peak_source": peak_kind,
+                     "kernel": "zr_tile_kernel" if not clip else
+                     f"zr_step ({launches_per_clip_step()} kernels)"},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches_per_step * K,
         "clocks": sampler.summary(),
+        "copy_reference": copy_ref,
     }
+    plan.close()
+    del grads, master, m, v, param_out, run_step
+    torch.cuda.empty_cache()
+    return entry
+
+
+def launches_per_clip_step():
+    """Kernel launches of one clipped zr_step: pass 1 (which also forms the
+    coefficient) and pass 2."""
+    return 2
+
+
+def peer_bytes(W, n):
+    """Bytes one rank of a W-rank peer-memory step moves per step for its
+    n owned parameters: gradient loads from the W - 1 peers' replicas (the
+    reduce-scatter), bf16 stores into the W - 1 peers' parameter buffers
+    (the all-gather), and its local HBM traffic (own replica, fp32 state
+    read and written, own parameter buffer)."""
+    return {"peer_loads": 2 * (W - 1) * n, "peer_stores": 2 * (W - 1) * n,
+            "local_hbm": 2 * n + 24 * n + 2 * n}
+
+
+def measure_peer(args, ctx):
+    """The ZeRO step across the processes of this run (one rank each, W =
+    the number of processes): PeerZero over CUDA IPC, the step reading every
+    replica's slice through peer loads and storing the bf16 results into
+    every rank's parameter buffer.  Beside it, on the same parameters, the
+    library-collective recipe: NCCL reduce-scatter (average) of the bf16
+    gradients, the local step on the owned chunk (one replica), NCCL
+    all-gather of the bf16 chunk.  Returns the entry (identical keys on
+    every process)."""
+    import torch
+    import synth
+    from sharded_optimizer_step_zr_b200.peer import PeerZero
+    from sharded_optimizer_step_zr_b200.plan import ZrPlan
+
+    wl = workload(args.config)
+    set_name = args.peer_set or wl.param_set
+    shapes = synth.PARAM_SETS[set_name]()
+    W, rank, dev = ctx.world, ctx.grank, ctx.dev
+    hp = wl.hp[:5] + (0.0,)
+    pz = PeerZero(ctx.dist.group.WORLD, shapes, 0, wl.bucket_cap_bytes, *hp, device=dev, stage=2)
+    n = pz.plan.owned_numel
+    N = pz.plan.total_numel
+    segs = pz.plan.segments()
+    runs_of = [synth.rank_runs(segs, r) for r in range(W)]
+    # this process is replica `rank`: its full gradient in the owner-major layout
+    for r in range(W):
+        a, b = pz.offsets[r], pz.offsets[r + 1]
+        synth.fill_owned_grad(pz.grad_buffer[a:b], runs_of[r], wl.seed, 1, rank, wl.grad_sigma,
+                              wl.outlier_frac, n_valid=N)
+    master = torch.empty(max(n, 8), dtype=torch.float32, device=dev)
+    synth.fill_owned_master(master, runs_of[rank], wl.seed, n_valid=N)
+    m, v = torch.zeros_like(master), torch.zeros_like(master)
+    stream = torch.cuda.current_stream()
+    t = 0
+    for _ in range(args.warmup):
+        t += 1
+        pz.step(master, m, v, t)
+    K = max(1, args.peer_steps)
+    ctx.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        t += 1
+        pz.step(master, m, v, t)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms, owned = ctx.reduce(e0.elapsed_time(e1), n * K)
+    entry = {"mode": "peer", "W": W, "param_set": set_name, "partition": "flat",
+             "bucket_cap_mb": wl.bucket_cap_mb, "total_params": N, "owned_params": n,
+             "steps": K, "ms_per_step": ms / K, "value": owned / (ms * 1e-3) / 1e9, "unit": UNIT,
+             "per_gpu_value": n / (ms / K * 1e-3) / 1e9,
+             "bytes_per_step_per_rank": peer_bytes(W, n),
+             "same_gpu": bool(args.same_gpu), "backend": ctx.backend,
+             "timing": "CUDA events over K steps, host barriers between the phases included; max over ranks"}
+
+    # the library-collective arm (flat partitions whose owner-major layout is the global one)
+    C = pz.plan.padded_numel // W
+    aligned = all(pz.offsets[r] == r * C for r in range(W + 1))
+    if ctx.backend != "nccl" or args.same_gpu:
+        entry["nccl_arm"] = {"skipped": "needs NCCL with one GPU per process"}
+    elif not aligned:
+        entry["nccl_arm"] = {"skipped": "owner-major layout differs from the global layout"}
+    else:
+        dist = ctx.dist
+        full_grad = pz.grad_buffer[:W * C]
+        shard_grad = torch.empty(C, dtype=torch.bfloat16, device=dev)
+        shard_out = torch.empty(C, dtype=torch.bfloat16, device=dev)
+        full_param = torch.empty(W * C, dtype=torch.bfloat16, device=dev)
+        one = ZrPlan([(C,)], 1, 0, 0, 1 << 40, *hp, device=dev)
+        mb = master[:n].clone() if C == n else torch.zeros(C, dtype=torch.float32, device=dev)
+        mmb, vvb = torch.zeros_like(mb), torch.zeros_like(mb)
+        local_step = one.bound_step([shard_grad], mb, mmb, vvb, shard_out, stream)
+
+        def nccl_step(tt):
+            dist.reduce_scatter_tensor(shard_grad, full_grad, op=dist.ReduceOp.AVG)
+            local_step(tt)
+            dist.all_gather_into_tensor(full_param, shard_out)
+
+        tt = 0
+        for _ in range(args.warmup):
+            tt += 1
+            nccl_step(tt)
+        ctx.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(K):
+            tt += 1
+            nccl_step(tt)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms2, owned2 = ctx.reduce(e0.elapsed_time(e1), C * K)
+        entry["nccl_arm"] = {"ms_per_step": ms2 / K, "value": owned2 / (ms2 * 1e-3) / 1e9, "unit": UNIT,
+                             "recipe": "reduce_scatter_tensor(bf16, AVG) + zr_step on the chunk (W = 1) "
+                                       "+ all_gather_into_tensor(bf16)"}
+        one.close()
+        del full_grad, shard_grad, shard_out, full_param, mb, mmb, vvb, local_step
+    pz.close()
+    del master, m, v
+    torch.cuda.empty_cache()
+    return entry
+
+
+def run_zr(args):
+    ctx = ProcessContext(args)
+    head = measure_local(args, ctx, workload(args.config), with_e2e=not args.no_e2e,
+                         with_cpu=not args.no_cpu_baseline)
+    per_config = []
+    if not (args.no_companions or args.per_bucket or args.checked):
+        for name in COMPANIONS:
+            if name != args.config:
+                per_config.append(measure_local(args, ctx, workload(name), with_e2e=False,
+                                                with_cpu=not args.no_cpu_baseline))
+    peer = None
+    if ctx.world > 1 and not args.no_peer:
+        peer = measure_peer(args, ctx)
+    ctx.close()
+    if ctx.grank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": ctx.world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": head["config"],
+        "hbm_gbs": head["hbm_gbs"],
+        "roofline": head["roofline"],
+        "cpu_baseline": head["cpu_baseline"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
+        "copy_reference": head["copy_reference"],
+        "per_config": per_config,
+    }
+    if peer is not None:
+        line["peer"] = peer
     print(json.dumps(line), flush=True)
 
 
@@ -783,6 +1032,41 @@ def run_zero3(args):
     block_us = timed(plan.bound_gather(2, per_block, shards, layer_buf[0]), 200)
     gb = lambda elems, us: 4 * elems / (us * 1e-6) / 1e9
 
+    def graph_us(bind, reps):
+        """Per-launch device time of `reps` launches replayed from one CUDA
+        graph: no host launch gap between them (a 6 us gather issued from
+        Python one call at a time waits on the host)."""
+        s = torch.cuda.Stream()
+        fn = bind(s)
+        with torch.cuda.stream(s):
+            for _ in range(3):
+                fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(reps):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        g.replay()
+        e1.record(s)
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) / reps * 1e3
+
+    # the same bytes moved by a plain device copy (torch), for the ceiling at each size
+    src_block = torch.empty(block_params, dtype=torch.bfloat16, device=dev)
+    src_whole = torch.empty(sum(numels), dtype=torch.bfloat16, device=dev)
+    graph = {
+        "gather_block_us": graph_us(lambda st: plan.bound_gather(2, per_block, shards, layer_buf[0], st), 100),
+        "copy_block_us": graph_us(lambda st: (lambda: layer_buf[1].copy_(src_block)), 100),
+        "gather_whole_model_us": graph_us(lambda st: plan.bound_gather(0, len(numels), shards, full, st), 10),
+        "copy_whole_model_us": graph_us(lambda st: (lambda: full.copy_(src_whole)), 10),
+    }
+    del src_whole
+
     # emulated forward: per block [8192, d] x [d, 12 d] bf16, 2 * 8192 * 12 * d^2 flops -- a
     # block's forward (12 d^2 weights) at 8192 tokens
     x = torch.randn(8192, d_model, dtype=torch.bfloat16, device=dev)
@@ -852,6 +1136,11 @@ def run_zero3(args):
         "exposed_gather_in_line_us": t_seq - t_fwd,
         "exposed_gather_prefetched_us": {k: v - t_fwd for k, v in t_pre.items()},
         "blocks": n_blocks,
+        "graph_replay": dict(graph, **{
+            "frac_block": gb(block_params, graph["gather_block_us"]) / peak,
+            "frac_whole_model": gb(sum(numels), graph["gather_whole_model_us"]) / peak,
+            "gather_over_copy_block": graph["copy_block_us"] / graph["gather_block_us"],
+            "gather_over_copy_whole_model": graph["copy_whole_model_us"] / graph["gather_whole_model_us"]}),
     }
     print(json.dumps(line), flush=True)
     plan.close()

@@ -161,10 +161,11 @@ def gpt2_small_shapes():
     return shapes
 
 
-def gpt_1p3b_shapes():
+def gpt_1p3b_shapes(L=24):
     """GPT-style 1.3B: d=2048, 24 blocks, MLP 8192, vocab 50304, 2048 learned
-    positions, biases and LayerNorm weight/bias, tied head."""
-    d, v, ctx, L, f = 2048, 50304, 2048, 24, 8192
+    positions, biases and LayerNorm weight/bias, tied head.  L < 24 keeps the
+    first L blocks (a smaller case of the same shapes)."""
+    d, v, ctx, f = 2048, 50304, 2048, 8192
     shapes = [(v, d), (ctx, d)]
     for _ in range(L):
         shapes += [(d,), (d,), (d, 3 * d), (3 * d,), (d, d), (d,),
@@ -173,10 +174,11 @@ def gpt_1p3b_shapes():
     return shapes
 
 
-def llama_7b_shapes():
+def llama_7b_shapes(L=32):
     """Llama-7B: untied embedding and head, RMSNorm weights, no biases;
-    each block declares attn_norm, q, k, v, o, mlp_norm, gate, up, down."""
-    d, v, L, f = 4096, 32000, 32, 11008
+    each block declares attn_norm, q, k, v, o, mlp_norm, gate, up, down.
+    L < 32 keeps the first L blocks (a smaller case of the same shapes)."""
+    d, v, f = 4096, 32000, 11008
     shapes = [(v, d)]
     for _ in range(L):
         shapes += [(d,), (d, d), (d, d), (d, d), (d, d), (d,), (f, d), (f, d), (d, f)]
@@ -189,6 +191,9 @@ PARAM_SETS = {
     "gpt2_124m": gpt2_small_shapes,
     "gpt_1p3b": gpt_1p3b_shapes,
     "llama_7b": llama_7b_shapes,
+    # smaller cases of the same shapes, for profiler captures of a few GB
+    "llama_7b_4blk": lambda: llama_7b_shapes(4),
+    "gpt_1p3b_6blk": lambda: gpt_1p3b_shapes(6),
 }
 
 MB = 1 << 20
@@ -244,6 +249,12 @@ WORKLOADS = {
     "gpt2_124m_w64": Workload("gpt2_124m_w64", "gpt2_124m", 64, (0,), 0, 25, 1e-3, 0.0),
     "gpt2_124m_w8_whole_clip": Workload("gpt2_124m_w8_whole_clip", "gpt2_124m", 8, (3,), 1, 25,
                                         1e-3, 0.01, max_grad_norm=1.0),
+    # The same kernels as the Llama-7B W = 64 and the 1.3B clipped workloads on
+    # the first blocks of those sets (about 4.5 and 2.5 GB on the device): the
+    # DRAM counters taken on them are scaled to the full workloads by owned params.
+    "llama_7b_4blk_w64": Workload("llama_7b_4blk_w64", "llama_7b_4blk", 64, (0,), 0, 25, 1e-3, 0.0),
+    "gpt_1p3b_6blk_w8_whole_clip": Workload("gpt_1p3b_6blk_w8_whole_clip", "gpt_1p3b_6blk", 8, (3,), 1, 25,
+                                            1e-3, 0.01, max_grad_norm=1.0),
 }
 
 

@@ -39,3 +39,32 @@ def test_zero3_train_mode_takes_identical_steps():
 def test_vs_torch_mode():
     d = run_mode("--vs-torch")
     assert d["mode"] == "vs_torch_adamw" and d["zr_step_ms"] > 0 and d["torch_fused_adamw_step_ms"] > 0
+
+
+def test_peer_mode_two_processes_one_gpu():
+    """`bench.py --gpus 2` as torchrun launches it, both processes on this
+    machine's one GPU (gloo for the host barriers; the kernels never wait on
+    the other process): the headline line, and the peer step of a W = 2 job
+    whose gradient loads and parameter stores cross into the other
+    process's memory through CUDA IPC.  The NCCL arm needs one GPU per
+    process and reports that it was skipped."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes", "1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--gpus", "2", "--backend", "gloo", "--same-gpu", "--config", "gpt2_124m_w8", "--no-companions",
+           "--no-cpu-baseline", "--no-e2e", "--peer-set", "gpt2_124m", "--steps", "20", "--warmup", "3",
+           "--peer-steps", "5"]
+    out = subprocess.run(["timeout", "-k", "30", "600"] + cmd, capture_output=True, text=True, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-3000:]
+    lines = [l for l in out.stdout.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1, out.stdout[-2000:]
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["config"]["workload"] == "gpt2_124m_w8" and d["value"] > 0
+    p = d["peer"]
+    assert p["W"] == 2 and p["param_set"] == "gpt2_124m" and p["value"] > 0
+    assert p["owned_params"] == 124439808 // 2
+    assert p["bytes_per_step_per_rank"]["peer_loads"] == 2 * p["owned_params"]
+    assert "skipped" in p["nccl_arm"]

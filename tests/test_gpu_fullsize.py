@@ -1,5 +1,7 @@
 """Parity at the workloads' full sizes, in the launch configuration the
-benchmark times (one zr_step through ZrPlan on one rank's whole shard).
+benchmark times (zr_step through ZrPlan on one rank's whole shard), after
+three steps for configs 2-4 and the 25 MB sweep points, after one for the
+other 32 points of the sweep.
 
 The oracle cannot step every element of these shards quickly, but the
 step is elementwise once the clip coefficient is known, so it is checked on
@@ -66,14 +68,20 @@ def host_global_sumsq(oplan, wl, step, threads):
 
 SWEEP = {wl.name: wl for wl in synth.sweep_workloads()}
 
+# Configs 2-4 (and the last rank of config 4, whose offsets pass 2**32), and
+# the 1.3B sweep at the 25 MB cap: three steps, each with fresh gradients,
+# so the checked m and v carry state from the earlier steps.
+THREE_STEP = ([("gpt2_124m_w8", None), ("llama_7b_w64", None), ("llama_7b_w64", 63),
+               ("gpt_1p3b_w8_whole_clip", None)] +
+              [(f"sweep_1p3b_{m}_w{w}_cap25", None) for m in ("flat", "whole") for w in (2, 8, 32, 64)])
+# The rest of the sweep (caps 1, 5, 100 and 400 MB): one step each.
+ONE_STEP = [(f"sweep_1p3b_{m}_w{w}_cap{c}", None) for m in ("flat", "whole") for w in (2, 8, 32, 64)
+            for c in (1, 5, 100, 400)]
 
-@pytest.mark.parametrize("name, rank", [("gpt2_124m_w8", None), ("llama_7b_w64", None),
-                                        ("llama_7b_w64", 63),   # parameter offsets beyond 2**32
-                                        ("gpt_1p3b_w8_whole_clip", None)] +
-                         # the 1.3B sweep: one point per (W, partition) at the 25 MB cap
-                         [(f"sweep_1p3b_{m}_w{w}_cap25", None) for m in ("flat", "whole")
-                          for w in (2, 8, 32, 64)])
-def test_full_size_sampled(name, rank):
+
+@pytest.mark.parametrize("name, rank, steps", [(n, r, 3) for n, r in THREE_STEP] +
+                         [(n, r, 1) for n, r in ONE_STEP])
+def test_full_size_sampled(name, rank, steps):
     wl = synth.WORKLOADS[name] if name in synth.WORKLOADS else SWEEP[name]
     rank = wl.ranks[0] if rank is None else rank
     W = wl.world_size
@@ -81,69 +89,71 @@ def test_full_size_sampled(name, rank):
     plan = ZrPlan(wl.shapes, W, rank, wl.mode, wl.bucket_cap_bytes, *wl.hp, device=DEV)
     n = plan.owned_numel
     runs = plan.runs()
-    step = 1
     grads = [torch.empty(n, dtype=torch.bfloat16, device=DEV) for _ in range(W)]
-    for w in range(W):
-        synth.fill_owned_grad(grads[w], runs, wl.seed, step, w, wl.grad_sigma, wl.outlier_frac,
-                              n_valid=plan.total_numel)
     master = torch.empty(n, dtype=torch.float32, device=DEV)
     synth.fill_owned_master(master, runs, wl.seed, n_valid=plan.total_numel)
     m, v = torch.zeros_like(master), torch.zeros_like(master)
     sentinel = -16447   # 0xBFC1 as int16: a value the step never writes by chance here
     param_out = torch.full((plan.padded_numel,), sentinel, dtype=torch.int16, device=DEV)
+    g_gpu = torch.empty(n, dtype=torch.float32, device=DEV)
 
     oplan = oracle.Plan(wl.shapes, W, wl.mode, wl.bucket_cap_bytes)
-    c = None
-    if clip:
-        # other ranks' S_w on the GPU (zr_grad_sumsq on their own shards)
-        parts_gpu = torch.zeros(W, dtype=torch.float64, device=DEV)
-        for r in range(W):
-            if r == rank:
-                continue
-            pr = ZrPlan(wl.shapes, W, r, wl.mode, wl.bucket_cap_bytes, *wl.hp, device=DEV)
-            rr = pr.runs()
-            gr = [torch.empty(max(pr.owned_numel, 8), dtype=torch.bfloat16, device=DEV) for _ in range(W)]
-            for w in range(W):
-                synth.fill_owned_grad(gr[w], rr, wl.seed, step, w, wl.grad_sigma, wl.outlier_frac,
-                                      n_valid=pr.total_numel)
-            pr.grad_sumsq(gr, parts_gpu[r:r + 1])
-            torch.cuda.synchronize()
-            del gr
-            pr.close()
-            torch.cuda.empty_cache()
-        plan.partials.copy_(parts_gpu)
-        S, parts_host = host_global_sumsq(oplan, wl, step, threads=min(32, os.cpu_count() or 1))
-        c = oracle.clip_coef(S, wl.max_grad_norm)
-
-    g_gpu = torch.empty(n, dtype=torch.float32, device=DEV)
-    plan.debug_reduce(grads, g_gpu)
-    plan.step(grads, master, m, v, param_out.view(torch.bfloat16), step)
-    torch.cuda.synchronize()
-
-    if clip:
-        got_parts = plan.partials.cpu().numpy()
-        for r in range(W):
-            assert abs(got_parts[r] - parts_host[r]) <= 1e-12 * parts_host[r], r
-
     own = sample_owned(runs, n)
     glob = owned_to_global(runs, own)
     assert np.array_equal(glob, oplan.owned_global_index(rank)[own])
     tg = torch.from_numpy(glob)
-    reps = [u16(synth.grad_bf16(wl.seed, step, w, tg, wl.grad_sigma, wl.outlier_frac,
-                                n_valid=oplan.total_numel)) for w in range(W)]
-    g_ref = oracle.reduce(reps)
     own_t = torch.from_numpy(own).to(DEV)
-    assert np.array_equal(bits32(g_gpu[own_t]), bits32(g_ref))
-    g_use = g_ref.copy()
-    if clip:
-        oracle.scale(g_use, c)
     p_ref = synth.master_f32(wl.seed, tg, n_valid=oplan.total_numel).numpy().copy()
     m_ref = np.zeros_like(p_ref)
     v_ref = np.zeros_like(p_ref)
-    oracle.adamw(wl.hp, step, g_use, p_ref, m_ref, v_ref)
-    assert_state_close(master[own_t].cpu().numpy(), p_ref, "master")
-    assert_state_close(m[own_t].cpu().numpy(), m_ref, "m")
-    assert_state_close(v[own_t].cpu().numpy(), v_ref, "v")
+
+    for step in range(1, steps + 1):
+        for w in range(W):
+            synth.fill_owned_grad(grads[w], runs, wl.seed, step, w, wl.grad_sigma, wl.outlier_frac,
+                                  n_valid=plan.total_numel)
+        c = None
+        if clip:
+            # other ranks' S_w for this step on the GPU (zr_grad_sumsq on their own shards)
+            parts_gpu = torch.zeros(W, dtype=torch.float64, device=DEV)
+            for r in range(W):
+                if r == rank:
+                    continue
+                pr = ZrPlan(wl.shapes, W, r, wl.mode, wl.bucket_cap_bytes, *wl.hp, device=DEV)
+                rr = pr.runs()
+                gr = [torch.empty(max(pr.owned_numel, 8), dtype=torch.bfloat16, device=DEV) for _ in range(W)]
+                for w in range(W):
+                    synth.fill_owned_grad(gr[w], rr, wl.seed, step, w, wl.grad_sigma, wl.outlier_frac,
+                                          n_valid=pr.total_numel)
+                pr.grad_sumsq(gr, parts_gpu[r:r + 1])
+                torch.cuda.synchronize()
+                del gr
+                pr.close()
+                torch.cuda.empty_cache()
+            plan.partials.copy_(parts_gpu)
+            S, parts_host = host_global_sumsq(oplan, wl, step, threads=min(32, os.cpu_count() or 1))
+            c = oracle.clip_coef(S, wl.max_grad_norm)
+
+        plan.debug_reduce(grads, g_gpu)
+        plan.step(grads, master, m, v, param_out.view(torch.bfloat16), step)
+        torch.cuda.synchronize()
+
+        if clip:
+            got_parts = plan.partials.cpu().numpy()
+            for r in range(W):
+                assert abs(got_parts[r] - parts_host[r]) <= 1e-12 * parts_host[r], (step, r)
+
+        # the oracle steps the sampled elements from their own host-generated gradients
+        reps = [u16(synth.grad_bf16(wl.seed, step, w, tg, wl.grad_sigma, wl.outlier_frac,
+                                    n_valid=oplan.total_numel)) for w in range(W)]
+        g_ref = oracle.reduce(reps)
+        assert np.array_equal(bits32(g_gpu[own_t]), bits32(g_ref)), f"reduced gradient, step {step}"
+        if clip:
+            oracle.scale(g_ref, c)
+        oracle.adamw(wl.hp, step, g_ref, p_ref, m_ref, v_ref)
+
+    assert_state_close(master[own_t].cpu().numpy(), p_ref, f"master after {steps} steps")
+    assert_state_close(m[own_t].cpu().numpy(), m_ref, f"m after {steps} steps")
+    assert_state_close(v[own_t].cpu().numpy(), v_ref, f"v after {steps} steps")
     out_ref = oracle.f32_to_bf16_array(p_ref)
     got = param_out[tg.to(DEV)].cpu().numpy().view(np.uint16)
     assert bf16_ulp_distance(got, out_ref).max() <= 1
@@ -156,5 +166,5 @@ def test_full_size_sampled(name, rank):
     vals = param_out[torch.from_numpy(probe[~mine]).to(DEV)].cpu().numpy()
     assert np.all(vals == sentinel)
     plan.close()
-    del grads, master, m, v, param_out
+    del grads, master, m, v, param_out, g_gpu
     torch.cuda.empty_cache()

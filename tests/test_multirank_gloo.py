@@ -155,3 +155,56 @@ def test_missing_peer_raises_before_the_next_launch(how):
         p.join(timeout=60)
     assert msg.startswith("step 2, gradients ready: a peer did not arrive"), msg
     assert waited < 30
+
+
+def _bench_ctx_worker(rank, world, port, result_q):
+    import sys
+    sys.path.insert(0, ROOT)
+    import argparse
+    import bench
+    import synth
+    from sharded_optimizer_step_zr_b200.plan import ZrPlan
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    args = argparse.Namespace(backend="gloo", same_gpu=False)
+    ctx = bench.ProcessContext(args, use_cuda=False)
+    try:
+        # the launch logic of `bench.py --gpus N`: each process one rank of
+        # the peer step's W = N job over the workload's parameter set
+        shapes = synth.PARAM_SETS["gpt2_124m"]()
+        plan = ZrPlan(shapes, ctx.world, ctx.grank, 0, 25 << 20, bind=False)
+        n, padded = plan.owned_numel, plan.padded_numel
+        plan.close()
+        moved = bench.peer_bytes(ctx.world, n)
+        ctx.barrier()
+        ms, owned = ctx.reduce(5.0 * (rank + 1), n)
+        result_q.put((rank, ctx.grank, ctx.world, n, padded, moved, ms, owned))
+    finally:
+        ctx.close()
+
+
+def test_bench_process_context_and_peer_accounting():
+    """bench.py's N > 1 plumbing over a real gloo group on the CPU: each
+    process's rank, the peer step's owned slices covering the padded set
+    (flat, W = 2), the bytes each rank moves over peers, and the max / sum
+    reduction of the timings."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bench_ctx_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in range(world):
+        r = q.get(timeout=180)
+        res[r[0]] = r
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [res[r][1] for r in range(world)] == [0, 1] and all(res[r][2] == 2 for r in range(world))
+    n0, padded = res[0][3], res[0][4]
+    assert n0 + res[1][3] == padded == 124439808
+    assert res[0][5] == {"peer_loads": 2 * n0, "peer_stores": 2 * n0, "local_hbm": 28 * n0}
+    for r in range(world):
+        assert res[r][6] == 10.0 and res[r][7] == float(padded)
