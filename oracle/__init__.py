@@ -73,6 +73,9 @@ def lib():
         L.oracle_plan.argtypes = [i32, vp, vp, i32, i32, u64, vp, vp, vp, vp, i64,
                                   ctypes.POINTER(_PlanInfo)]
         L.oracle_plan.restype = ctypes.c_int
+        L.oracle_plan_groups.argtypes = [i32, vp, vp, i32, i32, u64, vp, vp, vp, vp, vp, i64,
+                                         ctypes.POINTER(_PlanInfo)]
+        L.oracle_plan_groups.restype = ctypes.c_int
         L.oracle_reduce.argtypes = [i32, vp, i64, vp]
         L.oracle_adamw_scalars.argtypes = [ctypes.POINTER(_HP), i64, ctypes.POINTER(_Scalars)]
         L.oracle_adamw.argtypes = [ctypes.POINTER(_Scalars), vp, i64, vp, vp, vp]
@@ -132,11 +135,14 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
 # ---------------------------------------------------------------------------
 
 class Plan:
-    """Partition + bucket + segment tables for all ranks."""
+    """Partition + bucket + segment tables for all ranks.  groups (optional):
+    one id per tensor, non-decreasing; then one bucket per group instead of
+    the bucket_cap_bytes rule."""
 
-    def __init__(self, shapes, world_size, mode, bucket_cap_bytes):
+    def __init__(self, shapes, world_size, mode, bucket_cap_bytes, groups=None):
         shapes = [tuple(int(d) for d in s) for s in shapes]
         n = len(shapes)
+        grp = None if groups is None else np.array(list(groups) or [0], dtype=np.int32)
         ndims = np.array([len(s) for s in shapes] or [0], dtype=np.int32)
         dims = np.array([d for s in shapes for d in s] or [0], dtype=np.int64)
         owner = np.zeros(max(1, n), dtype=np.int32)
@@ -146,9 +152,14 @@ class Plan:
         cap = 16
         while True:
             segs = np.zeros(cap, dtype=SEGMENT_DTYPE)
-            rc = lib().oracle_plan(n, _ptr(ndims), _ptr(dims), world_size, mode,
-                                   int(bucket_cap_bytes), _ptr(owner), _ptr(bucket),
-                                   _ptr(owned), _ptr(segs), cap, ctypes.byref(info))
+            if grp is None:
+                rc = lib().oracle_plan(n, _ptr(ndims), _ptr(dims), world_size, mode,
+                                       int(bucket_cap_bytes), _ptr(owner), _ptr(bucket),
+                                       _ptr(owned), _ptr(segs), cap, ctypes.byref(info))
+            else:
+                rc = lib().oracle_plan_groups(n, _ptr(ndims), _ptr(dims), world_size, mode,
+                                              int(bucket_cap_bytes), _ptr(grp), _ptr(owner), _ptr(bucket),
+                                              _ptr(owned), _ptr(segs), cap, ctypes.byref(info))
             if rc == -2:
                 cap = int(info.n_segments)
                 continue
@@ -159,6 +170,7 @@ class Plan:
         self.world_size = world_size
         self.mode = mode
         self.bucket_cap_bytes = int(bucket_cap_bytes)
+        self.groups = None if groups is None else [int(g) for g in groups]
         self.total_numel = int(info.total_numel)
         self.padded_numel = int(info.padded_numel)
         self.chunk = int(info.chunk)

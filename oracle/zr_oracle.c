@@ -108,14 +108,19 @@ typedef struct {
 } oracle_plan_info;
 
 /* Returns 0 on success, -1 on bad arguments, -2 if seg_cap is too small
- * (n_segments is still filled in). */
-int oracle_plan(int32_t n_tensors, const int32_t* ndims, const int64_t* dims_flat,
-                int32_t world_size, int32_t mode, uint64_t cap_bytes,
-                int32_t* tensor_owner,     /* [n_tensors]; -1 in flat mode       */
-                int32_t* tensor_bucket,    /* [n_tensors]                        */
-                int64_t* owned_numel,      /* [world_size]                       */
-                oracle_segment* segs, int64_t seg_cap, oracle_plan_info* info) {
+ * (n_segments is still filled in).  groups == NULL: buckets by the cap
+ * rule; else one group id per tensor, non-decreasing in declaration order,
+ * and one bucket per group (cap_bytes unused). */
+int oracle_plan_groups(int32_t n_tensors, const int32_t* ndims, const int64_t* dims_flat,
+                       int32_t world_size, int32_t mode, uint64_t cap_bytes, const int32_t* groups,
+                       int32_t* tensor_owner,     /* [n_tensors]; -1 in flat mode       */
+                       int32_t* tensor_bucket,    /* [n_tensors]                        */
+                       int64_t* owned_numel,      /* [world_size]                       */
+                       oracle_segment* segs, int64_t seg_cap, oracle_plan_info* info) {
     if (n_tensors < 0 || world_size < 1 || (mode != OR_FLAT && mode != OR_WHOLE)) return -1;
+    if (groups)
+        for (int32_t t = 1; t < n_tensors; ++t)
+            if (groups[t] < groups[t - 1]) return -1;
 
     int64_t* numel = (int64_t*)calloc((size_t)n_tensors + 1, sizeof(int64_t));
     int64_t* goff = (int64_t*)calloc((size_t)n_tensors + 1, sizeof(int64_t));
@@ -179,13 +184,17 @@ int oracle_plan(int32_t n_tensors, const int32_t* ndims, const int64_t* dims_fla
 
     /* Buckets: walk the tensors in reverse declaration order (the order the
      * backward pass produces gradients); open a new bucket when the next
-     * tensor's bf16 gradient bytes would push a non-empty bucket past the cap. */
+     * tensor's bf16 gradient bytes would push a non-empty bucket past the cap
+     * -- or, with groups, whenever the next tensor belongs to another group
+     * (a layer's gradients are reduced together once its backward is done). */
     int32_t bucket = 0;
     uint64_t fill_bytes = 0;
     int holds_any = 0;
     for (int32_t t = n_tensors - 1; t >= 0; --t) {
         uint64_t bytes = 2u * (uint64_t)numel[t];
-        if (holds_any && fill_bytes + bytes > cap_bytes) {
+        int new_bucket = groups ? (holds_any && groups[t] != groups[t + 1])
+                                : (holds_any && fill_bytes + bytes > cap_bytes);
+        if (new_bucket) {
             bucket += 1;
             fill_bytes = 0;
             holds_any = 0;
@@ -245,6 +254,15 @@ int oracle_plan(int32_t n_tensors, const int32_t* ndims, const int64_t* dims_fla
     info->n_segments = ns;
     free(numel); free(goff); free(owned_off); free(order);
     return ns > seg_cap ? -2 : 0;
+}
+
+/* The cap rule alone (no groups). */
+int oracle_plan(int32_t n_tensors, const int32_t* ndims, const int64_t* dims_flat,
+                int32_t world_size, int32_t mode, uint64_t cap_bytes,
+                int32_t* tensor_owner, int32_t* tensor_bucket, int64_t* owned_numel,
+                oracle_segment* segs, int64_t seg_cap, oracle_plan_info* info) {
+    return oracle_plan_groups(n_tensors, ndims, dims_flat, world_size, mode, cap_bytes, NULL,
+                              tensor_owner, tensor_bucket, owned_numel, segs, seg_cap, info);
 }
 
 /* ------------------------------------------------------------------------ */

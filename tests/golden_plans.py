@@ -28,6 +28,8 @@ def load(path):
         "N": int(totals["N"]), "padded": int(totals["padded"]), "C": int(totals["C"]),
         "n_buckets": int(totals["n_buckets"]),
         "owned_numel": [int(x) for x in meta["owned_numel"].split()] if "owned_numel" in meta else None,
+        # one group id per tensor (one bucket per group), or None for the cap rule
+        "groups": [int(x) for x in meta["groups"].split()] if "groups" in meta else None,
         # bucket tensor owner offset_in_tensor length global_offset owned_offset
         "segments": rows,
     }

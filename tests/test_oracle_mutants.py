@@ -39,8 +39,10 @@ MUTANTS = [
      ["test_oracle_bf16.py"]),
     ("buckets_forward", "for (int32_t t = n_tensors - 1; t >= 0; --t) {\n        uint64_t bytes",
      "for (int32_t t = 0; t < n_tensors; ++t) {\n        uint64_t bytes", ["test_oracle_plan.py"]),
-    ("bucket_cap_inclusive", "if (holds_any && fill_bytes + bytes > cap_bytes)",
-     "if (holds_any && fill_bytes + bytes >= cap_bytes)", ["test_oracle_plan.py"]),
+    ("bucket_cap_inclusive", "(holds_any && fill_bytes + bytes > cap_bytes)",
+     "(holds_any && fill_bytes + bytes >= cap_bytes)", ["test_oracle_plan.py"]),
+    ("groups_merged", "(holds_any && groups[t] != groups[t + 1])", "(holds_any && groups[t] > groups[t + 1])",
+     ["test_oracle_plan.py"]),
     ("lpt_tie_to_highest_rank", "if (owned_numel[r] < owned_numel[best]) best = r;",
      "if (owned_numel[r] <= owned_numel[best]) best = r;", ["test_oracle_plan.py"]),
     ("flat_chunk_floor", "C = (N + world_size - 1) / world_size;", "C = N / world_size + 1;",

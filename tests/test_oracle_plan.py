@@ -25,7 +25,7 @@ def seg_tuples(plan):
 
 @pytest.mark.parametrize("g", all_golden_plans(), ids=lambda g: g["name"])
 def test_hand_derived_tables(g):
-    plan = oracle.Plan(g["shapes"], g["world_size"], g["mode"], g["cap_bytes"])
+    plan = oracle.Plan(g["shapes"], g["world_size"], g["mode"], g["cap_bytes"], groups=g["groups"])
     assert (plan.total_numel, plan.padded_numel, plan.chunk, plan.n_buckets) == \
         (g["N"], g["padded"], g["C"], g["n_buckets"])
     assert seg_tuples(plan) == g["segments"]
@@ -66,7 +66,13 @@ def check_invariants(plan):
         assert pos == n
         assert len({int(s["bucket"]) for s in segs if s["tensor"] == t}) <= 1
     # buckets: reverse declaration order, cap respected unless a single tensor
-    if len(numels):
+    if len(numels) and plan.groups is not None:
+        # one bucket per group, the last group first
+        bt = plan.tensor_bucket
+        distinct = sorted(set(plan.groups), reverse=True)
+        assert plan.n_buckets == len(distinct)
+        assert [distinct.index(g) for g in plan.groups] == bt.tolist()
+    elif len(numels):
         bt = plan.tensor_bucket
         assert bt[-1] == 0 and all(bt[i] >= bt[i + 1] for i in range(len(bt) - 1))
         for b in range(plan.n_buckets):
@@ -118,6 +124,36 @@ def test_random_plans_invariants():
         cap = int(rng.integers(1, 400))
         plan = oracle.Plan(shapes, W, mode, cap)
         check_invariants(plan)
+
+
+def test_random_grouped_plans_invariants():
+    """Buckets given by tensor groups: one bucket per group, in reverse
+    order; owners, global and owned offsets are those of the same set
+    under the cap rule (buckets change only bucket ids and segment order)."""
+    rng = np.random.default_rng(12)
+    for trial in range(300):
+        nt = int(rng.integers(0, 10))
+        shapes = [tuple(int(x) for x in rng.integers(0, 40, size=int(rng.integers(0, 3))))
+                  for _ in range(nt)]
+        groups = np.cumsum(rng.integers(0, 2, size=nt)).tolist()
+        W = int(rng.integers(1, 9))
+        mode = int(rng.integers(0, 2))
+        plan = oracle.Plan(shapes, W, mode, 0, groups=groups)
+        check_invariants(plan)
+        ref = oracle.Plan(shapes, W, mode, 1 << 20)
+        key = lambda seg: (int(seg["tensor"]), int(seg["offset_in_tensor"]))
+        rest = lambda segs: sorted((key(x), int(x["owner"]), int(x["length"]), int(x["global_offset"]),
+                                    int(x["owned_offset"])) for x in segs)
+        assert rest(plan.segments) == rest(ref.segments)
+        assert plan.owned_numel.tolist() == ref.owned_numel.tolist()
+
+
+def test_grouped_plans_reject_decreasing_groups():
+    with pytest.raises(ValueError):
+        oracle.Plan([(4,), (5,), (6,)], 2, oracle.FLAT, 0, groups=[0, 1, 0])
+    # one group: a single bucket holding everything (and the flat pad)
+    plan = oracle.Plan([(4,), (5,), (6,)], 2, oracle.FLAT, 0, groups=[3, 3, 3])
+    assert plan.n_buckets == 1 and set(plan.segments["bucket"].tolist()) == {0}
 
 
 def test_parameter_counts_of_the_sets():
