@@ -27,7 +27,7 @@
  *               ("CS336", ZeRO-1 sketch, update-then-gather).
  *
  * The four stages run as one fused, memory-bound GPU pass (two passes and a
- * tiny combine kernel when clipping).  The W replicas' gradients live in
+ * small combine kernel when clipping).  The W replicas' gradients live in
  * memory the GPU can load from: its own, or other GPUs' buffers mapped with
  * CUDA IPC (zr_ipc_*).  There is no collective: the reduce-scatter and the
  * all-gather are the kernel's own loads and stores.
@@ -127,6 +127,22 @@ zr_status zr_plan_create(int32_t n_tensors, const int32_t* ndims, const int64_t*
                          int32_t world_size, int32_t rank, zr_partition mode,
                          uint64_t bucket_cap_bytes, const zr_adamw* hp, zr_plan** out);
 
+/* zr_plan_create with buckets given by tensor groups instead of a byte cap:
+ * tensor_group[t] (n_tensors entries, non-decreasing in declaration order)
+ * names the unit tensor t belongs to -- typically its layer -- and every
+ * group becomes one bucket, numbered in backward order (the last group is
+ * bucket 0; the flat zero pad closes bucket 0 as usual).  The unit is the
+ * ZeRO-3 / FSDP one ("CS336 lecture 8", FSDP sketch; "Scaling training to
+ * thousands of GPUs", 11:24 ZeRO, stage 3): zr_step_bucket on a layer's
+ * bucket reduces that layer's gradients, and updates its slice, as soon as
+ * its backward has produced them.  Partition, owners, offsets and tiles are
+ * those of zr_plan_create; only bucket ids and segment order differ.
+ * Errors: as zr_plan_create, plus ZR_ERR_INVALID_ARG (tensor_group NULL
+ * with n_tensors > 0, or decreasing). */
+zr_status zr_plan_create_grouped(int32_t n_tensors, const int32_t* ndims, const int64_t* const* shapes,
+                                 const int32_t* tensor_group, int32_t world_size, int32_t rank,
+                                 zr_partition mode, const zr_adamw* hp, zr_plan** out);
+
 /* Sizes of the plan.  Any output pointer may be NULL.  owned_numel is this
  * rank's element count; n_segments counts all ranks' segments. */
 zr_status zr_plan_query(const zr_plan* plan, int64_t* total_numel, int64_t* padded_numel,
@@ -137,16 +153,17 @@ zr_status zr_plan_query(const zr_plan* plan, int64_t* total_numel, int64_t* padd
  * ZR_ERR_BUFFER_TOO_SMALL is returned (call with cap 0 to size). */
 zr_status zr_plan_segments(const zr_plan* plan, zr_segment* out, int64_t cap, int64_t* n);
 
-/* Device workspace the plan needs: the tile tables, the clip partial sums,
- * a few scalars and status words, the ZeRO-3 gather piece table (32 bytes
- * per piece of at most 16384 elements, all ranks) and (when clipping with
- * W > 4) an fp32 scratch copy of the reduced gradient. */
+/* Device workspace the plan needs: the tile tables, the clip partial sums
+ * (one double per tile, one per group of 1024 tiles, and a completion
+ * counter), a few scalars and status words, the ZeRO-3 gather
+ * piece table (32 bytes per piece of at most 16384 elements, all ranks) and
+ * (when clipping with W > 4) an fp32 scratch copy of the reduced gradient. */
 zr_status zr_plan_workspace_bytes(const zr_plan* plan, uint64_t* bytes);
 
 /* Bind a device workspace (>= zr_plan_workspace_bytes, 256-byte aligned,
  * owned by the caller, kept alive while the plan is used) and upload the
  * tile tables and the gather piece table into it with asynchronous copies
- * on `stream` (clearing checked mode's status).  Selects the
+ * on `stream` (clearing checked mode's status and the clip's counter).  Selects the
  * current CUDA device as the plan's device.  Errors: ZR_ERR_NO_WORKSPACE
  * (too small), ZR_ERR_ALIGNMENT, ZR_ERR_UNSUPPORTED (the current device is
  * not compute capability 10.x), ZR_ERR_CUDA. */
@@ -447,8 +464,8 @@ zr_status zr_gather_params(const zr_plan* plan, int32_t first_tensor, int32_t n_
  * reading those tables (zr_step, zr_step_device_count, zr_step_bucket,
  * zr_step_finish, zr_step_host, zr_grad_sumsq, zr_debug_reduce,
  * zr_gather_params) run that check first on its stream; 0 (the default)
- * turns it off.  zr_step_no_alloc uploads its own
- * table on every call and is not affected.
+ * turns it off.  zr_step_no_alloc keeps its own copy
+ * of the table and is not affected.
  * zr_plan_check_result synchronises `stream` and reads the status:
  * bad_tiles = entries that failed an invariant (all tables, counted at every
  * check since the workspace was bound), first_bad = the smallest failing
@@ -484,24 +501,38 @@ zr_status zr_plan_check_result(const zr_plan* plan, zr_check_result* out, zr_str
  * only; otherwise may be NULL): the device array of world_size doubles that
  * zr_plan_set_sumsq_partials would bind -- other ranks' S_w in, this rank's
  * entry written.  No workspace needs to be bound; the call makes no
- * cudaMalloc or cudaFree and calls no allocating routine.
+ * cudaMalloc or cudaFree and calls no allocating routine.  It runs zr_step's
+ * kernels in zr_step's order, so master, m, v, param_out and S_r are
+ * bit-identical to zr_step's.
  *
- * Scratch (the tile table and, with clipping, one double per tile) lives in a
- * file-scope device array of ZR_NO_ALLOC_SCRATCH_BYTES (4 MiB) that every GPU
- * that loads the library holds until the process exits.  The plan needs
- * 32 bytes per tile, plus 8 more per tile with clipping, plus about 1 KB:
- * up to about 131,000 tiles (about 104,800 with clipping).  A tile covers up
- * to 2048 owned elements, so a shard of up to about 268 M owned elements
- * fits (about 214 M with clipping).  A larger plan gets ZR_ERR_UNSUPPORTED before
- * anything is launched: use zr_step with a workspace instead.  With clipping,
- * the second pass reads the gradients again instead of keeping an fp32 copy
- * of the averaged gradient, so results are bit-identical to zr_step's.
+ * Scratch (the tile table and, with clipping, one double per tile, one per
+ * group of 1024 tiles and a counter) lives in a file-scope device
+ * array of ZR_NO_ALLOC_SCRATCH_BYTES (4 MiB) that every GPU that loads the
+ * library holds until the process exits.  The plan needs 32 bytes per tile,
+ * plus about 8 more per tile with clipping, plus about 1 KB: up to about
+ * 131,000 tiles (about 104,800 with clipping).  A tile covers up to 2048
+ * owned elements, so a shard of up to about 268 M owned elements fits
+ * (about 214 M with clipping).  A larger plan gets ZR_ERR_UNSUPPORTED before
+ * anything is launched: use zr_step with a workspace instead.  With
+ * clipping, the second pass reads the gradients again instead of keeping an
+ * fp32 copy of the averaged gradient (the same values: the fold is
+ * deterministic).
  *
- * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) and caches it: make that first call before any
- * stream capture.  Every call, on every plan, uses the same array and leaves
- * its contents behind; nothing in it needs to start at zero (each call writes
- * what it reads).  Calls whose work overlaps on the GPU (different streams
+ * Set-up: the first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it for the life of the process; make
+ * that first call before any stream capture.  cudaDeviceReset is not
+ * supported: after it the cached address, and the record of which table
+ * the array holds, would be stale.
+ *
+ * The tile table is copied from the plan's host memory (an asynchronous
+ * copy on `stream` from pageable memory) when the array does not already
+ * hold this plan's current table: on the plan's first call on the device,
+ * after another plan's call on that device, and after
+ * zr_plan_set_param_layout rebuilt the plan's tables.  A loop that steps one
+ * plan copies it once; its later calls enqueue only kernels (and, with
+ * clipping, a device-side memset of the counter, which must start at
+ * zero).  Every call, on every plan, uses the same array and leaves its
+ * contents behind.  Calls whose work overlaps on the GPU (different streams
  * without ordering between them) race on the array and give wrong results.
  * Errors: as zr_step, plus ZR_ERR_UNSUPPORTED (plan too large for the array,
  * or the current device is not compute capability 10.x). */

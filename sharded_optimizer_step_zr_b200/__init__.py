@@ -39,7 +39,7 @@ ZR_PARTITION_WHOLE_TENSOR = 1
 ZR_MAX_WORLD_SIZE = 512
 
 EXPORTED = [
-    "zr_plan_create", "zr_plan_query", "zr_plan_segments", "zr_plan_workspace_bytes",
+    "zr_plan_create", "zr_plan_create_grouped", "zr_plan_query", "zr_plan_segments", "zr_plan_workspace_bytes",
     "zr_plan_set_workspace", "zr_plan_set_adamw", "zr_plan_set_device_lr", "zr_plan_set_sumsq_partials", "zr_step", "zr_step_device_count",
     "zr_step_bucket",
     "zr_step_finish", "zr_step_host",
@@ -76,6 +76,7 @@ class zr_ipc_handle(ctypes.Structure):
 _vp, _i32, _i64, _u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64
 _P = ctypes.POINTER
 _lib.zr_plan_create.argtypes = [_i32, _vp, _vp, _i32, _i32, ctypes.c_int, _u64, _P(zr_adamw), _P(_vp)]
+_lib.zr_plan_create_grouped.argtypes = [_i32, _vp, _vp, _vp, _i32, _i32, ctypes.c_int, _P(zr_adamw), _P(_vp)]
 _lib.zr_plan_query.argtypes = [_vp, _P(_i64), _P(_i64), _P(_i64), _P(_i32), _P(_i64)]
 _lib.zr_plan_segments.argtypes = [_vp, _vp, _i64, _P(_i64)]
 _lib.zr_plan_workspace_bytes.argtypes = [_vp, _P(_u64)]
@@ -157,8 +158,10 @@ def zr_status_string(status: int) -> str:
 
 def zr_plan_create(shapes, world_size: int, rank: int, mode: int, bucket_cap_bytes: int,
                    lr=3e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.1,
-                   max_grad_norm=0.0) -> int:
-    """Returns the plan handle (an integer); release it with zr_plan_destroy."""
+                   max_grad_norm=0.0, groups=None) -> int:
+    """Returns the plan handle (an integer); release it with zr_plan_destroy.
+    groups (one id per tensor, non-decreasing): zr_plan_create_grouped, one
+    bucket per group, bucket_cap_bytes unused."""
     shapes = [tuple(int(d) for d in s) for s in shapes]
     n = len(shapes)
     ndims = (ctypes.c_int32 * max(1, n))(*[len(s) for s in shapes])
@@ -166,8 +169,16 @@ def zr_plan_create(shapes, world_size: int, rank: int, mode: int, bucket_cap_byt
     shape_ptrs = (ctypes.c_void_p * max(1, n))(*[ctypes.addressof(a) for a in dim_arrays])
     hp = zr_adamw(lr, beta1, beta2, eps, weight_decay, max_grad_norm)
     out = ctypes.c_void_p()
-    _check(_lib.zr_plan_create(n, ndims, shape_ptrs, world_size, rank, mode, int(bucket_cap_bytes),
-                               ctypes.byref(hp), ctypes.byref(out)), "zr_plan_create")
+    if groups is None:
+        _check(_lib.zr_plan_create(n, ndims, shape_ptrs, world_size, rank, mode, int(bucket_cap_bytes),
+                                   ctypes.byref(hp), ctypes.byref(out)), "zr_plan_create")
+    else:
+        groups = [int(g) for g in groups]
+        if len(groups) != n:
+            raise ValueError("groups: one id per tensor")
+        grp = (ctypes.c_int32 * max(1, n))(*groups)
+        _check(_lib.zr_plan_create_grouped(n, ndims, shape_ptrs, grp, world_size, rank, mode,
+                                           ctypes.byref(hp), ctypes.byref(out)), "zr_plan_create_grouped")
     return out.value
 
 

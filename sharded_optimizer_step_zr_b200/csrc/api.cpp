@@ -9,6 +9,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 #include <new>
 
@@ -40,6 +41,22 @@ zr::LaunchArgs base_args(const zr_plan* p) {
     a.n_targets = p->n_gather_targets;
     a.targets = p->d_gather_targets;
     return a;
+}
+
+// The clip's S_r / coefficient arguments over every tile of the plan.
+zr::ClipArgs clip_args(const zr_plan* p, double* partials_all, double* sumsq_out) {
+    zr::ClipArgs c{};
+    c.tile_partials = p->d_tile_partials;
+    c.n_tiles = static_cast<int32_t>(p->tiles.size());
+    c.world_size = p->world_size;
+    c.ticket = p->d_clip_ticket;
+    c.group_sums = p->d_clip_group_sums;
+    c.partials_all = partials_all;
+    c.sumsq_out = sumsq_out;
+    c.coef_out = p->d_clip_coef;
+    c.rank = p->rank;
+    c.max_norm = p->hp.max_grad_norm;
+    return c;
 }
 
 // The bf16 destination: param_out, or the plan's gather targets (then
@@ -106,6 +123,10 @@ zr_status upload_tables(zr_plan* p, zr_stream_t stream) {
     if (cudaMemsetAsync(p->d_check, 0, sizeof(uint64_t) * zr::kCheckWords, s) != cudaSuccess ||
         cudaMemsetAsync(p->d_check + 1, 0xFF, sizeof(uint64_t), s) != cudaSuccess)
         return ZR_ERR_CUDA;
+    // The clip's completion counter starts at zero (each combine leaves it
+    // at zero again).
+    if (p->d_clip_ticket && cudaMemsetAsync(p->d_clip_ticket, 0, sizeof(uint32_t), s) != cudaSuccess)
+        return ZR_ERR_CUDA;
     return ZR_OK;
 }
 
@@ -163,9 +184,31 @@ const char* zr_status_string(zr_status s) {
     return "unknown zr_status";
 }
 
+static zr_status create_plan(int32_t n_tensors, const int32_t* ndims, const int64_t* const* shapes,
+                             const int32_t* tensor_group, int32_t world_size, int32_t rank, zr_partition mode,
+                             uint64_t bucket_cap_bytes, const zr_adamw* hp, zr_plan** out);
+
 zr_status zr_plan_create(int32_t n_tensors, const int32_t* ndims, const int64_t* const* shapes,
                          int32_t world_size, int32_t rank, zr_partition mode,
                          uint64_t bucket_cap_bytes, const zr_adamw* hp, zr_plan** out) {
+    return create_plan(n_tensors, ndims, shapes, nullptr, world_size, rank, mode, bucket_cap_bytes, hp, out);
+}
+
+zr_status zr_plan_create_grouped(int32_t n_tensors, const int32_t* ndims, const int64_t* const* shapes,
+                                 const int32_t* tensor_group, int32_t world_size, int32_t rank,
+                                 zr_partition mode, const zr_adamw* hp, zr_plan** out) {
+    if (out) *out = nullptr;
+    if (n_tensors > 0 && !tensor_group) return ZR_ERR_INVALID_ARG;
+    for (int32_t t = 1; t < n_tensors; ++t)
+        if (tensor_group[t] < tensor_group[t - 1]) return ZR_ERR_INVALID_ARG;
+    static const int32_t none = 0;
+    return create_plan(n_tensors, ndims, shapes, n_tensors > 0 ? tensor_group : &none, world_size, rank, mode, 0,
+                       hp, out);
+}
+
+static zr_status create_plan(int32_t n_tensors, const int32_t* ndims, const int64_t* const* shapes,
+                             const int32_t* tensor_group, int32_t world_size, int32_t rank, zr_partition mode,
+                             uint64_t bucket_cap_bytes, const zr_adamw* hp, zr_plan** out) {
     if (!out) return ZR_ERR_INVALID_ARG;
     *out = nullptr;
     if (n_tensors < 0 || (n_tensors > 0 && (!ndims || !shapes)) || !hp) return ZR_ERR_INVALID_ARG;
@@ -174,11 +217,14 @@ zr_status zr_plan_create(int32_t n_tensors, const int32_t* ndims, const int64_t*
     if (mode != ZR_PARTITION_FLAT && mode != ZR_PARTITION_WHOLE_TENSOR) return ZR_ERR_INVALID_ARG;
     zr_plan* p = new (std::nothrow) zr_plan();
     if (!p) return ZR_ERR_INVALID_ARG;
+    static std::atomic<uint64_t> next_uid{1};
+    p->uid = next_uid.fetch_add(1);
     p->world_size = world_size;
     p->rank = rank;
     p->mode = mode;
     p->cap_bytes = bucket_cap_bytes;
     p->hp = *hp;
+    if (tensor_group && n_tensors > 0) p->tensor_group.assign(tensor_group, tensor_group + n_tensors);
     zr_status st;
     try {
         st = zr::build_plan(*p, n_tensors, ndims, shapes);
@@ -243,6 +289,8 @@ zr_status zr_plan_set_workspace(zr_plan* p, void* d_ws, uint64_t bytes, zr_strea
     p->d_tiles = reinterpret_cast<zr::Tile*>(base + L.tiles);
     p->d_tiles_by_owned = reinterpret_cast<zr::Tile*>(base + L.tiles_by_owned);
     p->d_tile_partials = p->clip_enabled() ? reinterpret_cast<double*>(base + L.tile_partials) : nullptr;
+    p->d_clip_ticket = p->clip_enabled() ? reinterpret_cast<uint32_t*>(base + L.clip_ticket) : nullptr;
+    p->d_clip_group_sums = p->clip_enabled() ? reinterpret_cast<double*>(base + L.clip_group_sums) : nullptr;
     p->d_clip_coef = reinterpret_cast<float*>(base + L.clip_coef);
     p->d_own_sumsq = reinterpret_cast<double*>(base + L.own_sumsq);
     p->d_gather_targets = reinterpret_cast<uint16_t**>(base + L.gather_targets);
@@ -444,9 +492,9 @@ static zr_status step_impl(const zr_plan* p, const void* const* grad_ptrs, float
     a.tile_partials = p->d_tile_partials;
     int e = zr::launch_tiles(zr::Pass::kSumsq, a, grad_ptrs, false, scratch, s);
     if (e != cudaSuccess) return ZR_ERR_CUDA;
-    // Combine: this rank's S_r, all ranks' S in rank order, the coefficient.
-    e = zr::launch_clip_combine(p->d_tile_partials, a.n_tiles, p->d_sumsq_partials, p->world_size, p->rank,
-                                p->hp.max_grad_norm, p->d_clip_coef, p->d_own_sumsq, s);
+    // This rank's S_r (groups of tiles in parallel, then the groups), all
+    // ranks' S in rank order, the coefficient.
+    e = zr::launch_clip_combine(clip_args(p, p->d_sumsq_partials, p->d_own_sumsq), s);
     if (e != cudaSuccess) return ZR_ERR_CUDA;
     // Pass 2: scale by the coefficient, AdamW, cast.  Tiles in reverse
     // order: the first CTAs then read the g scratch that pass 1's last CTAs
@@ -527,8 +575,7 @@ zr_status zr_step_finish(const zr_plan* p, const void* const* grad_ptrs, float* 
     a.s = zr::adam_scalars(p->hp, step);
     a.g_buf = p->d_g_scratch;
     void* s = stream;
-    int e = zr::launch_clip_combine(p->d_tile_partials, a.n_tiles, p->d_sumsq_partials, p->world_size, p->rank,
-                                    p->hp.max_grad_norm, p->d_clip_coef, p->d_own_sumsq, s);
+    int e = zr::launch_clip_combine(clip_args(p, p->d_sumsq_partials, p->d_own_sumsq), s);
     if (e != cudaSuccess) return ZR_ERR_CUDA;
     a.clip_coef = p->d_clip_coef;
     a.reverse = 1;
@@ -559,9 +606,7 @@ zr_status zr_grad_sumsq(const zr_plan* p, const void* const* grad_ptrs, double* 
     a.tile_partials = p->d_tile_partials;
     int e = zr::launch_tiles(zr::Pass::kSumsq, a, grad_ptrs, false, false, s);
     if (e != cudaSuccess) return ZR_ERR_CUDA;
-    e = zr::launch_clip_combine(p->d_tile_partials, a.n_tiles, nullptr, p->world_size, p->rank,
-                                p->hp.max_grad_norm, nullptr, d_out, s);
-    return cuda_status(static_cast<cudaError_t>(e));
+    return cuda_status(static_cast<cudaError_t>(zr::launch_clip_combine(clip_args(p, nullptr, d_out), s)));
 }
 
 zr_status zr_debug_reduce(const zr_plan* p, const void* const* grad_ptrs, float* g_out, zr_stream_t stream) {
@@ -703,8 +748,7 @@ zr_status zr_step_host(const zr_plan* p, const void* const* host_grad_ptrs, void
         }
     }
     if (clip) {
-        if (zr::launch_clip_combine(p->d_tile_partials, n_tiles, p->d_sumsq_partials, p->world_size, p->rank,
-                                    p->hp.max_grad_norm, p->d_clip_coef, p->d_own_sumsq, S) != cudaSuccess)
+        if (zr::launch_clip_combine(clip_args(p, p->d_sumsq_partials, p->d_own_sumsq), S) != cudaSuccess)
             return ZR_ERR_CUDA;
         a.clip_coef = p->d_clip_coef;
         for (int k = 0; k < K; ++k) {

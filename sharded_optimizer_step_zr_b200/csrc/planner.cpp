@@ -6,7 +6,8 @@
 // element count, largest first).  Buckets ("Scaling training ...", 03:41 DP;
 // "DDP -> ZeRO" blog section 2.1): whole tensors in the order the backward
 // pass produces their gradients (reverse declaration order), capped by
-// bucket_cap_bytes of bf16 gradient.
+// bucket_cap_bytes of bf16 gradient -- or one bucket per group of tensors
+// (a layer: the FSDP unit of "CS336 lecture 8", FSDP sketch).
 #include <algorithm>
 #include <cstring>
 #include <cmath>
@@ -54,7 +55,11 @@ void pack_buckets(zr_plan& p) {
     uint64_t bytes_in_open = 0;
     for (int32_t t = p.n_tensors - 1; t >= 0; --t) {
         const uint64_t b = 2ull * static_cast<uint64_t>(p.numel[t]);
-        const bool open_new = members.empty() || (!members.back().empty() && bytes_in_open + b > p.cap_bytes);
+        // grouped plans: a new bucket wherever the (next in backward order) tensor changes group
+        const bool open_new = members.empty() ||
+                              (p.tensor_group.empty()
+                                   ? (!members.back().empty() && bytes_in_open + b > p.cap_bytes)
+                                   : p.tensor_group[t] != p.tensor_group[t + 1]);
         if (open_new) {
             members.emplace_back();
             bytes_in_open = 0;
@@ -120,6 +125,7 @@ void cut_segments(zr_plan& p) {
 // layout, then cut into tiles: a scalar head up to the next multiple of 8
 // owned elements, vector tiles of kTileElems, a scalar tail.
 void build_tiles(zr_plan& p) {
+    ++p.table_generation;
     p.tiles.clear();
     p.bucket_first_tile.assign(p.n_buckets + 1, 0);
     struct Run { int64_t owned, global, len; };
@@ -298,6 +304,11 @@ WorkspaceLayout workspace_layout(const zr_plan& p) {
     off = align256(off + sizeof(Tile) * std::max<size_t>(1, p.tiles.size()));
     L.tile_partials = off;
     off = align256(off + (p.clip_enabled() ? sizeof(double) * std::max<size_t>(1, p.tiles.size()) : 0));
+    const uint64_t groups = static_cast<uint64_t>(clip_groups(static_cast<int32_t>(std::max<size_t>(1, p.tiles.size()))));
+    L.clip_ticket = off;
+    off = align256(off + (p.clip_enabled() ? sizeof(uint32_t) : 0));
+    L.clip_group_sums = off;
+    off = align256(off + (p.clip_enabled() ? sizeof(double) * groups : 0));
     L.clip_coef = off;
     off = align256(off + sizeof(float));
     L.own_sumsq = off;

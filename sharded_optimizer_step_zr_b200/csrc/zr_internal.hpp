@@ -92,6 +92,28 @@ enum class Pass : int {
     kStepClip = 3,     // (reduce | read g scratch) -> * clip coef -> AdamW -> cast
 };
 
+// The clip's sum of squares S_r of a rank's averaged gradient, in a fixed
+// order: the per-tile partials (by tile index) in groups of
+// kClipGroupTiles; each group's total by fixed_sum128, then the groups'
+// totals by fixed_sum128 again (zr_kernels.cu: one CTA per group, the last
+// to finish sums the groups).  Every path that forms S_r uses that kernel,
+// so S_r and the coefficient are the same bits on every call and every rank.
+constexpr int32_t kClipGroupTiles = 1024;
+ZR_HOST_DEVICE inline int32_t clip_groups(int32_t n_tiles) { return (n_tiles + kClipGroupTiles - 1) / kClipGroupTiles; }
+
+struct ClipArgs {
+    const double* tile_partials;  // one per tile of the plan (tile index)
+    int32_t n_tiles;               // every tile of the plan
+    int32_t world_size;
+    uint32_t* ticket;              // completion counter of the groups, zero between launches
+    double* group_sums;            // clip_groups(n_tiles) group totals
+    double* partials_all;          // world_size entries: this rank's S_r written, all summed (or null)
+    double* sumsq_out;             // this rank's S_r alone (or null)
+    float* coef_out;               // the clip coefficient (when partials_all is set)
+    int32_t rank;
+    float max_norm;
+};
+
 struct LaunchArgs {
     const Tile* tiles;
     int32_t n_tiles;
@@ -118,9 +140,9 @@ struct LaunchArgs {
 int launch_tiles(Pass pass, const LaunchArgs& a, const void* const* grad_ptrs, bool g_from_scratch,
                  bool write_g_scratch, void* stream);
 int launch_device_scalars(int64_t* d_step, const zr_adamw& hp, const float* d_lr, AdamScalars* out, void* stream);
-int launch_clip_combine(const double* tile_partials, int32_t n_tiles, double* partials_all,
-                        int32_t world_size, int32_t rank, float max_norm, float* clip_coef_out,
-                        double* sumsq_out, void* stream);
+// S_r and the coefficient from the per-tile partials of pass 1: one
+// 128-thread CTA per group of tiles, the last to finish sums the groups.
+int launch_clip_combine(const ClipArgs& c, void* stream);
 // ZeRO-3 gather: copy pieces [first, first + n) from the W shards to dst,
 // where dst holds the global range starting at dst_base, on at most
 // max_ctas CTAs (<= 0: one per piece).  shard_ptrs: host
@@ -165,6 +187,7 @@ struct zr_plan {
     std::vector<int64_t> goff;           // per tensor, global layout
     std::vector<int32_t> tensor_owner;   // whole-tensor mode
     std::vector<int32_t> tensor_bucket;
+    std::vector<int32_t> tensor_group;   // empty: buckets by cap_bytes; else one bucket per group
     std::vector<int64_t> rank_numel;     // owned element count per rank
     int64_t total_numel = 0;
     int64_t padded_numel = 0;
@@ -183,6 +206,8 @@ struct zr_plan {
     zr::Tile* d_tiles = nullptr;
     zr::Tile* d_tiles_by_owned = nullptr;
     double* d_tile_partials = nullptr;
+    uint32_t* d_clip_ticket = nullptr;    // workspace: the combine's completion counter (zeroed at upload)
+    double* d_clip_group_sums = nullptr;  // workspace: clip_groups(n_tiles) group totals
     float* d_clip_coef = nullptr;
     double* d_own_sumsq = nullptr;
     float* d_g_scratch = nullptr;
@@ -197,6 +222,8 @@ struct zr_plan {
     std::vector<int32_t> tensor_first_piece;        // n_tensors + 1 entries
     zr::GatherPiece* d_gather_pieces = nullptr;     // workspace copy
     bool checked = false;                  // verify the tables before every launch
+    uint64_t uid = 0;                      // unique per plan in this process (never reused)
+    uint64_t table_generation = 0;         // bumped whenever the tile tables are rebuilt
     uint64_t hash_tiles = 0;               // tile_word_hash sums of the host tables
     uint64_t hash_tiles_by_owned = 0;
     uint64_t hash_gather_pieces = 0;
@@ -222,8 +249,8 @@ zr_status build_plan(zr_plan& p, int32_t n_tensors, const int32_t* ndims,
                      const int64_t* const* shapes);
 // Workspace layout: offsets of each region, total bytes.
 struct WorkspaceLayout {
-    uint64_t tiles, tiles_by_owned, tile_partials, clip_coef, own_sumsq, gather_targets, dev_scalars, check,
-        gather_pieces, g_scratch, total;
+    uint64_t tiles, tiles_by_owned, tile_partials, clip_ticket, clip_group_sums, clip_coef, own_sumsq,
+        gather_targets, dev_scalars, check, gather_pieces, g_scratch, total;
 };
 WorkspaceLayout workspace_layout(const zr_plan& p);
 // Rebuilds this rank's tile tables for the plan's parameter layout: the

@@ -179,12 +179,80 @@ __device__ double block_sum(double x) {
 }
 
 // ---------------------------------------------------------------------------
+// the clip's sum of squares, in a fixed order
+// ---------------------------------------------------------------------------
+
+// Sum of count doubles at p by one 128-thread CTA, in a fixed order: thread
+// t adds p[t], p[t + 128], p[t + 256], ... in turn (loads of eight issued
+// before their additions), then block_sum.  L2 loads: the values were
+// written by other CTAs of this or an earlier launch.  Valid in thread 0.
+__device__ double fixed_sum128(const double* p, int32_t count) {
+    double x = 0.0;
+    for (int32_t i0 = threadIdx.x; i0 < count; i0 += 8 * kThreads) {
+        double v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = (i0 + k * kThreads < count) ? __ldcg(p + i0 + k * kThreads) : 0.0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (i0 + k * kThreads < count) x += v[k];
+    }
+    return block_sum(x);
+}
+
+// This rank's S_r is final: store it, and from all ranks' entries (summed in
+// rank order) the clip coefficient min(1, max_norm / (sqrt(S) + 1e-6)).
+__device__ void clip_coefficient(const ClipArgs& c, double own) {
+    if (c.sumsq_out) *c.sumsq_out = own;
+    if (c.partials_all) {
+        c.partials_all[c.rank] = own;
+        double S = c.partials_all[0];
+        for (int32_t w = 1; w < c.world_size; ++w) S += c.partials_all[w];
+        const double coef = static_cast<double>(c.max_norm) / (sqrt(S) + 1e-6);
+        *c.coef_out = static_cast<float>(coef < 1.0 ? coef : 1.0);
+    }
+}
+
+// CTA g of the combine: group g's total to group_sums[g]; the CTA that
+// finishes last then sums the groups and forms the coefficient.  "Last" is
+// decided by an atomic ticket after a memory fence (publish, then count);
+// no CTA ever waits for another, and the last one resets the counter for
+// the next launch.
+__device__ void clip_group_done(const ClipArgs& c, int32_t g) {
+    __shared__ int s_last;
+    const int32_t n_groups = clip_groups(c.n_tiles);
+    const int32_t first = g * kClipGroupTiles;
+    const double T = fixed_sum128(c.tile_partials + first, min(kClipGroupTiles, c.n_tiles - first));
+    if (threadIdx.x == 0) {
+        c.group_sums[g] = T;
+        __threadfence();
+        const uint32_t prev = atomicAdd(c.ticket, 1u);
+        s_last = prev == static_cast<uint32_t>(n_groups - 1);
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const double own = fixed_sum128(c.group_sums, n_groups);
+    if (threadIdx.x == 0) {
+        *c.ticket = 0u;
+        clip_coefficient(c, own);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // the tile kernel
 // ---------------------------------------------------------------------------
 
 template <int CAP, int G, Pass PASS, bool G_FROM_SCRATCH, bool WRITE_G, bool DEV_SCALARS, bool GATHER>
 __global__ void __launch_bounds__(kThreads)
 zr_tile_kernel(const GradPtrs<CAP> gp, const LaunchArgs a) {
+    // Launched as a programmatic dependent of the previous kernel on the
+    // stream (see launch_one): this grid may be scheduled while that one
+    // drains, and waits here until it has completed and its writes are
+    // visible -- before touching any memory (the previous kernel may be the
+    // last step, which wrote master / m / v, or checked mode's table check).
+    // Then it lets the next launch be scheduled as its own last CTAs run.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
     const int32_t tix = a.reverse ? a.n_tiles - 1 - static_cast<int32_t>(blockIdx.x)
                                   : static_cast<int32_t>(blockIdx.x);
     const Tile tile = a.tiles[tix];
@@ -296,46 +364,14 @@ zr_tile_kernel(const GradPtrs<CAP> gp, const LaunchArgs a) {
     }
 }
 
-// One block: S_r = sum of the per-tile partials in a fixed order, stored as
-// this rank's entry of the partials array (or to sumsq_out alone); then the
-// clip coefficient from all ranks' entries, summed in rank order.
-__global__ void __launch_bounds__(1024)
-zr_clip_combine_kernel(const double* __restrict__ tile_partials, int32_t n_tiles,
-                       double* partials_all, int32_t world_size, int32_t rank, float max_norm,
-                       float* clip_coef_out, double* sumsq_out) {
-    __shared__ double part[1024];
-    // Thread t adds partials t, t + B, t + 2B, ... in that order (B = block
-    // size); the loads of 16 of them are issued before their additions so
-    // the block is not bound by one memory round trip per partial.
-    constexpr int kBatch = 16;
-    const int32_t B = static_cast<int32_t>(blockDim.x);
-    double x = 0.0;
-    int32_t i = threadIdx.x;
-    for (; i + (kBatch - 1) * B < n_tiles; i += kBatch * B) {
-        double v[kBatch];
-#pragma unroll
-        for (int k = 0; k < kBatch; ++k) v[k] = tile_partials[i + k * B];
-#pragma unroll
-        for (int k = 0; k < kBatch; ++k) x += v[k];
-    }
-    for (; i < n_tiles; i += B) x += tile_partials[i];
-    part[threadIdx.x] = x;
-    __syncthreads();
-    for (int stride = blockDim.x / 2; stride >= 1; stride >>= 1) {
-        if (threadIdx.x < stride) part[threadIdx.x] += part[threadIdx.x + stride];
-        __syncthreads();
-    }
-    if (threadIdx.x == 0) {
-        const double own = part[0];
-        if (sumsq_out) *sumsq_out = own;
-        if (partials_all) {
-            partials_all[rank] = own;
-            double S = partials_all[0];
-            for (int32_t w = 1; w < world_size; ++w) S += partials_all[w];
-            const double c = static_cast<double>(max_norm) / (sqrt(S) + 1e-6);
-            *clip_coef_out = static_cast<float>(c < 1.0 ? c : 1.0);
-        }
-    }
+// S_r and the coefficient from the per-tile partials of pass 1: CTA g sums
+// group g, the last to finish sums the groups (clip_group_done).  Launched
+// as a programmatic dependent of pass 1 (it waits for it here) and lets
+// pass 2 be scheduled while it runs.
+__global__ void __launch_bounds__(kThreads) zr_clip_combine_kernel(const ClipArgs c) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+    clip_group_done(c, static_cast<int32_t>(blockIdx.x));
 }
 
 template <int CAP, int G, Pass PASS, bool FROM, bool WRITE, bool DEVSC, bool GATHER>
@@ -344,8 +380,20 @@ cudaError_t launch_one(const LaunchArgs& a, const void* const* grad_ptrs, cudaSt
     GradPtrs<CAP> gp;
     for (int w = 0; w < CAP; ++w)
         gp.p[w] = (grad_ptrs != nullptr && w < a.world_size) ? static_cast<const uint16_t*>(grad_ptrs[w]) : nullptr;
-    zr_tile_kernel<CAP, G, PASS, FROM, WRITE, DEVSC, GATHER><<<a.n_tiles, kThreads, 0, stream>>>(gp, a);
-    return cudaGetLastError();
+    // Programmatic dependent launch: the grid's scheduling overlaps the
+    // previous kernel's tail (back-to-back steps lose less to the launch
+    // gap); the kernel's first instruction waits for that kernel.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(a.n_tiles));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, zr_tile_kernel<CAP, G, PASS, FROM, WRITE, DEVSC, GATHER>, gp, a);
 }
 
 template <Pass PASS, bool FROM, bool WRITE, bool DEVSC = false, bool GATHER = false>
@@ -393,12 +441,19 @@ int launch_tiles(Pass pass, const LaunchArgs& a, const void* const* grad_ptrs, b
     return cudaErrorInvalidValue;
 }
 
-int launch_clip_combine(const double* tile_partials, int32_t n_tiles, double* partials_all,
-                        int32_t world_size, int32_t rank, float max_norm, float* clip_coef_out,
-                        double* sumsq_out, void* stream_v) {
-    zr_clip_combine_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream_v)>>>(
-        tile_partials, n_tiles, partials_all, world_size, rank, max_norm, clip_coef_out, sumsq_out);
-    return cudaGetLastError();
+int launch_clip_combine(const ClipArgs& c, void* stream_v) {
+    if (c.n_tiles <= 0) return cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(clip_groups(c.n_tiles)));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = static_cast<cudaStream_t>(stream_v);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, zr_clip_combine_kernel, c);
 }
 
 }  // namespace zr

@@ -28,37 +28,36 @@ namespace {
 // device address obtained with cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char zr_no_alloc_scratch[ZR_NO_ALLOC_SCRATCH_BYTES];
 
+// Per device: the array's device address (looked up once), and which plan's
+// tile table the array holds now (that plan's uid and table generation), so
+// a loop stepping one plan uploads its table once, not on every call.
+struct DeviceScratch {
+    void* address = nullptr;
+    uint64_t plan_uid = 0;          // 0: no table uploaded yet
+    uint64_t table_generation = 0;
+};
 constexpr int kMaxDevices = 256;
-void* g_scratch_address[kMaxDevices] = {};
-std::mutex g_scratch_mutex;
-
-// Device address of the scratch on `device` (which must be current): looked
-// up once per device, then cached.
-zr_status scratch_address(int device, void** out) {
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (g_scratch_address[device] == nullptr) {
-        void* p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, zr_no_alloc_scratch);
-        if (e != cudaSuccess || p == nullptr) return ZR_ERR_CUDA;
-        g_scratch_address[device] = p;
-    }
-    *out = g_scratch_address[device];
-    return ZR_OK;
-}
+DeviceScratch g_device[kMaxDevices];
+std::mutex g_mutex;
 
 struct ScratchLayout {
-    uint64_t tiles, tile_partials, clip_coef, own_sumsq, total;
+    uint64_t tiles, tile_partials, ticket, group_sums, clip_coef, own_sumsq, total;
 };
 
 uint64_t up256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
 
 ScratchLayout scratch_layout(uint64_t n_tiles, bool clip) {
+    const uint64_t groups = clip ? static_cast<uint64_t>(zr::clip_groups(static_cast<int32_t>(n_tiles))) : 0;
     ScratchLayout L{};
     uint64_t off = 0;
     L.tiles = off;
     off = up256(off + sizeof(zr::Tile) * n_tiles);
     L.tile_partials = off;
     off = up256(off + (clip ? sizeof(double) * n_tiles : 0));
+    L.ticket = off;
+    off = up256(off + (clip ? sizeof(uint32_t) : 0));
+    L.group_sums = off;
+    off = up256(off + sizeof(double) * groups);
     L.clip_coef = off;
     off = up256(off + sizeof(float));
     L.own_sumsq = off;
@@ -97,17 +96,34 @@ extern "C" zr_status zr_step_no_alloc(const zr_plan* p, const void* const* grad_
     int major = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return ZR_ERR_CUDA;
     if (major != 10) return ZR_ERR_UNSUPPORTED;
-    void* base_v = nullptr;
-    zr_status st = scratch_address(dev, &base_v);
-    if (st != ZR_OK) return st;
-    char* base = static_cast<char*>(base_v);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
-    // This call's tile table replaces whatever the previous call left.
-    zr::Tile* d_tiles = reinterpret_cast<zr::Tile*>(base + L.tiles);
-    if (cudaMemcpyAsync(d_tiles, p->tiles.data(), sizeof(zr::Tile) * p->tiles.size(), cudaMemcpyHostToDevice, s) !=
-        cudaSuccess)
-        return ZR_ERR_CUDA;
+    char* base = nullptr;
+    zr::Tile* d_tiles = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        DeviceScratch& ds = g_device[dev];
+        if (ds.address == nullptr) {
+            // Set-up on this device's first call: the array's device address.
+            void* addr = nullptr;
+            const cudaError_t e = cudaGetSymbolAddress(&addr, zr_no_alloc_scratch);
+            if (e != cudaSuccess || addr == nullptr) return ZR_ERR_CUDA;
+            ds.address = addr;
+        }
+        base = static_cast<char*>(ds.address);
+        d_tiles = reinterpret_cast<zr::Tile*>(base + L.tiles);
+        // The tile table, unless this plan's current table is the one the
+        // array already holds (the host-to-device copy from the plan's host
+        // memory happens once per plan and table, not once per step).
+        if (ds.plan_uid != p->uid || ds.table_generation != p->table_generation) {
+            ds.plan_uid = 0;   // stays unset if the copy cannot be enqueued
+            if (cudaMemcpyAsync(d_tiles, p->tiles.data(), sizeof(zr::Tile) * p->tiles.size(),
+                                cudaMemcpyHostToDevice, s) != cudaSuccess)
+                return ZR_ERR_CUDA;
+            ds.plan_uid = p->uid;
+            ds.table_generation = p->table_generation;
+        }
+    }
 
     zr::LaunchArgs a{};
     a.tiles = d_tiles;
@@ -124,17 +140,28 @@ extern "C" zr_status zr_step_no_alloc(const zr_plan* p, const void* const* grad_
     if (!clip)
         return zr::launch_tiles(zr::Pass::kStep, a, grad_ptrs, false, false, s) == cudaSuccess ? ZR_OK : ZR_ERR_CUDA;
 
-    // Every scratch word the kernels read below is written earlier in this
-    // call (one partial per tile, then the coefficient), so nothing needs
-    // clearing between calls.
-    double* d_tile_partials = reinterpret_cast<double*>(base + L.tile_partials);
+    // The combine's completion counter must start at zero: cleared on every
+    // call (a device-side memset, no host copy).  Every other scratch word
+    // the kernels read is written earlier in this call (one partial per
+    // tile, the group totals, the coefficient).
+    uint32_t* d_ticket = reinterpret_cast<uint32_t*>(base + L.ticket);
+    if (cudaMemsetAsync(d_ticket, 0, sizeof(uint32_t), s) != cudaSuccess) return ZR_ERR_CUDA;
     float* d_coef = reinterpret_cast<float*>(base + L.clip_coef);
-    double* d_own = reinterpret_cast<double*>(base + L.own_sumsq);
-    a.tile_partials = d_tile_partials;
+    a.tile_partials = reinterpret_cast<double*>(base + L.tile_partials);
     if (zr::launch_tiles(zr::Pass::kSumsq, a, grad_ptrs, false, false, s) != cudaSuccess) return ZR_ERR_CUDA;
-    if (zr::launch_clip_combine(d_tile_partials, a.n_tiles, d_sumsq_partials, p->world_size, p->rank,
-                                p->hp.max_grad_norm, d_coef, d_own, s) != cudaSuccess)
-        return ZR_ERR_CUDA;
+    zr::ClipArgs c{};
+    c.tile_partials = a.tile_partials;
+    c.n_tiles = a.n_tiles;
+    c.world_size = p->world_size;
+    c.ticket = d_ticket;
+    c.group_sums = reinterpret_cast<double*>(base + L.group_sums);
+    c.partials_all = d_sumsq_partials;
+    c.sumsq_out = reinterpret_cast<double*>(base + L.own_sumsq);
+    c.coef_out = d_coef;
+    c.rank = p->rank;
+    c.max_norm = p->hp.max_grad_norm;
+    if (zr::launch_clip_combine(c, s) != cudaSuccess) return ZR_ERR_CUDA;
     a.clip_coef = d_coef;
+    a.reverse = 1;
     return zr::launch_tiles(zr::Pass::kStepClip, a, grad_ptrs, false, false, s) == cudaSuccess ? ZR_OK : ZR_ERR_CUDA;
 }

@@ -52,9 +52,9 @@ class ZrPlan:
 
     def __init__(self, shapes, world_size, rank, mode=ZR_PARTITION_FLAT, bucket_cap_bytes=25 << 20,
                  lr=3e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.1, max_grad_norm=0.0,
-                 device=None, stream=None, bind=True):
+                 device=None, stream=None, bind=True, groups=None):
         self.handle = zr_plan_create(shapes, world_size, rank, mode, bucket_cap_bytes, lr, beta1,
-                                     beta2, eps, weight_decay, max_grad_norm)
+                                     beta2, eps, weight_decay, max_grad_norm, groups=groups)
         self.world_size = world_size
         self.rank = rank
         self.mode = mode

@@ -48,8 +48,8 @@ def test_status_strings():
     assert "unknown" in zr.zr_status_string(99)
 
 
-def lib_plan_table(shapes, W, rank, mode, cap):
-    h = zr.zr_plan_create(shapes, W, rank, mode, cap)
+def lib_plan_table(shapes, W, rank, mode, cap, groups=None):
+    h = zr.zr_plan_create(shapes, W, rank, mode, cap, groups=groups)
     try:
         segs = zr.zr_plan_segments(h)
         info = zr.zr_plan_query(h)
@@ -58,15 +58,15 @@ def lib_plan_table(shapes, W, rank, mode, cap):
     return [tuple(s[f] for f in FIELDS) for s in segs], info
 
 
-def oracle_table(shapes, W, mode, cap):
-    p = oracle.Plan(shapes, W, mode, cap)
+def oracle_table(shapes, W, mode, cap, groups=None):
+    p = oracle.Plan(shapes, W, mode, cap, groups=groups)
     return [tuple(int(s[f]) for f in FIELDS) for s in p.segments], p
 
 
-def assert_tables_equal(shapes, W, mode, cap):
-    want, p = oracle_table(shapes, W, mode, cap)
+def assert_tables_equal(shapes, W, mode, cap, groups=None):
+    want, p = oracle_table(shapes, W, mode, cap, groups)
     for rank in sorted({0, W - 1, W // 2}):
-        got, info = lib_plan_table(shapes, W, rank, mode, cap)
+        got, info = lib_plan_table(shapes, W, rank, mode, cap, groups)
         assert got == want
         assert info["total_numel"] == p.total_numel
         assert info["padded_numel"] == p.padded_numel
@@ -77,7 +77,7 @@ def assert_tables_equal(shapes, W, mode, cap):
 
 @pytest.mark.parametrize("g", all_golden_plans(), ids=lambda g: g["name"])
 def test_tables_match_hand_derived(g):
-    got, info = lib_plan_table(g["shapes"], g["world_size"], 0, g["mode"], g["cap_bytes"])
+    got, info = lib_plan_table(g["shapes"], g["world_size"], 0, g["mode"], g["cap_bytes"], g["groups"])
     assert got == g["segments"]
     assert (info["total_numel"], info["padded_numel"], info["n_buckets"]) == (g["N"], g["padded"], g["n_buckets"])
 
@@ -102,6 +102,40 @@ def test_tables_match_oracle_random():
         mode = int(rng.integers(0, 2))
         cap = int(rng.integers(0, 300))
         assert_tables_equal(shapes, W, mode, cap)
+
+
+def test_grouped_tables_match_oracle_random():
+    """Buckets given by tensor groups (one per layer): the library's tables
+    equal the oracle's bit for bit on random sets, and on the GPT-2 set
+    grouped by block (embeddings, 12 blocks, final norm)."""
+    rng = np.random.default_rng(23)
+    for _ in range(300):
+        nt = int(rng.integers(0, 10))
+        shapes = [tuple(int(x) for x in rng.integers(0, 30, size=int(rng.integers(0, 3))))
+                  for _ in range(nt)]
+        groups = np.cumsum(rng.integers(0, 2, size=nt)).tolist()
+        assert_tables_equal(shapes, int(rng.integers(1, 12)), int(rng.integers(0, 2)), 0, groups)
+    shapes = synth.gpt2_small_shapes()
+    groups = [0, 0] + [1 + i // 12 for i in range(12 * 12)] + [13, 13]
+    for mode in (0, 1):
+        assert_tables_equal(shapes, 8, mode, 0, groups)
+        h = zr.zr_plan_create(shapes, 8, 0, mode, 0, groups=groups)
+        assert zr.zr_plan_query(h)["n_buckets"] == 14
+        zr.zr_plan_destroy(h)
+
+
+def test_grouped_plan_argument_errors():
+    shapes = [(4,), (5,), (6,)]
+    with pytest.raises(zr.ZrError) as e:
+        zr.zr_plan_create(shapes, 2, 0, 0, 0, groups=[0, 1, 0])
+    assert e.value.status == zr.ZR_ERR_INVALID_ARG
+    hp = zr.zr_adamw(3e-4, 0.9, 0.999, 1e-8, 0.1, 0.0)
+    out = ctypes.c_void_p()
+    ndims = (ctypes.c_int32 * 3)(1, 1, 1)
+    dims = [(ctypes.c_int64 * 1)(n) for n in (4, 5, 6)]
+    ptrs = (ctypes.c_void_p * 3)(*[ctypes.addressof(d) for d in dims])
+    st = zr.raw_call("zr_plan_create_grouped", 3, ndims, ptrs, None, 2, 0, 0, ctypes.byref(hp), ctypes.byref(out))
+    assert st == zr.ZR_ERR_INVALID_ARG and not out.value
 
 
 def test_empty_parameter_set():
