@@ -84,6 +84,8 @@ def parse():
                     help="tensor set of --zero3 (gpt2: a small case, e.g. for profiling)")
     ap.add_argument("--checked", action="store_true",
                     help="checked mode: the device tile tables verified before every launch")
+    ap.add_argument("--no-alloc", action="store_true",
+                    help="step through zr_step_no_alloc (the library's static scratch, no workspace)")
     ap.add_argument("--sweep", action="store_true",
                     help="1.3B set: bucket cap x W x partition; one JSON record per point")
     ap.add_argument("--no-companions", action="store_true",
@@ -515,6 +517,8 @@ def measure_local(args, ctx, wl, with_e2e, with_cpu):
     my_buckets = sorted({s["bucket"] for s in plan.segments() if s["owner"] == zr_rank})
     if args.per_bucket:
         run_step = bound_bucket_steps(plan, my_buckets, grads, master, m, v, param_out, stream)
+    if args.no_alloc:
+        run_step = bound_no_alloc_steps(plan, grads, master, m, v, param_out, stream)
 
     for _ in range(args.warmup):
         step_no += 1
@@ -544,6 +548,8 @@ def measure_local(args, ctx, wl, with_e2e, with_cpu):
     # its average launch duration is this process's timed region / K; with
     # clipping the step's launches are taken together.
     bpp = bytes_per_owned_param(W, clip)
+    if args.no_alloc and clip and W > 4:
+        bpp = 2 * W + 26 + 2 * W        # pass 2 reads the gradients again instead of an fp32 copy
     alg_bytes = n * bpp
     avg_ms = local_ms / K
     achieved = alg_bytes / (avg_ms * 1e-3) / 1e9
@@ -551,7 +557,7 @@ def measure_local(args, ctx, wl, with_e2e, with_cpu):
     # (bucket-by-bucket or checked steps launch more kernels: no per-launch record)
     traffic = None
     traffic_note = None
-    if not (args.per_bucket or args.checked):
+    if not (args.per_bucket or args.checked or args.no_alloc):
         traffic, traffic_note = recorded_traffic(wl.name, clip, n)
 
     # the ceiling at this size: a plain device copy (torch) moving the step's
@@ -618,7 +624,7 @@ def measure_local(args, ctx, wl, with_e2e, with_cpu):
                    "partition": "flat" if wl.mode == 0 else "whole_tensor",
                    "bucket_cap_mb": wl.bucket_cap_mb, "clip": clip, "owned_params": n,
                    "per_bucket": bool(args.per_bucket), "buckets_stepped": len(my_buckets),
-                   "checked": bool(args.checked),
+                   "checked": bool(args.checked), "no_alloc": bool(args.no_alloc),
                    "bytes_per_owned_param": bpp,
                    "l2": f"no flush: each step touches {alg_bytes / 1e6:.0f} MB > 126 MB L2"},
         "hbm_gbs": achieved,
@@ -756,6 +762,25 @@ def measure_peer(args, ctx):
     del master, m, v
     torch.cuda.empty_cache()
     return entry
+
+
+def bound_no_alloc_steps(plan, grads, master, m, v, param_out, stream):
+    """f(step): zr_step_no_alloc on fixed buffers, arguments marshalled once
+    (its scratch is the library's static array; the plan's partials array,
+    if any, is passed as the sums-of-squares array)."""
+    from sharded_optimizer_step_zr_b200 import _addr, _check, _lib, _ptr_array, _stream
+    arr = _ptr_array(grads)
+    args = (plan.handle, arr, _addr(master), _addr(m), _addr(v), _addr(param_out),
+            _addr(plan.partials) if plan.partials is not None else None)
+    s = _stream(stream)
+    fn = _lib.zr_step_no_alloc
+
+    def step_fn(step):
+        st = fn(*args, step, s)
+        if st:
+            _check(st, "zr_step_no_alloc")
+    step_fn._keepalive = (arr, grads, master, m, v, param_out)
+    return step_fn
 
 
 def run_zr(args):
@@ -1046,12 +1071,14 @@ def run_zero3(args):
         with torch.cuda.graph(g, stream=s):
             for _ in range(reps):
                 fn()
-        g.replay()
+        with torch.cuda.stream(s):                     # replay() launches on the current stream
+            g.replay()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(s)
-        g.replay()
-        e1.record(s)
+        with torch.cuda.stream(s):
+            e0.record(s)
+            g.replay()
+            e1.record(s)
         torch.cuda.synchronize()
         del g
         return e0.elapsed_time(e1) / reps * 1e3
@@ -1149,11 +1176,14 @@ def run_zero3(args):
 def run_zero3_train(args):
     """Training steps of a stack of MLP blocks (12 x [Linear(d, 4d), GELU,
     Linear(4d, d)], d = 2048: 403 M bf16 parameters; 4096 tokens) with
-    ZeroAdamW (every parameter resident) and with Zero3 (each layer
-    gathered from the shard before its forward and again before its
-    backward, the next layer's forward gather prefetched), one rank.  Both
-    take the same steps (checked); the difference in step time is what the
-    layer loop costs on one GPU.  Prints one JSON record."""
+    ZeroAdamW (every parameter resident), with Zero3 (each layer gathered
+    from the shard before its forward and again before its backward, the
+    next layer's forward gather prefetched) and with Zero3's
+    reduce_in_backward (each layer's gradients reduced and applied as its
+    backward ends, two layer-sized gradient slots instead of a full
+    gradient buffer), one rank.  All take the same steps (checked); the
+    differences in step time are what the layer loop costs on one GPU.
+    Prints one JSON record."""
     import torch
     from sharded_optimizer_step_zr_b200.optim import Zero3, ZeroAdamW
     torch.cuda.set_device(0)
@@ -1167,11 +1197,12 @@ def run_zero3_train(args):
             layers += [torch.nn.Linear(d, 4 * d), torch.nn.GELU(), torch.nn.Linear(4 * d, d)]
         return torch.nn.Sequential(*layers).to(dev).to(torch.bfloat16)
 
-    a, b, c = model(1), model(1), model(1)
+    a, b, c, e = model(1), model(1), model(1), model(1)
     n_params = sum(p.numel() for p in a.parameters())
     z2 = ZeroAdamW(list(a.parameters()), lr=1e-4)
     z3 = Zero3(b, lr=1e-4)
     z3_fwd_only = Zero3(c, lr=1e-4, backward_prefetch=False)
+    z3_rib = Zero3(e, lr=1e-4, reduce_in_backward=True)
     x = torch.randn(tokens, d, device=dev, dtype=torch.bfloat16)
 
     def step(m, opt):
@@ -1194,20 +1225,28 @@ def run_zero3_train(args):
     t2 = timed(a, z2, 5)
     t3 = timed(b, z3, 5)
     t3f = timed(c, z3_fwd_only, 5)
+    t3r = timed(e, z3_rib, 5)
     full = torch.empty(n_params, dtype=torch.bfloat16, device=dev)
     z3.gather_all(full)
     resident = torch.cat([p.detach().reshape(-1) for p in a.parameters()])
     same = bool(torch.equal(full.view(torch.int16), resident.view(torch.int16)))
+    full_r = torch.empty(n_params, dtype=torch.bfloat16, device=dev)
+    z3_rib.gather_all(full_r)
+    same_rib = bool(torch.equal(full.view(torch.int16), full_r.view(torch.int16)))
     flops = 6 * tokens * n_params
     line = {"mode": "zero3_train", "params": n_params, "tokens": tokens, "blocks": n_blocks, "unit": "ms",
             "zero_adamw_step_ms": t2, "zero3_step_ms": t3, "layer_loop_overhead_ms": t3 - t2,
             "zero3_forward_prefetch_only_step_ms": t3f,
             "gathers_per_step": 2 * len(z3.units), "gathered_bytes_per_step": 2 * 2 * n_params,
-            "model_tflops_zero_adamw": flops / (t2 * 1e-3) / 1e12, "same_parameters": same}
+            "model_tflops_zero_adamw": flops / (t2 * 1e-3) / 1e12, "same_parameters": same,
+            "zero3_reduce_in_backward_step_ms": t3r, "reduce_in_backward_same_parameters": same_rib,
+            "gradient_bytes": {"zero3": 2 * z3.grad_buffer.numel(),
+                               "zero3_reduce_in_backward": 2 * sum(g.numel() for g in z3_rib.grad_slots)}}
     print(json.dumps(line), flush=True)
     z2.close()
     z3.close()
     z3_fwd_only.close()
+    z3_rib.close()
 
 
 def run_vs_torch(args):

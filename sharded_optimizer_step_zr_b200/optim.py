@@ -160,6 +160,55 @@ class ZeroAdamW:
             self.plan.close()
 
 
+def unit_grad_layout(segments, first, count, last_unit, world_size):
+    """Where one unit's (tensors first .. first + count - 1) gradients sit in
+    a gradient slot.  Each owner's elements of the unit are one run in its
+    owned order; the slot holds those runs owner by owner, each starting at
+    its owned offset's phase mod 8, so that for every rank r there is an
+    offset d_r with replica w's slot + d_r serving as r's grad_ptrs[w] for
+    the unit's tiles (slot element d_r + owned offset, 16-byte aligned).  The
+    last unit's run also covers the flat zero pad (its bucket holds it).
+
+    Returns (pieces of each tensor as (offset in tensor, slot offset,
+    length), d_r per rank, slot elements used).  A tensor whose pieces are
+    contiguous in the slot can be one .grad view of it; with a flat chunk
+    that is a multiple of 8 elements (or one rank) every tensor is."""
+    segs = [s for s in segments
+            if first <= s["tensor"] < first + count or (last_unit and s["tensor"] == -1)]
+    pieces = {t: [] for t in range(first, first + count)}
+    ptr_off = [0] * world_size
+    cursor = 0
+    for r in range(world_size):
+        mine = sorted((s["owned_offset"], s["tensor"], s["offset_in_tensor"], s["length"])
+                      for s in segs if s["owner"] == r)
+        if not mine:
+            continue
+        lo = mine[0][0]
+        hi = mine[-1][0] + mine[-1][3]
+        base = (cursor + 7) // 8 * 8 + lo % 8
+        for o, t, off, n in mine:
+            if t >= 0:
+                pieces[t].append((off, base + (o - lo), n))
+        ptr_off[r] = base - lo
+        cursor = base + (hi - lo)
+    for t in pieces:
+        pieces[t].sort()
+    return pieces, ptr_off, cursor
+
+
+def contiguous_in_slot(pieces):
+    """Slot offset of a tensor whose pieces (sorted by offset in the tensor)
+    follow each other in the slot from its first element, else None."""
+    if not pieces:
+        return 0
+    if pieces[0][0] != 0:
+        return None
+    for (off, pos, n), (off2, pos2, _) in zip(pieces, pieces[1:]):
+        if off2 != off + n or pos2 != pos + n:
+            return None
+    return pieces[0][1]
+
+
 class Zero3:
     """ZeRO stage 3 for a torch module ("Scaling training to thousands of
     GPUs", talk summary, section 11:24 ZeRO; "CS336 lecture 8", section
@@ -184,10 +233,24 @@ class Zero3:
 
         z = Zero3(model, group=None, lr=3e-4)
         loss = model(x).sum(); loss.backward(); z.step(); z.zero_grad()
+
+    reduce_in_backward=True is the gradient side of stage 3: no replica
+    keeps its whole gradient.  The plan's buckets are the units (one per
+    module), gradients accumulate into two rotating gradient slots (module
+    i: slot i mod 2, laid out so every owner's part is one run), and as
+    soon as a module's gradients are complete the fused step reduces that
+    module's slice from every replica's slot (through peer memory across
+    processes) and updates it -- zr_step_bucket on the module's bucket --
+    after which the slot is cleared for module i - 2.  z.step() then only
+    steps modules that received no gradient and advances the count.  One
+    backward per step (no accumulation over several), every parameter of a
+    module receiving a gradient, and no clipping (the norm needs every
+    layer's gradient before the first update).
     """
 
     def __init__(self, module, group=None, lr=3e-4, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.1,
-                 max_grad_norm=0.0, partition="flat", bucket_cap_mb=25, backward_prefetch=True):
+                 max_grad_norm=0.0, partition="flat", bucket_cap_mb=25, backward_prefetch=True,
+                 reduce_in_backward=False):
         import torch
         from . import ZR_PARAMS_OWNED
         self.module = module
@@ -222,21 +285,52 @@ class Zero3:
         if group is not None:
             import torch.distributed as dist
             world = dist.get_world_size(group)
+        self.reduce_in_backward = bool(reduce_in_backward)
+        groups = None
+        slot_elems = 0
+        if self.reduce_in_backward:
+            if max_grad_norm > 0:
+                raise ValueError("reduce_in_backward: clipping needs every layer's gradient before any update")
+            groups = [0] * len(params)
+            for u, (_, a, k) in enumerate(self.units):
+                for t in range(a, a + k):
+                    groups[t] = u
+            # the units' gradient layouts, from the host-only plan (same tables on every rank)
+            from .plan import ZrPlan
+            probe = ZrPlan(shapes, world, 0, mode, cap, *hp, bind=False, groups=groups)
+            segs = probe.segments()
+            probe.close()
+            self._unit_layouts = [unit_grad_layout(segs, a, k, a + k == len(params), world)
+                                  for _, a, k in self.units]
+            self._unit_bucket = []
+            for _, a, k in self.units:
+                bs = {s["bucket"] for s in segs if a <= s["tensor"] < a + k}
+                self._unit_bucket.append(bs.pop() if bs else None)
+            slot_elems = max(8, max(L[2] for L in self._unit_layouts))
         if world > 1:
             from .peer import PeerZero
-            self.peer = PeerZero(group, shapes, mode, cap, *hp, device=dev, stage=3)
+            self.peer = PeerZero(group, shapes, mode, cap, *hp, device=dev, stage=3, groups=groups,
+                                 grad_slot_elems=slot_elems)
             self.plan = self.peer.plan
             self.grad_buffer = self.peer.grad_buffer
             self.offsets = self.peer.offsets
             self.shard = self.peer.param_shard
             shard_ptrs = self.peer.shard_ptrs
+            if self.reduce_in_backward:
+                self.grad_slots = self.peer.grad_slots
+                self._slot_bases = self.peer.grad_slot_bases            # [w][slot] byte addresses
         else:
             from .plan import ZrPlan
             self.peer = None
-            self.plan = ZrPlan(shapes, 1, 0, mode, cap, *hp, device=dev)
+            self.plan = ZrPlan(shapes, 1, 0, mode, cap, *hp, device=dev, groups=groups)
             self.plan.set_param_layout(ZR_PARAMS_OWNED)
             self.offsets = [0, self.plan.padded_numel]
-            self.grad_buffer = torch.zeros(max(self.plan.padded_numel, 8), dtype=torch.bfloat16, device=dev)
+            if self.reduce_in_backward:
+                self.grad_buffer = None
+                self.grad_slots = [torch.zeros(slot_elems, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+                self._slot_bases = [[g.data_ptr() for g in self.grad_slots]]
+            else:
+                self.grad_buffer = torch.zeros(max(self.plan.padded_numel, 8), dtype=torch.bfloat16, device=dev)
             self.shard = torch.zeros(max(self.plan.owned_numel, 8), dtype=torch.bfloat16, device=dev)
             shard_ptrs = [self.shard]
         # this rank's shard and fp32 state from the current (whole) parameters
@@ -274,10 +368,14 @@ class Zero3:
         self.back_ready = [torch.cuda.Event() for _ in self.units]
         self._back_prefetched = [False] * len(self.units)
         self.backward_prefetch = backward_prefetch
-        # gradients: as ZeroAdamW
-        segs = self.plan.segments()
         self.params = params
         self._bound, self._copy_in = [], []
+        if self.reduce_in_backward:
+            self._bind_grad_slots()
+            self.step_count = 0
+            return
+        # gradients: as ZeroAdamW
+        segs = self.plan.segments()
         for t, p in enumerate(params):
             pieces = sorted((s["offset_in_tensor"], s["owner"], s["owned_offset"], s["length"])
                             for s in segs if s["tensor"] == t)
@@ -290,6 +388,81 @@ class Zero3:
                 p.grad = torch.zeros_like(p)
                 self._copy_in.append((p, [(off, self.offsets[r] + o, n_) for off, r, o, n_ in pieces]))
         self.step_count = 0
+
+    def _bind_grad_slots(self):
+        """reduce_in_backward: every parameter's .grad a view of its unit's
+        slot; hooks that fire once a unit's gradients are all accumulated."""
+        import torch
+        W, me = self.plan.world_size, self.plan.rank
+        self._unit_grad_ptrs = []
+        self._unit_grad_views = []
+        for u, (_, a, k) in enumerate(self.units):
+            pieces, ptr_off, used = self._unit_layouts[u]
+            slot = self.grad_slots[u % 2]
+            views = []
+            for t in range(a, a + k):
+                p = self.params[t]
+                at = contiguous_in_slot(pieces[t])
+                if at is not None:
+                    v = slot[at:at + p.numel()].view(p.shape)
+                    p.grad = v
+                    views.append((p, v, None))
+                else:
+                    # split across two owners' runs that do not meet: its own .grad, copied in
+                    p.grad = torch.zeros_like(p)
+                    views.append((p, None, [(off, slot[pos:pos + n]) for off, pos, n in pieces[t]]))
+            self._unit_grad_views.append(views)
+            self._unit_grad_ptrs.append([self._slot_bases[w][u % 2] + 2 * ptr_off[me] for w in range(W)])
+            for p in [self.params[t] for t in range(a, a + k)]:
+                self._hooks.append(p.register_post_accumulate_grad_hook(self._make_grad_hook(u, p)))
+        self._unit_seen = [set() for _ in self.units]
+        self._unit_done = [False] * len(self.units)
+
+    def _make_grad_hook(self, u, param):
+        def hook(p):
+            if self._unit_done[u]:
+                raise RuntimeError("reduce_in_backward: a second backward before step(); "
+                                   "gradients cannot be accumulated over several passes in this mode")
+            self._unit_seen[u].add(id(param))
+            if len(self._unit_seen[u]) == len(self._unit_grad_views[u]):
+                self._reduce_unit(u)
+        return hook
+
+    def _reduce_unit(self, u):
+        """Unit u's gradients are complete on this replica: (every replica's,
+        across processes) reduce its slice and update it, then clear the slot."""
+        import torch
+        from . import zr_step_bucket
+        from .peer import sync_point
+        cur = torch.cuda.current_stream()
+        t = self.step_count + 1
+        for p, v, split in self._unit_grad_views[u]:
+            if split is not None:
+                g = p.grad.reshape(-1) if p.grad is not None else None
+                for off, dst in split:
+                    if g is None:
+                        dst.zero_()
+                    else:
+                        dst.copy_(g[off:off + dst.numel()])
+                if p.grad is not None:
+                    p.grad.zero_()
+                continue
+            if p.grad is None:
+                v.zero_()
+            elif p.grad.data_ptr() != v.data_ptr():        # autograd replaced the view: copy in
+                v.copy_(p.grad)
+            p.grad = v
+        if self.peer is not None:
+            cur.synchronize()                              # this replica's gradients are written
+            sync_point(self.peer.dist, self.peer.group, f"layer {u} gradients ready", t)
+        if self._unit_bucket[u] is not None:
+            zr_step_bucket(self.plan.handle, self._unit_bucket[u], self._unit_grad_ptrs[u], self.master, self.m,
+                           self.v, self.shard, t, cur)
+        if self.peer is not None:
+            cur.synchronize()
+            sync_point(self.peer.dist, self.peer.group, f"layer {u} reduced", t)   # no rank reads the slot now
+        self.grad_slots[u % 2][:self._unit_layouts[u][2]].zero_()
+        self._unit_done[u] = True
 
     def _gather(self, u, stream):
         # one bound call per (unit, stream): the arguments are marshalled once
@@ -337,7 +510,10 @@ class Zero3:
         return hook
 
     def zero_grad(self, set_to_none=False):
-        """Zeroes the gradient buffer (the .grad views stay bound)."""
+        """Zeroes the gradient buffer (the .grad views stay bound); with
+        reduce_in_backward the slots are already clear after each unit."""
+        if self.reduce_in_backward:
+            return
         self.grad_buffer.zero_()
         for p, _ in self._copy_in:
             p.grad.zero_()
@@ -349,8 +525,24 @@ class Zero3:
 
     def step(self):
         """One optimizer step (every rank together): the rank's slice of the
-        averaged gradient, AdamW, the bf16 result into the rank's shard."""
+        averaged gradient, AdamW, the bf16 result into the rank's shard.
+        With reduce_in_backward the backward has stepped every unit that got
+        gradients: the rest are stepped here (zero gradient)."""
         from . import zr_step
+        if self.reduce_in_backward:
+            for u in range(len(self.units)):
+                if self._unit_done[u]:
+                    continue
+                if self._unit_seen[u]:
+                    raise RuntimeError(f"reduce_in_backward: module {u} received gradients for only some "
+                                       "of its parameters")
+                self._reduce_unit(u)
+            self.step_count += 1
+            self._unit_seen = [set() for _ in self.units]
+            self._unit_done = [False] * len(self.units)
+            self._prefetched = [False] * len(self.units)
+            self._back_prefetched = [False] * len(self.units)
+            return
         flat_grad = self.grad_buffer.view(-1)
         for p, start in self._bound:
             view = flat_grad[start:start + p.numel()]

@@ -10,7 +10,10 @@ the per-rank sums of squares.
 
 Every replica keeps its full gradient in the plan's owner-major layout
 (``grad_view(t)`` is tensor t's slice of it, for the backward pass to write
-into).  Stages 1 and 2: ``param_buffer`` holds the full bf16 parameters in
+into) -- or, for the stage-3 layer loop with grad_slot_elems, only two
+rotating gradient slots of one layer each (``grad_slots``; every replica's
+slot j at byte address ``grad_slot_bases[w][j]``), which the caller lays
+out and steps layer by layer with zr_step_bucket on a grouped plan.  Stages 1 and 2: ``param_buffer`` holds the full bf16 parameters in
 the global layout, written by every rank's step.  Stage 3: each rank keeps
 only ``param_shard``, its bf16 parameters in owned order, and ``gather``
 assembles whole tensors (one layer, ahead of its use) from every rank's
@@ -49,30 +52,36 @@ class PeerZero:
 
     def __init__(self, group, shapes, mode=ZR_PARTITION_FLAT, bucket_cap_bytes=25 << 20, lr=3e-4,
                  beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.1, max_grad_norm=0.0, device=None,
-                 stage=2):
+                 stage=2, groups=None, grad_slot_elems=0):
         import torch
         import torch.distributed as dist
         if stage not in (1, 2, 3):
             raise ValueError("stage is 1, 2 or 3")
+        if grad_slot_elems and stage != 3:
+            raise ValueError("gradient slots are the stage-3 layer loop's")
         self.dist, self.group, self.stage = dist, group, stage
         self.world_size = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
         device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
         self.device = device
         self.plan = ZrPlan(shapes, self.world_size, self.rank, mode, bucket_cap_bytes, lr, beta1, beta2,
-                           eps, weight_decay, max_grad_norm, device=device)
+                           eps, weight_decay, max_grad_norm, device=device, groups=groups)
         self.offsets = zr_plan_owner_offsets(self.plan.handle, self.world_size)
         P = self.plan.padded_numel
         # One allocation holds both shared buffers, so each peer maps one
-        # IPC handle per rank: the gradient buffer, then (256-byte aligned)
-        # the full parameter buffer (stages 1, 2) or this rank's parameter
-        # shard (stage 3).  The gradient part has the same size on every
-        # rank, so the second part starts at the same offset everywhere.
+        # IPC handle per rank: the gradient buffer -- or, with
+        # grad_slot_elems, two rotating gradient slots of that many elements
+        # (one layer's gradients at a time) -- then (256-byte aligned) the
+        # full parameter buffer (stages 1, 2) or this rank's parameter shard
+        # (stage 3).  The gradient part has the same size on every rank, so
+        # the second part starts at the same offset everywhere.
         round128 = lambda x: max(128, (x + 127) // 128 * 128)
-        half = round128(max(P, self.offsets[-1]))
+        slot = round128(grad_slot_elems) if grad_slot_elems else 0
+        half = 2 * slot if grad_slot_elems else round128(max(P, self.offsets[-1]))
         second = round128(self.plan.owned_numel) if stage == 3 else half
         self._shared = torch.zeros(half + second, dtype=torch.bfloat16, device=device)
-        self.grad_buffer = self._shared[:half]
+        self.grad_buffer = None if grad_slot_elems else self._shared[:half]
+        self.grad_slots = [self._shared[:slot], self._shared[slot:2 * slot]] if grad_slot_elems else None
         everyone = [None] * self.world_size
         dist.all_gather_object(everyone, zr_ipc_export(self._shared), group=group)
         self._opened = []
@@ -84,7 +93,9 @@ class PeerZero:
             grad_bases.append(base)
             second_bases.append(base + 2 * half)
         start = 2 * self.offsets[self.rank]                 # bytes: bf16 elements
-        self.grad_ptrs = [b + start for b in grad_bases]
+        self.grad_ptrs = None if grad_slot_elems else [b + start for b in grad_bases]
+        # with slots: every replica's slot j starts at byte grad_slot_bases[w][j]
+        self.grad_slot_bases = [[b, b + 2 * slot] for b in grad_bases] if grad_slot_elems else None
         if stage == 3:
             self.param_shard = self._shared[half:half + self.plan.owned_numel]
             self.shard_ptrs = second_bases

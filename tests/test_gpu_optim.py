@@ -204,3 +204,47 @@ def test_zero3_accumulation_and_evaluation():
         assert np.array_equal(full.cpu().view(torch.int16).numpy(), flat_u16(a.parameters()).view(np.int16)), t
     z2.close()
     z3.close()
+
+
+@pytest.mark.parametrize("partition", ["flat", "whole"])
+def test_zero3_reduce_in_backward_takes_the_same_steps(partition):
+    """The gradient side of stage 3: each module's gradients accumulate into
+    one of two rotating slots and are reduced and applied (zr_step_bucket on
+    the module's bucket) as soon as the module's backward is done; no
+    full-model gradient buffer exists.  Three steps equal Zero3's ordinary
+    step (and so ZeroAdamW's) bit for bit, weights and losses; a second
+    backward before step() is refused."""
+    from sharded_optimizer_step_zr_b200.optim import Zero3
+    a, b = make_deep_model(8), make_deep_model(8)
+    za = Zero3(a, lr=1e-3, partition=partition)
+    zb = Zero3(b, lr=1e-3, partition=partition, reduce_in_backward=True)
+    assert zb.grad_buffer is None and len(zb.grad_slots) == 2
+    big = max(sum(p.numel() for p in m.parameters(recurse=False)) for m in b.modules())
+    assert all(s.numel() <= big + 8 for s in zb.grad_slots)     # one module's gradients per slot
+    N = sum(p.numel() for p in a.parameters())
+    gen = torch.Generator(device=DEV).manual_seed(23)
+    for t in (1, 2, 3):
+        x = torch.randn(32, 64, device=DEV, generator=gen).to(torch.bfloat16)
+        la = a(x).float().pow(2).mean()
+        la.backward()
+        za.step()
+        za.zero_grad()
+        lb = b(x).float().pow(2).mean()
+        lb.backward()
+        zb.step()
+        zb.zero_grad()
+        torch.cuda.synchronize()
+        assert la.item() == lb.item(), t
+        fa = torch.empty(N, dtype=torch.bfloat16, device=DEV)
+        fb = torch.empty(N, dtype=torch.bfloat16, device=DEV)
+        za.gather_all(fa)
+        zb.gather_all(fb)
+        torch.cuda.synchronize()
+        assert torch.equal(fa.view(torch.int16), fb.view(torch.int16)), t
+        assert all(not s.view(torch.int16).any() for s in zb.grad_slots)   # cleared after every module
+    x = torch.randn(32, 64, device=DEV, generator=gen).to(torch.bfloat16)
+    b(x).float().pow(2).mean().backward()
+    with pytest.raises(RuntimeError, match="second backward"):
+        b(x).float().pow(2).mean().backward()
+    za.close()
+    zb.close()

@@ -252,11 +252,14 @@ def test_zero_adamw_two_processes():
     assert all(p.exitcode == 0 for p in procs)
 
 
-def _rank_main_zero3(rank, world, port, q):
+def _rank_main_zero3(rank, world, port, q, partition="flat"):
     """Zero3 over a two-process group: parameters gathered from both ranks'
     shards (one through IPC) before each module's forward and backward;
     after every step the gathered model equals the oracle's unsharded step
-    on the two replicas' gradients."""
+    on the two replicas' gradients.  Beside it, on a copy of the model, the
+    same job with reduce_in_backward (each module's slice reduced from both
+    replicas' gradient slots through IPC and applied during the backward):
+    its gathered model equals the first one bit for bit after every step."""
     import sys
     sys.path.insert(0, ROOT)
     os.environ["MASTER_ADDR"] = "127.0.0.1"
@@ -276,8 +279,15 @@ def _rank_main_zero3(rank, world, port, q):
             .view(np.uint16).copy()
         init = flat(model.parameters())
         hp = (1e-3, 0.9, 0.999, 1e-8, 0.1, 0.0)
-        z = Zero3(model, group=dist.group.WORLD, lr=hp[0], weight_decay=hp[4], bucket_cap_mb=0.01)
+        torch.manual_seed(6)
+        model2 = torch.nn.Sequential(torch.nn.Linear(64, 128), torch.nn.GELU(), torch.nn.Linear(128, 96),
+                                     torch.nn.LayerNorm(96), torch.nn.Linear(96, 24)).to("cuda:0").to(torch.bfloat16)
+        z = Zero3(model, group=dist.group.WORLD, lr=hp[0], weight_decay=hp[4], bucket_cap_mb=0.01,
+                  partition=partition)
+        z2 = Zero3(model2, group=dist.group.WORLD, lr=hp[0], weight_decay=hp[4], partition=partition,
+                   reduce_in_backward=True)
         N = init.size
+        full2 = torch.empty(N, dtype=torch.bfloat16, device="cuda:0")
         o_master = (init.astype(np.uint32) << 16).view(np.float32).copy()
         o_m, o_v, o_out = np.zeros(N, np.float32), np.zeros(N, np.float32), np.zeros(N, np.uint16)
         gen = torch.Generator(device="cuda:0").manual_seed(300 + rank)
@@ -294,11 +304,16 @@ def _rank_main_zero3(rank, world, port, q):
             z.step()
             z.zero_grad()
             z.gather_all(full)
+            model2(x).float().pow(2).mean().backward()
+            z2.step()
+            z2.gather_all(full2)
             torch.cuda.synchronize()
             ok = ok and bool(np.array_equal(full.cpu().view(torch.int16).numpy().view(np.uint16), o_out))
+            ok = ok and bool(torch.equal(full.view(torch.int16), full2.view(torch.int16)))
         q.put((rank, ok))
         dist.barrier()
         z.close()
+        z2.close()
     except Exception as e:
         q.put((rank, "error", repr(e)))
         raise
@@ -306,11 +321,12 @@ def _rank_main_zero3(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_zero3_module_two_processes():
+@pytest.mark.parametrize("partition", ["flat", "whole"])
+def test_zero3_module_two_processes(partition):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _port()
-    procs = [ctx.Process(target=_rank_main_zero3, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_rank_main_zero3, args=(r, 2, port, q, partition)) for r in range(2)]
     for p in procs:
         p.start()
     results = [q.get(timeout=240) for _ in range(2)]
