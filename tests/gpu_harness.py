@@ -24,11 +24,11 @@ def bits32(a) -> np.ndarray:
 class GpuRank:
     """One rank's plan and device buffers."""
 
-    def __init__(self, shapes, W, rank, mode, cap, hp, seed, max_grad_norm=None):
+    def __init__(self, shapes, W, rank, mode, cap, hp, seed, max_grad_norm=None, groups=None):
         lr, b1, b2, eps, wd, mgn = hp
         if max_grad_norm is not None:
             mgn = max_grad_norm
-        self.plan = ZrPlan(shapes, W, rank, mode, cap, lr, b1, b2, eps, wd, mgn, device=DEV)
+        self.plan = ZrPlan(shapes, W, rank, mode, cap, lr, b1, b2, eps, wd, mgn, device=DEV, groups=groups)
         self.W, self.rank, self.seed = W, rank, seed
         n = self.plan.owned_numel
         self.runs = self.plan.runs()

@@ -25,19 +25,27 @@ def bucket_owned_ranges(plan, bucket):
             if s["owner"] == plan.rank and s["bucket"] == bucket]
 
 
-@pytest.mark.parametrize("shapes, W, rank, mode, cap, max_norm", [
-    (synth.gpt2_small_shapes()[:26], 8, 0, 0, 1 << 20, 0.0),          # flat, many buckets
-    ([(4096 * 3 + 5,), (17,), (1,), (300, 7)], 3, 1, 0, 9000, 0.0),    # ragged tiles, pad
-    ([(1000, 3), (8191,), (9, 9), (2048,)], 4, 2, 1, 4096, 0.0),       # whole-tensor
-    ([(3000, 7), (5001,), (64, 64), (129,)], 8, 3, 0, 8192, 0.05),    # clip, W > 4 (scratch)
-    ([(3000, 7), (5001,), (64, 64), (129,)], 8, 5, 1, 8192, 0.05),    # clip, whole-tensor
-    ([(3000, 7), (5001,), (64, 64), (129,)], 3, 1, 0, 8192, 0.05),    # clip, W <= 4 (re-read)
+GPT2_BLOCKS = [0, 0] + [1 + i // 12 for i in range(24)]      # the first 26 tensors: embeddings, 2 blocks
+
+
+@pytest.mark.parametrize("shapes, W, rank, mode, cap, max_norm, groups", [
+    (synth.gpt2_small_shapes()[:26], 8, 0, 0, 1 << 20, 0.0, None),          # flat, many buckets
+    ([(4096 * 3 + 5,), (17,), (1,), (300, 7)], 3, 1, 0, 9000, 0.0, None),    # ragged tiles, pad
+    ([(1000, 3), (8191,), (9, 9), (2048,)], 4, 2, 1, 4096, 0.0, None),       # whole-tensor
+    ([(3000, 7), (5001,), (64, 64), (129,)], 8, 3, 0, 8192, 0.05, None),    # clip, W > 4 (scratch)
+    ([(3000, 7), (5001,), (64, 64), (129,)], 8, 5, 1, 8192, 0.05, None),    # clip, whole-tensor
+    ([(3000, 7), (5001,), (64, 64), (129,)], 3, 1, 0, 8192, 0.05, None),    # clip, W <= 4 (re-read)
+    # buckets by tensor group (one per GPT-2 block): the per-layer reduce of ZeRO-3
+    (synth.gpt2_small_shapes()[:26], 8, 3, 0, 0, 0.0, GPT2_BLOCKS),
+    (synth.gpt2_small_shapes()[:26], 3, 1, 1, 0, 0.05, GPT2_BLOCKS),
 ])
-def test_buckets_equal_full_step(shapes, W, rank, mode, cap, max_norm):
+def test_buckets_equal_full_step(shapes, W, rank, mode, cap, max_norm, groups):
     hp = (3e-4, 0.9, 0.999, 1e-8, 0.1, max_norm)
-    full = GpuRank(shapes, W, rank, mode, cap, hp, seed=21)
-    byb = GpuRank(shapes, W, rank, mode, cap, hp, seed=21)
-    oplan = oracle.Plan(shapes, W, mode, cap)
+    full = GpuRank(shapes, W, rank, mode, cap, hp, seed=21, groups=groups)
+    byb = GpuRank(shapes, W, rank, mode, cap, hp, seed=21, groups=groups)
+    oplan = oracle.Plan(shapes, W, mode, cap, groups=groups)
+    if groups is not None:
+        assert byb.plan.n_buckets == len(set(groups))
     orc = OracleRank(oplan, rank, seed=21)
     P = oplan.padded_numel
     out_full = torch.zeros(P, dtype=torch.bfloat16, device=DEV)
