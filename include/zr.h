@@ -157,7 +157,8 @@ zr_status zr_plan_segments(const zr_plan* plan, zr_segment* out, int64_t cap, in
  * (one double per tile, one per group of 1024 tiles, and a completion
  * counter), a few scalars and status words, the ZeRO-3 gather
  * piece table (32 bytes per piece of at most 16384 elements, all ranks) and
- * (when clipping with W > 4) an fp32 scratch copy of the reduced gradient. */
+ * (when clipping with W > 4, or with a grouped plan) an fp32 scratch copy
+ * of the reduced gradient. */
 zr_status zr_plan_workspace_bytes(const zr_plan* plan, uint64_t* bytes);
 
 /* Bind a device workspace (>= zr_plan_workspace_bytes, 256-byte aligned,
@@ -246,9 +247,11 @@ zr_status zr_step_device_count(const zr_plan* plan, const void* const* grad_ptrs
  *   is elementwise).
  *   With clipping: the coefficient needs every bucket's sum of squares, so
  *   this runs the reduce and the sums of squares for the bucket (writing the
- *   fp32 averaged gradient to the workspace when W > 4; master, m, v and
+ *   fp32 averaged gradient to the workspace when W > 4 or the plan is
+ *   grouped; master, m, v and
  *   param_out are not touched and may be NULL); after every bucket,
- *   zr_step_finish updates all elements.  For W > 4 the bucket's gradient
+ *   zr_step_finish updates all elements.  For W > 4 (or a grouped plan)
+ *   the bucket's gradient
  *   buffers may be released as soon as this call's work is done.
  * Errors: as zr_step; ZR_ERR_INVALID_ARG for a bucket out of range. */
 zr_status zr_step_bucket(const zr_plan* plan, int32_t bucket, const void* const* grad_ptrs,
@@ -258,13 +261,26 @@ zr_status zr_step_bucket(const zr_plan* plan, int32_t bucket, const void* const*
 /* Completes a bucket-by-bucket step of a plan with clipping: the norm from
  * all buckets' sums of squares (and the other ranks' entries of the
  * partials array, as for zr_step), then the scaled AdamW update and bf16
- * cast of every owned element.  For W > 4 it reads the averaged gradient
- * that zr_step_bucket stored and grad_ptrs may be NULL; for W <= 4 it reads
+ * cast of every owned element.  For W > 4 (or a grouped plan) it reads the
+ * averaged gradient that zr_step_bucket stored and grad_ptrs may be NULL;
+ * otherwise it reads
  * the gradients again, so grad_ptrs must still hold every bucket's values.
  * For plans without clipping it does nothing and returns ZR_OK.  The result
  * equals zr_step's bit for bit. */
 zr_status zr_step_finish(const zr_plan* plan, const void* const* grad_ptrs, float* master, float* m,
                          float* v, void* param_out, int64_t step, zr_stream_t stream);
+
+/* Between a bucket-by-bucket pass and zr_step_finish, with clipping: this
+ * rank's S_r from the sums of squares zr_step_bucket left in the workspace
+ * (every bucket of the step called once), to the device double *d_out,
+ * without reading any gradient -- the value zr_step_finish will use for
+ * this rank, bit for bit.  Its purpose is the cross-rank exchange of a
+ * layer-by-layer step whose gradients are released as each layer is
+ * reduced (ZeRO-3): every rank calls it, the W values are all-gathered into
+ * the partials array, then zr_step_finish.  Errors: ZR_ERR_INVALID_ARG (no
+ * clipping, NULL), ZR_ERR_ALIGNMENT (d_out not 8-byte aligned),
+ * ZR_ERR_NO_WORKSPACE, ZR_ERR_CUDA. */
+zr_status zr_bucket_sumsq(const zr_plan* plan, double* d_out, zr_stream_t stream);
 
 /* zr_step with host-resident gradients and a host copy of the result, for
  * callers whose gradients arrive in host memory.  Copies host_grad_ptrs[w]

@@ -43,7 +43,7 @@ EXPORTED = [
     "zr_plan_set_workspace", "zr_plan_set_adamw", "zr_plan_set_device_lr", "zr_plan_set_sumsq_partials", "zr_step", "zr_step_device_count",
     "zr_step_bucket",
     "zr_step_finish", "zr_step_host",
-    "zr_grad_sumsq", "zr_debug_reduce", "zr_step_no_alloc", "zr_state_save", "zr_state_load",
+    "zr_grad_sumsq", "zr_bucket_sumsq", "zr_debug_reduce", "zr_step_no_alloc", "zr_state_save", "zr_state_load",
     "zr_state_reshard", "zr_state_export_params", "zr_plan_set_checked", "zr_plan_verify",
     "zr_plan_check_result", "zr_plan_set_param_layout", "zr_gather_params", "zr_plan_owner_offsets", "zr_plan_set_gather_targets", "zr_ipc_export",
     "zr_ipc_open", "zr_ipc_close", "zr_plan_destroy", "zr_status_string",
@@ -88,6 +88,7 @@ _lib.zr_step_bucket.argtypes = [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_step_finish.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_step_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_grad_sumsq.argtypes = [_vp, _vp, _vp, _vp]
+_lib.zr_bucket_sumsq.argtypes = [_vp, _vp, _vp]
 _lib.zr_debug_reduce.argtypes = [_vp, _vp, _vp, _vp]
 _lib.zr_step_no_alloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_state_save.argtypes = [_vp, ctypes.c_char_p, _vp, _vp, _vp, _i64, _vp]
@@ -260,6 +261,12 @@ def zr_grad_sumsq(plan: int, grads, out, stream=None) -> None:
 def zr_debug_reduce(plan: int, grads, g_out, stream=None) -> None:
     _check(_lib.zr_debug_reduce(plan, _ptr_array(grads), _addr(g_out), _stream(stream)),
            "zr_debug_reduce")
+
+
+def zr_bucket_sumsq(plan: int, out, stream=None) -> None:
+    """This rank's S_r from the sums of squares of a bucket-by-bucket pass
+    (every bucket's zr_step_bucket called), into the device double `out`."""
+    _check(_lib.zr_bucket_sumsq(plan, _addr(out), _stream(stream)), "zr_bucket_sumsq")
 
 
 def zr_step_no_alloc(plan: int, grads, master, m, v, param_out, sumsq_partials, step: int,

@@ -583,6 +583,20 @@ zr_status zr_step_finish(const zr_plan* p, const void* const* grad_ptrs, float* 
     return cuda_status(static_cast<cudaError_t>(e));
 }
 
+zr_status zr_bucket_sumsq(const zr_plan* p, double* d_out, zr_stream_t stream) {
+    if (!p || !d_out) return ZR_ERR_INVALID_ARG;
+    if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;
+    {
+        const zr_status dst = check_device(p);
+        if (dst != ZR_OK) return dst;
+    }
+    if (!p->clip_enabled()) return ZR_ERR_INVALID_ARG;   // tile partials live in the clip workspace
+    if ((reinterpret_cast<uintptr_t>(d_out) & 7u) != 0) return ZR_ERR_ALIGNMENT;
+    if (p->owned_numel() == 0)
+        return cuda_status(cudaMemsetAsync(d_out, 0, sizeof(double), reinterpret_cast<cudaStream_t>(stream)));
+    return cuda_status(static_cast<cudaError_t>(zr::launch_clip_combine(clip_args(p, nullptr, d_out), stream)));
+}
+
 zr_status zr_grad_sumsq(const zr_plan* p, const void* const* grad_ptrs, double* d_out, zr_stream_t stream) {
     if (!p || !d_out) return ZR_ERR_INVALID_ARG;
     if (!p->d_workspace) return ZR_ERR_NO_WORKSPACE;

@@ -239,7 +239,11 @@ struct zr_plan {
     ~zr_plan();
 
     bool clip_enabled() const { return hp.max_grad_norm > 0.0f; }
-    bool clip_uses_scratch() const { return clip_enabled() && world_size > 4; }
+    // Clipping keeps the fp32 averaged gradient for pass 2 when re-reading W
+    // replicas would cost more than writing and reading 8 bytes (W > 4), and
+    // always for grouped plans, whose per-layer gradients are released
+    // before the norm is known.
+    bool clip_uses_scratch() const { return clip_enabled() && (world_size > 4 || !tensor_group.empty()); }
     int64_t owned_numel() const { return rank_numel[rank]; }
 };
 

@@ -25,10 +25,22 @@ from . import ZR_PARTITION_FLAT, ZR_PARTITION_WHOLE_TENSOR
 
 class ZeroAdamW:
     """ZeRO stage 1/2 AdamW with a torch-optimizer interface (see the module
-    docstring): step(), zero_grad(), set_lr(), save() / load(), close()."""
+    docstring): step(), zero_grad(), set_lr(), save() / load(), close().
+
+    overlap=True steps each bucket as soon as the backward pass has filled
+    it ("Scaling training to thousands of GPUs", 03:41 DP: a bucket's
+    collective starts as soon as backward has produced its gradients): a
+    hook after every parameter's gradient accumulation counts the bucket's
+    tensors, and the last one enqueues zr_step_bucket for the bucket on a
+    side stream that waits for the backward's work so far (across
+    processes, after a barrier: every replica's part of the bucket is
+    written).  A bucket's tensors are not read again by the rest of the
+    backward, so their update can run beside it.  step() then steps buckets
+    that got no gradient, finishes the clip when there is one, and joins the
+    side stream.  One backward per step in this mode."""
 
     def __init__(self, params, group=None, lr=3e-4, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.1,
-                 max_grad_norm=0.0, partition="flat", bucket_cap_mb=25):
+                 max_grad_norm=0.0, partition="flat", bucket_cap_mb=25, overlap=False):
         import torch
         self.params = [p for p in params]
         if not self.params:
@@ -98,6 +110,77 @@ class ZeroAdamW:
         self.v = torch.zeros_like(self.master)
         self.rank, self.step_count = rank, 0
         self._grads = [self.grad_buffer[self.offsets[rank]:]]
+        self.overlap = bool(overlap)
+        self._hooks = []
+        if self.overlap:
+            # each tensor's bucket; hooks count a bucket's tensors as autograd fills them
+            bucket_of = {}
+            for s_ in segs:
+                if s_["tensor"] >= 0:
+                    bucket_of[int(s_["tensor"])] = int(s_["bucket"])
+            self._bucket_tensors = {}
+            for t in range(len(self.params)):
+                if t in bucket_of:
+                    self._bucket_tensors.setdefault(bucket_of[t], []).append(t)
+            self._side = torch.cuda.Stream(device=dev)
+            self._seen = {b: set() for b in self._bucket_tensors}
+            self._stepped = set()
+            for b, ts in self._bucket_tensors.items():
+                for t in ts:
+                    self._hooks.append(self.params[t].register_post_accumulate_grad_hook(self._make_hook(b, t)))
+
+    def _make_hook(self, b, t):
+        def hook(p):
+            if b in self._stepped:
+                raise RuntimeError("overlap: a second backward before step(); "
+                                   "gradients cannot be accumulated over several passes in this mode")
+            self._seen[b].add(t)
+            if len(self._seen[b]) == len(self._bucket_tensors[b]):
+                self._step_bucket(b)
+        return hook
+
+    def _bind_and_copy_in(self, tensors=None):
+        """Autograd accumulates into a bound .grad in place; should anything
+        have replaced it with a new tensor, copy that in and bind again; the
+        .grad of a tensor split across rank regions is copied in."""
+        flat_grad = self.grad_buffer.view(-1)
+        for p, start in self._bound:
+            if tensors is not None and id(p) not in tensors:
+                continue
+            view = flat_grad[start:start + p.numel()]
+            if p.grad is None or p.grad.data_ptr() != view.data_ptr():
+                if p.grad is not None:
+                    view.copy_(p.grad.reshape(-1))
+                else:
+                    view.zero_()
+                p.grad = view.view(p.shape)
+        for p, pieces in self._copy_in:
+            if tensors is not None and id(p) not in tensors:
+                continue
+            g = p.grad.reshape(-1)
+            for off, start, n in pieces:
+                flat_grad[start:start + n].copy_(g[off:off + n])
+
+    def _step_bucket(self, b):
+        """Bucket b's gradients are complete on this replica: step the
+        bucket (across processes once every replica's are) on the side
+        stream."""
+        import torch
+        from . import zr_step_bucket
+        from .peer import sync_point
+        t = self.step_count + 1
+        cur = torch.cuda.current_stream()
+        self._bind_and_copy_in({id(self.params[i]) for i in self._bucket_tensors[b]})
+        if self.peer is not None:
+            cur.synchronize()
+            sync_point(self.peer.dist, self.peer.group, f"bucket {b} gradients ready", t)
+            grads = self.peer.grad_ptrs
+        else:
+            grads = self._grads
+        self._side.wait_stream(cur)
+        zr_step_bucket(self.plan.handle, b, grads, self.master, self.m, self.v,
+                       None if self.peer is not None else self.param_buffer, t, self._side)
+        self._stepped.add(b)
 
     def zero_grad(self, set_to_none=False):
         """Zeroes the gradient buffer; the .grad views stay bound (set_to_none
@@ -115,26 +198,44 @@ class ZeroAdamW:
         """One optimizer step: this rank's slice of the averaged gradient,
         AdamW on its fp32 state, the bf16 result into every rank's
         parameters.  With several ranks, every rank calls it together."""
-        flat_grad = self.grad_buffer.view(-1)
-        # autograd accumulates into a bound .grad in place; should anything
-        # have replaced it with a new tensor, copy that in and bind again
-        for p, start in self._bound:
-            view = flat_grad[start:start + p.numel()]
-            if p.grad is None or p.grad.data_ptr() != view.data_ptr():
-                if p.grad is not None:
-                    view.copy_(p.grad.reshape(-1))
-                else:
-                    view.zero_()
-                p.grad = view.view(p.shape)
-        for p, pieces in self._copy_in:
-            g = p.grad.reshape(-1)
-            for off, start, n in pieces:
-                flat_grad[start:start + n].copy_(g[off:off + n])
+        if self.overlap:
+            return self._finish_overlapped()
+        self._bind_and_copy_in()
         self.step_count += 1
         if self.peer is not None:
             self.peer.step(self.master, self.m, self.v, self.step_count)
         else:
             self.plan.step(self._grads, self.master, self.m, self.v, self.param_buffer, self.step_count)
+        return None
+
+    def _finish_overlapped(self):
+        import torch
+        from . import zr_step_finish
+        from .peer import sync_point
+        for b in sorted(self._bucket_tensors):
+            if b not in self._stepped:
+                if self._seen[b]:
+                    raise RuntimeError(f"overlap: bucket {b} received gradients for only some of its tensors")
+                self._step_bucket(b)
+        t = self.step_count + 1
+        cur = torch.cuda.current_stream()
+        cur.wait_stream(self._side)
+        if self.plan.max_grad_norm > 0:
+            if self.peer is not None:
+                me = self.plan.rank
+                self.plan.bucket_sumsq(self.plan.partials[me:me + 1])
+                self.peer.all_gather_partials()
+                # (the finish reads the gradients again only when W <= 4; they are all still there)
+                zr_step_finish(self.plan.handle, self.peer.grad_ptrs, self.master, self.m, self.v, None, t, cur)
+            else:
+                zr_step_finish(self.plan.handle, self._grads, self.master, self.m, self.v, self.param_buffer,
+                               t, cur)
+        if self.peer is not None:
+            cur.synchronize()
+            sync_point(self.peer.dist, self.peer.group, "parameters written", t)
+        self.step_count = t
+        self._seen = {b: set() for b in self._bucket_tensors}
+        self._stepped = set()
         return None
 
     def save(self, path):
@@ -154,6 +255,9 @@ class ZeroAdamW:
             self.param_buffer[glob:glob + length] = self.master[owned:owned + length].to(self.param_buffer.dtype)
 
     def close(self):
+        for h in self._hooks:
+            h.remove()
+        self._hooks = []
         if self.peer is not None:
             self.peer.close()
         else:
@@ -242,10 +346,13 @@ class Zero3:
     module's slice from every replica's slot (through peer memory across
     processes) and updates it -- zr_step_bucket on the module's bucket --
     after which the slot is cleared for module i - 2.  z.step() then only
-    steps modules that received no gradient and advances the count.  One
-    backward per step (no accumulation over several), every parameter of a
-    module receiving a gradient, and no clipping (the norm needs every
-    layer's gradient before the first update).
+    steps modules that received no gradient and advances the count.  With
+    clipping the backward's per-module calls are the reduce and the sums of
+    squares, keeping the rank's fp32 averaged gradient (ZeRO-2's sharded
+    gradient); z.step() exchanges the ranks' sums of squares
+    (zr_bucket_sumsq) and applies the clipped update (zr_step_finish).  One
+    backward per step (no accumulation over several), and every parameter
+    of a module receiving a gradient.
     """
 
     def __init__(self, module, group=None, lr=3e-4, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.1,
@@ -289,8 +396,6 @@ class Zero3:
         groups = None
         slot_elems = 0
         if self.reduce_in_backward:
-            if max_grad_norm > 0:
-                raise ValueError("reduce_in_backward: clipping needs every layer's gradient before any update")
             groups = [0] * len(params)
             for u, (_, a, k) in enumerate(self.units):
                 for t in range(a, a + k):
@@ -530,6 +635,9 @@ class Zero3:
         gradients: the rest are stepped here (zero gradient)."""
         from . import zr_step
         if self.reduce_in_backward:
+            import torch
+            from . import zr_step_finish
+            from .peer import sync_point
             for u in range(len(self.units)):
                 if self._unit_done[u]:
                     continue
@@ -537,6 +645,19 @@ class Zero3:
                     raise RuntimeError(f"reduce_in_backward: module {u} received gradients for only some "
                                        "of its parameters")
                 self._reduce_unit(u)
+            if self.plan.max_grad_norm > 0:
+                # the per-module calls were the reduce and the sums of squares:
+                # the global norm, then the clipped update from the fp32 gradient
+                t = self.step_count + 1
+                cur = torch.cuda.current_stream()
+                if self.peer is not None:
+                    me = self.plan.rank
+                    self.plan.bucket_sumsq(self.plan.partials[me:me + 1])
+                    self.peer.all_gather_partials()
+                zr_step_finish(self.plan.handle, None, self.master, self.m, self.v, self.shard, t, cur)
+                if self.peer is not None:
+                    cur.synchronize()
+                    sync_point(self.peer.dist, self.peer.group, "parameters written", t)
             self.step_count += 1
             self._unit_seen = [set() for _ in self.units]
             self._unit_done = [False] * len(self.units)

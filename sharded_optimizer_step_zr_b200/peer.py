@@ -129,10 +129,16 @@ class PeerZero:
         return v.view(shape) if shape is not None else v
 
     def _exchange_sumsq(self):
+        self.plan.grad_sumsq(self.grad_ptrs, self.plan.partials[self.rank:self.rank + 1])
+        self.all_gather_partials()
+
+    def all_gather_partials(self):
+        """Every rank's entry of the clip's partials array (each rank's own
+        S_r written there already) to every rank: the scalar exchange of the
+        global-norm clip."""
         import torch
         dist = self.dist
         part = self.plan.partials
-        self.plan.grad_sumsq(self.grad_ptrs, part[self.rank:self.rank + 1])
         backend = dist.get_backend(self.group)
         mine = part[self.rank:self.rank + 1].clone()
         if backend != "nccl":

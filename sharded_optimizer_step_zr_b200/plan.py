@@ -207,6 +207,14 @@ class ZrPlan:
         _require_all(specs + [(out, "out", torch.float64, 1, False)], self.device)
         zr_grad_sumsq(self.handle, grads, out, stream)
 
+    def bucket_sumsq(self, out, stream=None):
+        """zr_bucket_sumsq: this rank's sum of squares after a bucket-by-bucket
+        pass, into out[0] (fp64), without reading gradients."""
+        import torch
+        from . import zr_bucket_sumsq
+        _require_all([(out, "out", torch.float64, 1, False)], self.device)
+        zr_bucket_sumsq(self.handle, out, stream)
+
     def debug_reduce(self, grads, g_out, stream=None):
         """zr_debug_reduce: the averaged fp32 gradient, owned order."""
         import torch

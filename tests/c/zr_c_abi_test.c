@@ -4,8 +4,9 @@
  * gradients (the last in checked mode, whose status must stay clean) and
  * checks the closed form of AdamW with a constant gradient: each step moves
  * p to p * (1 - lr * wd) - lr * g / (|g| + eps) (the bias corrections
- * cancel), within fp32 rounding.  Then the ZeRO-3 calls (see below).  Exit
- * status 0 on success. */
+ * cancel), within fp32 rounding.  Then the ZeRO-3 calls and a grouped
+ * plan stepped bucket by bucket with clipping (see below).  Exit status 0
+ * on success. */
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -164,7 +165,91 @@ int main(void) {
         zr_plan_destroy(g1);
         zr_plan_destroy(s1);
     }
-    printf("owned %lld, mismatches %lld, zero-3 mismatches %lld\n", (long long)owned, (long long)bad,
-           (long long)mism3);
-    return (bad == 0 && mism3 == 0) ? 0 : 1;
+    /* Buckets by tensor group with clipping, from C: one rank, groups
+     * {0, 1, 1} (two buckets).  zr_step on one copy of the state; on the
+     * other, zr_step_bucket for both buckets (each bucket's gradient is
+     * overwritten right after its call: a grouped plan keeps the fp32
+     * averaged gradient), zr_bucket_sumsq, zr_step_finish.  Master weights
+     * and the sum of squares must agree bit for bit. */
+    int64_t mismg = 0;
+    {
+        const zr_adamw hpc = {3e-4f, 0.9f, 0.999f, 1e-8f, 0.1f, 0.5f};
+        const int32_t groups[3] = {0, 1, 1};
+        zr_plan *pa = NULL, *pb = NULL;
+        CHECK_ZR(zr_plan_create_grouped(3, ndims, shapes, groups, 1, 0, ZR_PARTITION_FLAT, &hpc, &pa));
+        CHECK_ZR(zr_plan_create_grouped(3, ndims, shapes, groups, 1, 0, ZR_PARTITION_FLAT, &hpc, &pb));
+        int32_t n_buckets = 0;
+        CHECK_ZR(zr_plan_query(pb, NULL, NULL, NULL, &n_buckets, NULL));
+        if (n_buckets != 2) {
+            fprintf(stderr, "grouped plan: %d buckets\n", (int)n_buckets);
+            return 1;
+        }
+        uint64_t ba = 0, bb = 0;
+        CHECK_ZR(zr_plan_workspace_bytes(pa, &ba));
+        CHECK_ZR(zr_plan_workspace_bytes(pb, &bb));
+        void *wa, *wb;
+        double* part;                       /* [0]: plan a's partials, [1]: plan b's, [2]: zr_bucket_sumsq */
+        CHECK_CUDA(cudaMalloc(&wa, ba));
+        CHECK_CUDA(cudaMalloc(&wb, bb));
+        CHECK_CUDA(cudaMalloc((void**)&part, 3 * sizeof(double)));
+        CHECK_ZR(zr_plan_set_workspace(pa, wa, ba, (zr_stream_t)stream));
+        CHECK_ZR(zr_plan_set_workspace(pb, wb, bb, (zr_stream_t)stream));
+        CHECK_ZR(zr_plan_set_sumsq_partials(pa, part));
+        CHECK_ZR(zr_plan_set_sumsq_partials(pb, part + 1));
+        const int64_t N = total;
+        uint16_t* hg = (uint16_t*)malloc(sizeof(uint16_t) * N);
+        float* hp0 = (float*)malloc(sizeof(float) * N);
+        for (int64_t i = 0; i < N; ++i) {
+            hg[i] = bf16_of((float)((i % 11) - 5) / 16.0f);
+            hp0[i] = 0.01f * (float)((i % 9) - 4);
+        }
+        void *ga, *gb, *oa, *ob;
+        float *ms[2], *mm[2], *vv[2];
+        CHECK_CUDA(cudaMalloc(&ga, sizeof(uint16_t) * N));
+        CHECK_CUDA(cudaMalloc(&gb, sizeof(uint16_t) * N));
+        CHECK_CUDA(cudaMemcpy(ga, hg, sizeof(uint16_t) * N, cudaMemcpyHostToDevice));
+        CHECK_CUDA(cudaMemcpy(gb, hg, sizeof(uint16_t) * N, cudaMemcpyHostToDevice));
+        for (int k = 0; k < 2; ++k) {
+            CHECK_CUDA(cudaMalloc((void**)&ms[k], sizeof(float) * N));
+            CHECK_CUDA(cudaMalloc((void**)&mm[k], sizeof(float) * N));
+            CHECK_CUDA(cudaMalloc((void**)&vv[k], sizeof(float) * N));
+            CHECK_CUDA(cudaMemcpy(ms[k], hp0, sizeof(float) * N, cudaMemcpyHostToDevice));
+            CHECK_CUDA(cudaMemset(mm[k], 0, sizeof(float) * N));
+            CHECK_CUDA(cudaMemset(vv[k], 0, sizeof(float) * N));
+        }
+        CHECK_CUDA(cudaMalloc(&oa, sizeof(uint16_t) * N));
+        CHECK_CUDA(cudaMalloc(&ob, sizeof(uint16_t) * N));
+        const void* grad_a[1] = {ga};
+        const void* grad_b[1] = {gb};
+        CHECK_ZR(zr_step(pa, grad_a, ms[0], mm[0], vv[0], oa, 1, (zr_stream_t)stream));
+        zr_segment segs[16];
+        int64_t n_seg = 0;
+        CHECK_ZR(zr_plan_segments(pb, segs, 16, &n_seg));
+        for (int32_t bkt = 0; bkt < n_buckets; ++bkt) {
+            CHECK_ZR(zr_step_bucket(pb, bkt, grad_b, ms[1], mm[1], vv[1], ob, 1, (zr_stream_t)stream));
+            for (int64_t k = 0; k < n_seg; ++k)     /* release: the bucket's gradient is gone */
+                if (segs[k].bucket == bkt)
+                    CHECK_CUDA(cudaMemsetAsync((uint16_t*)gb + segs[k].owned_offset, 0xFF,
+                                               sizeof(uint16_t) * segs[k].length, stream));
+        }
+        CHECK_ZR(zr_bucket_sumsq(pb, part + 2, (zr_stream_t)stream));
+        CHECK_ZR(zr_step_finish(pb, NULL, ms[1], mm[1], vv[1], ob, 1, (zr_stream_t)stream));
+        CHECK_CUDA(cudaStreamSynchronize(stream));
+        uint32_t* a = (uint32_t*)malloc(sizeof(float) * N);
+        uint32_t* b = (uint32_t*)malloc(sizeof(float) * N);
+        CHECK_CUDA(cudaMemcpy(a, ms[0], sizeof(float) * N, cudaMemcpyDeviceToHost));
+        CHECK_CUDA(cudaMemcpy(b, ms[1], sizeof(float) * N, cudaMemcpyDeviceToHost));
+        for (int64_t i = 0; i < N; ++i) mismg += a[i] != b[i];
+        double hpart[3];
+        CHECK_CUDA(cudaMemcpy(hpart, part, sizeof(hpart), cudaMemcpyDeviceToHost));
+        if (hpart[0] != hpart[1] || hpart[1] != hpart[2] || !(hpart[0] > 0.0)) {
+            fprintf(stderr, "sums of squares differ: %.17g %.17g %.17g\n", hpart[0], hpart[1], hpart[2]);
+            ++mismg;
+        }
+        zr_plan_destroy(pa);
+        zr_plan_destroy(pb);
+    }
+    printf("owned %lld, mismatches %lld, zero-3 mismatches %lld, grouped mismatches %lld\n", (long long)owned,
+           (long long)bad, (long long)mism3, (long long)mismg);
+    return (bad == 0 && mism3 == 0 && mismg == 0) ? 0 : 1;
 }

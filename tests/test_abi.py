@@ -285,6 +285,22 @@ def test_zero3_calls_without_a_device():
         zr.zr_plan_destroy(h)
 
 
+def test_grouped_plans_keep_the_clip_scratch():
+    """With clipping a grouped plan's workspace holds the fp32 averaged
+    gradient at any W (its per-layer gradients are released before the
+    norm is known); a plan of the byte-cap rule holds it only for W > 4."""
+    shapes = [(4096,), (100,), (2048,)]
+    for W, grouped, scratch in ((2, False, False), (2, True, True), (8, False, True), (8, True, True)):
+        sizes = []
+        for mgn in (0.0, 1.0):
+            h = zr.zr_plan_create(shapes, W, 0, 0, 1 << 20, max_grad_norm=mgn,
+                                  groups=[0, 1, 2] if grouped else None)
+            sizes.append((zr.zr_plan_workspace_bytes(h), zr.zr_plan_query(h)["owned_numel"]))
+            zr.zr_plan_destroy(h)
+        (plain, n), (clip, _) = sizes
+        assert (clip - plain >= 4 * n) == scratch, (W, grouped)
+
+
 def test_set_adamw_refuses_turning_clipping_on_or_off():
     h = zr.zr_plan_create([(4096,)], 2, 0, 0, 1 << 20)                     # no clipping
     hc = zr.zr_plan_create([(4096,)], 2, 0, 0, 1 << 20, max_grad_norm=1.0)
@@ -345,6 +361,9 @@ def test_early_argument_errors_of_every_launching_call():
         assert L.zr_step_device_count(h, g, 16, 16, 16, 16, 4, None) == zr.ZR_ERR_ALIGNMENT
         assert L.zr_step_device_count(h, g, 16, 16, 16, 16, 16, None) == zr.ZR_ERR_NO_WORKSPACE
         assert L.zr_grad_sumsq(None, g, 16, None) == zr.ZR_ERR_INVALID_ARG
+        assert L.zr_bucket_sumsq(None, 16, None) == zr.ZR_ERR_INVALID_ARG
+        assert L.zr_bucket_sumsq(h, None, None) == zr.ZR_ERR_INVALID_ARG
+        assert L.zr_bucket_sumsq(h, 16, None) == zr.ZR_ERR_NO_WORKSPACE
         assert L.zr_debug_reduce(None, g, 16, None) == zr.ZR_ERR_INVALID_ARG
         assert L.zr_step_no_alloc(None, g, 16, 16, 16, 16, None, 1, None) == zr.ZR_ERR_INVALID_ARG
         assert L.zr_step_no_alloc(h, None, 16, 16, 16, 16, None, 1, None) == zr.ZR_ERR_INVALID_ARG

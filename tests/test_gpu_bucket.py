@@ -62,7 +62,12 @@ def test_buckets_equal_full_step(shapes, W, rank, mode, cap, max_norm, groups):
             full.plan.partials.copy_(others)
             byb.plan.partials.copy_(others)
         full.step(out_full, t)
-        release = max_norm > 0 and W > 4
+        # with clipping and W > 4 (or a grouped plan) pass 1 keeps the fp32
+        # averaged gradient, so each bucket's gradients may go right away
+        release = max_norm > 0 and (W > 4 or groups is not None)
+        if max_norm > 0:
+            want_sumsq = torch.zeros(1, dtype=torch.float64, device=DEV)
+            byb.plan.grad_sumsq(byb.grads, want_sumsq)
         for b in rng.permutation(nb):
             byb.plan.step_bucket(int(b), byb.grads, byb.master, byb.m, byb.v, out_byb, t)
             if release:
@@ -70,6 +75,12 @@ def test_buckets_equal_full_step(shapes, W, rank, mode, cap, max_norm, groups):
                 for owned, length in bucket_owned_ranges(byb.plan, int(b)):
                     for g in byb.grads:
                         g[owned: owned + length] = float("nan")
+        if max_norm > 0:
+            # this rank's S_r from the per-bucket pass, without the gradients
+            got_sumsq = torch.zeros(1, dtype=torch.float64, device=DEV)
+            byb.plan.bucket_sumsq(got_sumsq)
+            torch.cuda.synchronize()
+            assert got_sumsq.item() == want_sumsq.item()
         byb.plan.step_finish(None if release else byb.grads, byb.master, byb.m, byb.v, out_byb, t)
         c = None
         if max_norm > 0:

@@ -7,7 +7,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_harness import DEV, bf16_ulp_distance, bits32
+from gpu_harness import DEV, assert_state_close, bf16_ulp_distance, bits32
 from sharded_optimizer_step_zr_b200.optim import ZeroAdamW
 
 pytestmark = pytest.mark.gpu
@@ -23,14 +23,20 @@ def flat_u16(tensors):
     return torch.cat([t.detach().reshape(-1) for t in tensors]).cpu().view(torch.int16).numpy().view(np.uint16)
 
 
-@pytest.mark.parametrize("partition, clip", [("flat", 0.0), ("whole", 1.0)])
-def test_zero_adamw_one_rank_matches_the_oracle(partition, clip):
+@pytest.mark.parametrize("partition, clip, overlap", [("flat", 0.0, False), ("whole", 1.0, False),
+                                                     ("flat", 0.0, True), ("whole", 1.0, True),
+                                                     ("flat", 0.05, True)])
+def test_zero_adamw_one_rank_matches_the_oracle(partition, clip, overlap):
+    """overlap=True steps each 10 KB bucket on a side stream as the backward
+    fills it (the rest of the backward runs beside it): the same steps."""
     model = make_model(5)
     params = list(model.parameters())
     hp = (1e-3, 0.9, 0.999, 1e-8, 0.1, clip)
     init = flat_u16(params)
     opt = ZeroAdamW(params, lr=hp[0], betas=hp[1:3], eps=hp[3], weight_decay=hp[4], max_grad_norm=clip,
-                    partition=partition, bucket_cap_mb=0.01)
+                    partition=partition, bucket_cap_mb=0.01, overlap=overlap)
+    if overlap:
+        assert opt.plan.n_buckets > 3
     assert np.array_equal(flat_u16(params), init)          # rebinding kept the values
     N = init.size
     o_master = (init.astype(np.uint32) << 16).view(np.float32)      # bf16 -> fp32 is exact
@@ -204,6 +210,46 @@ def test_zero3_accumulation_and_evaluation():
         assert np.array_equal(full.cpu().view(torch.int16).numpy(), flat_u16(a.parameters()).view(np.int16)), t
     z2.close()
     z3.close()
+
+
+@pytest.mark.parametrize("partition", ["flat", "whole"])
+def test_zero3_reduce_in_backward_with_clipping(partition):
+    """reduce_in_backward with a global-norm clip small enough to bite: the
+    backward's per-module calls reduce and sum the squares (the fp32
+    averaged gradient kept), step() applies the clipped update.  The
+    modules' buckets cut the tiles differently from the byte-cap plan, so
+    the norm's fp64 sum runs in another order: the parameters equal
+    ordinary Zero3's within 1 bf16 ulp over three steps, not bit for bit."""
+    from sharded_optimizer_step_zr_b200.optim import Zero3
+    a, b = make_deep_model(9), make_deep_model(9)
+    za = Zero3(a, lr=1e-3, partition=partition, max_grad_norm=0.01)
+    zb = Zero3(b, lr=1e-3, partition=partition, max_grad_norm=0.01, reduce_in_backward=True)
+    N = sum(p.numel() for p in a.parameters())
+    gen = torch.Generator(device=DEV).manual_seed(29)
+    for t in (1, 2, 3):
+        x = torch.randn(32, 64, device=DEV, generator=gen).to(torch.bfloat16)
+        a(x).float().pow(2).mean().backward()
+        za.step()
+        za.zero_grad()
+        b(x).float().pow(2).mean().backward()
+        zb.step()
+        torch.cuda.synchronize()
+        assert all(not s_.view(torch.int16).any() for s_ in zb.grad_slots)
+        fa = torch.empty(N, dtype=torch.bfloat16, device=DEV)
+        fb = torch.empty(N, dtype=torch.bfloat16, device=DEV)
+        za.gather_all(fa)
+        zb.gather_all(fb)
+        torch.cuda.synchronize()
+        ua = fa.cpu().view(torch.int16).numpy().view(np.uint16)
+        ub = fb.cpu().view(torch.int16).numpy().view(np.uint16)
+        assert bf16_ulp_distance(ua, ub).max() <= 1, t
+        assert_state_close(zb.master[:zb.plan.owned_numel].cpu().numpy(),
+                           za.master[:za.plan.owned_numel].cpu().numpy(), f"master step {t}")
+    # the clip did bite: the coefficient is below 1
+    S = float(zb.plan.partials.sum().item())
+    assert 0.01 / (S ** 0.5 + 1e-6) < 1.0
+    za.close()
+    zb.close()
 
 
 @pytest.mark.parametrize("partition", ["flat", "whole"])

@@ -185,10 +185,12 @@ def test_two_processes_stage3_gather(shapes, mode):
     assert all(p.exitcode == 0 for p in procs)
 
 
-def _rank_main_optim(rank, world, port, q):
+def _rank_main_optim(rank, world, port, q, max_norm=0.0, overlap=False):
     """ZeroAdamW over a two-process group: the same bf16 model on both
     ranks, different data; after each step both models equal the oracle's
-    unsharded step on the two replicas' gradients."""
+    unsharded step on the two replicas' gradients (within 1 ulp with
+    clipping).  overlap: each bucket stepped as the backward fills it, its
+    reduce reading the other replica's gradients through IPC."""
     import sys
     sys.path.insert(0, ROOT)
     os.environ["MASTER_ADDR"] = "127.0.0.1"
@@ -208,8 +210,9 @@ def _rank_main_optim(rank, world, port, q):
         flat = lambda ts: torch.cat([t.detach().reshape(-1) for t in ts]).cpu().view(torch.int16).numpy() \
             .view(np.uint16).copy()
         init = flat(params)
-        hp = (1e-3, 0.9, 0.999, 1e-8, 0.1, 0.0)
-        opt = ZeroAdamW(params, group=dist.group.WORLD, lr=hp[0], weight_decay=hp[4], bucket_cap_mb=0.01)
+        hp = (1e-3, 0.9, 0.999, 1e-8, 0.1, max_norm)
+        opt = ZeroAdamW(params, group=dist.group.WORLD, lr=hp[0], weight_decay=hp[4], bucket_cap_mb=0.01,
+                        max_grad_norm=max_norm, overlap=overlap)
         N = init.size
         o_master = (init.astype(np.uint32) << 16).view(np.float32).copy()
         o_m, o_v, o_out = np.zeros(N, np.float32), np.zeros(N, np.float32), np.zeros(N, np.uint16)
@@ -222,11 +225,17 @@ def _rank_main_optim(rank, world, port, q):
             mine = flat([p.grad for p in params])
             reps = [None] * world
             dist.all_gather_object(reps, mine)
-            oracle.ddp_step(reps, o_master, o_m, o_v, o_out, hp, t)
+            c = oracle.clip_coef(oracle.sumsq(oracle.reduce(reps)), max_norm) if max_norm > 0 else None
+            oracle.ddp_step(reps, o_master, o_m, o_v, o_out, hp, t, clip=c)
             opt.step()
             opt.zero_grad()
             torch.cuda.synchronize()
-            ok = ok and bool(np.array_equal(flat(params), o_out))
+            got = flat(params)
+            if max_norm > 0:
+                d = np.abs(got.astype(np.int64) - o_out.astype(np.int64))
+                ok = ok and int(d.max()) <= 1
+            else:
+                ok = ok and bool(np.array_equal(got, o_out))
         q.put((rank, ok, len(opt._copy_in)))
         dist.barrier()
         opt.close()
@@ -237,11 +246,12 @@ def _rank_main_optim(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_zero_adamw_two_processes():
+@pytest.mark.parametrize("max_norm, overlap", [(0.0, False), (0.0, True), (0.05, True)])
+def test_zero_adamw_two_processes(max_norm, overlap):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _port()
-    procs = [ctx.Process(target=_rank_main_optim, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_rank_main_optim, args=(r, 2, port, q, max_norm, overlap)) for r in range(2)]
     for p in procs:
         p.start()
     results = [q.get(timeout=240) for _ in range(2)]
@@ -252,7 +262,7 @@ def test_zero_adamw_two_processes():
     assert all(p.exitcode == 0 for p in procs)
 
 
-def _rank_main_zero3(rank, world, port, q, partition="flat"):
+def _rank_main_zero3(rank, world, port, q, partition="flat", max_norm=0.0):
     """Zero3 over a two-process group: parameters gathered from both ranks'
     shards (one through IPC) before each module's forward and backward;
     after every step the gathered model equals the oracle's unsharded step
@@ -269,6 +279,8 @@ def _rank_main_zero3(rank, world, port, q, partition="flat"):
     import torch.distributed as dist
     import oracle
     from sharded_optimizer_step_zr_b200.optim import Zero3
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from gpu_harness import bf16_ulp_distance
     torch.cuda.set_device(0)
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=90))
     try:
@@ -278,14 +290,14 @@ def _rank_main_zero3(rank, world, port, q, partition="flat"):
         flat = lambda ts: torch.cat([t.detach().reshape(-1) for t in ts]).cpu().view(torch.int16).numpy() \
             .view(np.uint16).copy()
         init = flat(model.parameters())
-        hp = (1e-3, 0.9, 0.999, 1e-8, 0.1, 0.0)
+        hp = (1e-3, 0.9, 0.999, 1e-8, 0.1, max_norm)
         torch.manual_seed(6)
         model2 = torch.nn.Sequential(torch.nn.Linear(64, 128), torch.nn.GELU(), torch.nn.Linear(128, 96),
                                      torch.nn.LayerNorm(96), torch.nn.Linear(96, 24)).to("cuda:0").to(torch.bfloat16)
         z = Zero3(model, group=dist.group.WORLD, lr=hp[0], weight_decay=hp[4], bucket_cap_mb=0.01,
-                  partition=partition)
+                  partition=partition, max_grad_norm=max_norm)
         z2 = Zero3(model2, group=dist.group.WORLD, lr=hp[0], weight_decay=hp[4], partition=partition,
-                   reduce_in_backward=True)
+                   reduce_in_backward=True, max_grad_norm=max_norm)
         N = init.size
         full2 = torch.empty(N, dtype=torch.bfloat16, device="cuda:0")
         o_master = (init.astype(np.uint32) << 16).view(np.float32).copy()
@@ -300,7 +312,8 @@ def _rank_main_zero3(rank, world, port, q, partition="flat"):
             mine = flat([p.grad for p in z.params])
             reps = [None] * world
             dist.all_gather_object(reps, mine)
-            oracle.ddp_step(reps, o_master, o_m, o_v, o_out, hp, t)
+            c = oracle.clip_coef(oracle.sumsq(oracle.reduce(reps)), max_norm) if max_norm > 0 else None
+            oracle.ddp_step(reps, o_master, o_m, o_v, o_out, hp, t, clip=c)
             z.step()
             z.zero_grad()
             z.gather_all(full)
@@ -308,8 +321,15 @@ def _rank_main_zero3(rank, world, port, q, partition="flat"):
             z2.step()
             z2.gather_all(full2)
             torch.cuda.synchronize()
-            ok = ok and bool(np.array_equal(full.cpu().view(torch.int16).numpy().view(np.uint16), o_out))
-            ok = ok and bool(torch.equal(full.view(torch.int16), full2.view(torch.int16)))
+            got = full.cpu().view(torch.int16).numpy().view(np.uint16)
+            got2 = full2.cpu().view(torch.int16).numpy().view(np.uint16)
+            if max_norm > 0:
+                # the norm's fp64 sums run in other orders (oracle, byte-cap and grouped plans)
+                ok = ok and int(bf16_ulp_distance(got, o_out).max()) <= 1
+                ok = ok and int(bf16_ulp_distance(got2, got).max()) <= 1
+            else:
+                ok = ok and bool(np.array_equal(got, o_out))
+                ok = ok and bool(np.array_equal(got2, got))
         q.put((rank, ok))
         dist.barrier()
         z.close()
@@ -321,12 +341,12 @@ def _rank_main_zero3(rank, world, port, q, partition="flat"):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("partition", ["flat", "whole"])
-def test_zero3_module_two_processes(partition):
+@pytest.mark.parametrize("partition, max_norm", [("flat", 0.0), ("whole", 0.0), ("flat", 0.01)])
+def test_zero3_module_two_processes(partition, max_norm):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _port()
-    procs = [ctx.Process(target=_rank_main_zero3, args=(r, 2, port, q, partition)) for r in range(2)]
+    procs = [ctx.Process(target=_rank_main_zero3, args=(r, 2, port, q, partition, max_norm)) for r in range(2)]
     for p in procs:
         p.start()
     results = [q.get(timeout=240) for _ in range(2)]
