@@ -92,8 +92,9 @@ def parse():
                     help="time the --config workload alone (no per_config entries)")
     ap.add_argument("--no-peer", action="store_true",
                     help="N > 1: skip the ZeRO step across the processes over peer memory")
-    ap.add_argument("--peer-set", default=None, choices=sorted(__import__("synth").PARAM_SETS),
-                    help="parameter set of the N > 1 peer step (default: the --config workload's)")
+    ap.add_argument("--peer-set", default="gpt_1p3b", choices=sorted(__import__("synth").PARAM_SETS),
+                    help="parameter set of the N > 1 peer step (default: the 1.3B set of the sweep, "
+                         "which with the NCCL arm's buffers fits one GPU at every N)")
     ap.add_argument("--peer-steps", type=int, default=20, help="timed steps of the N > 1 peer step")
     ap.add_argument("--backend", default="nccl", choices=["nccl", "gloo"],
                     help="process-group backend for N > 1 (gloo: tests of several processes on one GPU)")
@@ -646,9 +647,9 @@ def measure_local(args, ctx, wl, with_e2e, with_cpu):
 
 
 def launches_per_clip_step():
-    """Kernel launches of one clipped zr_step: pass 1 (which also forms the
-    coefficient) and pass 2."""
-    return 2
+    """Kernel launches of one clipped zr_step: pass 1, the combine (S_r, S,
+    the coefficient) and pass 2."""
+    return 3
 
 
 def peer_bytes(W, n):
@@ -676,7 +677,7 @@ def measure_peer(args, ctx):
     from sharded_optimizer_step_zr_b200.plan import ZrPlan
 
     wl = workload(args.config)
-    set_name = args.peer_set or wl.param_set
+    set_name = args.peer_set
     shapes = synth.PARAM_SETS[set_name]()
     W, rank, dev = ctx.world, ctx.grank, ctx.dev
     hp = wl.hp[:5] + (0.0,)
@@ -1197,9 +1198,10 @@ def run_zero3_train(args):
             layers += [torch.nn.Linear(d, 4 * d), torch.nn.GELU(), torch.nn.Linear(4 * d, d)]
         return torch.nn.Sequential(*layers).to(dev).to(torch.bfloat16)
 
-    a, b, c, e = model(1), model(1), model(1), model(1)
+    a, b, c, e, f = model(1), model(1), model(1), model(1), model(1)
     n_params = sum(p.numel() for p in a.parameters())
     z2 = ZeroAdamW(list(a.parameters()), lr=1e-4)
+    z2_overlap = ZeroAdamW(list(f.parameters()), lr=1e-4, overlap=True)
     z3 = Zero3(b, lr=1e-4)
     z3_fwd_only = Zero3(c, lr=1e-4, backward_prefetch=False)
     z3_rib = Zero3(e, lr=1e-4, reduce_in_backward=True)
@@ -1223,6 +1225,7 @@ def run_zero3_train(args):
         return e0.elapsed_time(e1) / reps
 
     t2 = timed(a, z2, 5)
+    t2o = timed(f, z2_overlap, 5)
     t3 = timed(b, z3, 5)
     t3f = timed(c, z3_fwd_only, 5)
     t3r = timed(e, z3_rib, 5)
@@ -1230,6 +1233,8 @@ def run_zero3_train(args):
     z3.gather_all(full)
     resident = torch.cat([p.detach().reshape(-1) for p in a.parameters()])
     same = bool(torch.equal(full.view(torch.int16), resident.view(torch.int16)))
+    overlap_same = bool(torch.equal(torch.cat([p.detach().reshape(-1) for p in f.parameters()]).view(torch.int16),
+                                    resident.view(torch.int16)))
     full_r = torch.empty(n_params, dtype=torch.bfloat16, device=dev)
     z3_rib.gather_all(full_r)
     same_rib = bool(torch.equal(full.view(torch.int16), full_r.view(torch.int16)))
@@ -1240,10 +1245,12 @@ def run_zero3_train(args):
             "gathers_per_step": 2 * len(z3.units), "gathered_bytes_per_step": 2 * 2 * n_params,
             "model_tflops_zero_adamw": flops / (t2 * 1e-3) / 1e12, "same_parameters": same,
             "zero3_reduce_in_backward_step_ms": t3r, "reduce_in_backward_same_parameters": same_rib,
+            "zero_adamw_overlap_step_ms": t2o, "overlap_same_parameters": overlap_same,
             "gradient_bytes": {"zero3": 2 * z3.grad_buffer.numel(),
                                "zero3_reduce_in_backward": 2 * sum(g.numel() for g in z3_rib.grad_slots)}}
     print(json.dumps(line), flush=True)
     z2.close()
+    z2_overlap.close()
     z3.close()
     z3_fwd_only.close()
     z3_rib.close()

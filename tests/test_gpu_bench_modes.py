@@ -33,7 +33,7 @@ def test_zero3_gather_mode():
 def test_zero3_train_mode_takes_identical_steps():
     d = run_mode("--zero3-train")
     assert d["mode"] == "zero3_train" and d["same_parameters"] is True
-    assert d["reduce_in_backward_same_parameters"] is True
+    assert d["reduce_in_backward_same_parameters"] is True and d["overlap_same_parameters"] is True
     assert d["gradient_bytes"]["zero3_reduce_in_backward"] < d["gradient_bytes"]["zero3"] / 4
     assert d["zero3_step_ms"] > 0 and d["zero_adamw_step_ms"] > 0
 
