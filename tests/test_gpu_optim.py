@@ -36,7 +36,7 @@ def test_zero_adamw_one_rank_matches_the_oracle(partition, clip, overlap):
     opt = ZeroAdamW(params, lr=hp[0], betas=hp[1:3], eps=hp[3], weight_decay=hp[4], max_grad_norm=clip,
                     partition=partition, bucket_cap_mb=0.01, overlap=overlap)
     if overlap:
-        assert opt.plan.n_buckets > 3
+        assert opt.plan.n_buckets >= 2
     assert np.array_equal(flat_u16(params), init)          # rebinding kept the values
     N = init.size
     o_master = (init.astype(np.uint32) << 16).view(np.float32)      # bf16 -> fp32 is exact
