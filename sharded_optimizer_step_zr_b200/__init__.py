@@ -39,14 +39,15 @@ ZR_PARTITION_WHOLE_TENSOR = 1
 ZR_MAX_WORLD_SIZE = 512
 
 EXPORTED = [
-    "zr_plan_create", "zr_plan_create_grouped", "zr_plan_query", "zr_plan_segments", "zr_plan_workspace_bytes",
-    "zr_plan_set_workspace", "zr_plan_set_adamw", "zr_plan_set_device_lr", "zr_plan_set_sumsq_partials", "zr_step", "zr_step_device_count",
-    "zr_step_bucket",
-    "zr_step_finish", "zr_step_host",
-    "zr_grad_sumsq", "zr_bucket_sumsq", "zr_debug_reduce", "zr_step_no_alloc", "zr_state_save", "zr_state_load",
-    "zr_state_reshard", "zr_state_export_params", "zr_plan_set_checked", "zr_plan_verify",
-    "zr_plan_check_result", "zr_plan_set_param_layout", "zr_gather_params", "zr_plan_owner_offsets", "zr_plan_set_gather_targets", "zr_ipc_export",
-    "zr_ipc_open", "zr_ipc_close", "zr_plan_destroy", "zr_status_string",
+    "zr_plan_create", "zr_plan_create_grouped", "zr_plan_query", "zr_plan_segments",
+    "zr_plan_workspace_bytes", "zr_plan_set_workspace", "zr_plan_set_adamw",
+    "zr_plan_set_device_lr", "zr_plan_set_sumsq_partials", "zr_step", "zr_step_device_count",
+    "zr_step_bucket", "zr_step_finish", "zr_step_host", "zr_grad_sumsq", "zr_bucket_sumsq",
+    "zr_debug_reduce", "zr_step_no_alloc", "zr_state_save", "zr_state_load", "zr_state_reshard",
+    "zr_state_export_params", "zr_plan_set_checked", "zr_plan_verify", "zr_plan_check_result",
+    "zr_plan_set_param_layout", "zr_gather_params", "zr_plan_owner_offsets",
+    "zr_plan_set_gather_targets", "zr_ipc_export", "zr_ipc_open", "zr_ipc_close", "zr_plan_destroy",
+    "zr_status_string",
 ]
 ZR_NO_ALLOC_SCRATCH_BYTES = 4 << 20
 

@@ -12,7 +12,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libzr.so")
-SOURCES = ["zr_kernels.cu", "zr_scalars.cu", "zr_check.cu", "zr_gather.cu", "zr_no_alloc.cu", "planner.cpp", "api.cpp", "checkpoint.cpp", "peer.cpp"]
+SOURCES = ["zr_kernels.cu", "zr_scalars.cu", "zr_check.cu", "zr_gather.cu", "zr_no_alloc.cu",
+           "planner.cpp", "api.cpp", "checkpoint.cpp", "peer.cpp"]
 HEADERS = ["zr_internal.hpp", os.path.join(ROOT, "include", "zr.h"), "exports.map"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -201,9 +201,8 @@ zr_status zr_plan_create_grouped(int32_t n_tensors, const int32_t* ndims, const 
     if (n_tensors > 0 && !tensor_group) return ZR_ERR_INVALID_ARG;
     for (int32_t t = 1; t < n_tensors; ++t)
         if (tensor_group[t] < tensor_group[t - 1]) return ZR_ERR_INVALID_ARG;
-    static const int32_t none = 0;
-    return create_plan(n_tensors, ndims, shapes, n_tensors > 0 ? tensor_group : &none, world_size, rank, mode, 0,
-                       hp, out);
+    // (an empty set has no buckets either way)
+    return create_plan(n_tensors, ndims, shapes, tensor_group, world_size, rank, mode, 0, hp, out);
 }
 
 static zr_status create_plan(int32_t n_tensors, const int32_t* ndims, const int64_t* const* shapes,

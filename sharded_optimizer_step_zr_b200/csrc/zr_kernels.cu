@@ -374,26 +374,36 @@ __global__ void __launch_bounds__(kThreads) zr_clip_combine_kernel(const ClipArg
     clip_group_done(c, static_cast<int32_t>(blockIdx.x));
 }
 
+// Launch configuration for a programmatic dependent launch: the grid may be
+// scheduled while the previous kernel on the stream drains (the kernel's
+// first instruction, griddepcontrol.wait, holds it until that kernel has
+// completed and its writes are visible).  Copies, memsets and event waits
+// before it keep their full ordering.
+struct PdlLaunch {
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    PdlLaunch(unsigned grid, cudaStream_t stream) {
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = stream;
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+};
+
 template <int CAP, int G, Pass PASS, bool FROM, bool WRITE, bool DEVSC, bool GATHER>
 cudaError_t launch_one(const LaunchArgs& a, const void* const* grad_ptrs, cudaStream_t stream) {
     // grad_ptrs may be NULL for the pass that reads the g scratch instead.
     GradPtrs<CAP> gp;
     for (int w = 0; w < CAP; ++w)
         gp.p[w] = (grad_ptrs != nullptr && w < a.world_size) ? static_cast<const uint16_t*>(grad_ptrs[w]) : nullptr;
-    // Programmatic dependent launch: the grid's scheduling overlaps the
-    // previous kernel's tail (back-to-back steps lose less to the launch
-    // gap); the kernel's first instruction waits for that kernel.
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(a.n_tiles));
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, zr_tile_kernel<CAP, G, PASS, FROM, WRITE, DEVSC, GATHER>, gp, a);
+    // Programmatic dependent launch: back-to-back steps lose less to the
+    // launch gap.
+    PdlLaunch l(static_cast<unsigned>(a.n_tiles), stream);
+    return cudaLaunchKernelEx(&l.cfg, zr_tile_kernel<CAP, G, PASS, FROM, WRITE, DEVSC, GATHER>, gp, a);
 }
 
 template <Pass PASS, bool FROM, bool WRITE, bool DEVSC = false, bool GATHER = false>
@@ -443,17 +453,8 @@ int launch_tiles(Pass pass, const LaunchArgs& a, const void* const* grad_ptrs, b
 
 int launch_clip_combine(const ClipArgs& c, void* stream_v) {
     if (c.n_tiles <= 0) return cudaSuccess;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(clip_groups(c.n_tiles)));
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = static_cast<cudaStream_t>(stream_v);
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, zr_clip_combine_kernel, c);
+    PdlLaunch l(static_cast<unsigned>(clip_groups(c.n_tiles)), static_cast<cudaStream_t>(stream_v));
+    return cudaLaunchKernelEx(&l.cfg, zr_clip_combine_kernel, c);
 }
 
 }  // namespace zr

@@ -13,8 +13,9 @@ Every replica keeps its full gradient in the plan's owner-major layout
 into) -- or, for the stage-3 layer loop with grad_slot_elems, only two
 rotating gradient slots of one layer each (``grad_slots``; every replica's
 slot j at byte address ``grad_slot_bases[w][j]``), which the caller lays
-out and steps layer by layer with zr_step_bucket on a grouped plan.  Stages 1 and 2: ``param_buffer`` holds the full bf16 parameters in
-the global layout, written by every rank's step.  Stage 3: each rank keeps
+out and steps layer by layer with zr_step_bucket on a grouped plan.
+Stages 1 and 2: ``param_buffer`` holds the full bf16 parameters in the
+global layout, written by every rank's step.  Stage 3: each rank keeps
 only ``param_shard``, its bf16 parameters in owned order, and ``gather``
 assembles whole tensors (one layer, ahead of its use) from every rank's
 shard through the same peer mappings.
