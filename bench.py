@@ -86,6 +86,9 @@ def parse():
                     help="checked mode: the device tile tables verified before every launch")
     ap.add_argument("--no-alloc", action="store_true",
                     help="step through zr_step_no_alloc (the library's static scratch, no workspace)")
+    ap.add_argument("--gather-targets", action="store_true",
+                    help="the step stores each bf16 result into W parameter buffers of this GPU (the "
+                         "all-gather by stores of the step across GPUs, its HBM side); W <= 8 workloads")
     ap.add_argument("--sweep", action="store_true",
                     help="1.3B set: bucket cap x W x partition; one JSON record per point")
     ap.add_argument("--no-companions", action="store_true",
@@ -520,6 +523,14 @@ def measure_local(args, ctx, wl, with_e2e, with_cpu):
         run_step = bound_bucket_steps(plan, my_buckets, grads, master, m, v, param_out, stream)
     if args.no_alloc:
         run_step = bound_no_alloc_steps(plan, grads, master, m, v, param_out, stream)
+    targets = None
+    if args.gather_targets:
+        if W > 8:
+            raise SystemExit("--gather-targets: W parameter buffers of the full set fit one GPU only for W <= 8")
+        from sharded_optimizer_step_zr_b200 import zr_plan_set_gather_targets
+        targets = [param_out] + [torch.zeros_like(param_out) for _ in range(W - 1)]
+        zr_plan_set_gather_targets(plan.handle, targets, stream)
+        run_step = plan.bound_step(grads, master, m, v, None, stream)
 
     for _ in range(args.warmup):
         step_no += 1
@@ -551,6 +562,8 @@ def measure_local(args, ctx, wl, with_e2e, with_cpu):
     bpp = bytes_per_owned_param(W, clip)
     if args.no_alloc and clip and W > 4:
         bpp = 2 * W + 26 + 2 * W        # pass 2 reads the gradients again instead of an fp32 copy
+    if args.gather_targets:
+        bpp += 2 * (W - 1)              # the bf16 result stored into W buffers instead of one
     alg_bytes = n * bpp
     avg_ms = local_ms / K
     achieved = alg_bytes / (avg_ms * 1e-3) / 1e9
@@ -558,7 +571,7 @@ def measure_local(args, ctx, wl, with_e2e, with_cpu):
     # (bucket-by-bucket or checked steps launch more kernels: no per-launch record)
     traffic = None
     traffic_note = None
-    if not (args.per_bucket or args.checked or args.no_alloc):
+    if not (args.per_bucket or args.checked or args.no_alloc or args.gather_targets):
         traffic, traffic_note = recorded_traffic(wl.name, clip, n)
 
     # the ceiling at this size: a plain device copy (torch) moving the step's
@@ -586,7 +599,7 @@ def measure_local(args, ctx, wl, with_e2e, with_cpu):
 
     # end to end through zr_step_host: pinned host gradients in, result out
     e2e = None
-    if with_e2e:
+    if with_e2e and not args.gather_targets:
         host_grads = [g.cpu().pin_memory() for g in grads]
         host_out = torch.empty(plan.padded_numel, dtype=torch.bfloat16).pin_memory()
         for _ in range(3):
@@ -626,6 +639,7 @@ def measure_local(args, ctx, wl, with_e2e, with_cpu):
                    "bucket_cap_mb": wl.bucket_cap_mb, "clip": clip, "owned_params": n,
                    "per_bucket": bool(args.per_bucket), "buckets_stepped": len(my_buckets),
                    "checked": bool(args.checked), "no_alloc": bool(args.no_alloc),
+                   "gather_targets": W if args.gather_targets else 0,
                    "bytes_per_owned_param": bpp,
                    "l2": f"no flush: each step touches {alg_bytes / 1e6:.0f} MB > 126 MB L2"},
         "hbm_gbs": achieved,
@@ -641,7 +655,7 @@ def measure_local(args, ctx, wl, with_e2e, with_cpu):
         "copy_reference": copy_ref,
     }
     plan.close()
-    del grads, master, m, v, param_out, run_step
+    del grads, master, m, v, param_out, run_step, targets
     torch.cuda.empty_cache()
     return entry
 
