@@ -70,3 +70,15 @@ def test_peer_mode_two_processes_one_gpu():
     assert p["owned_params"] == 124439808 // 2
     assert p["bytes_per_step_per_rank"]["peer_loads"] == 2 * p["owned_params"]
     assert "skipped" in p["nccl_arm"]
+
+
+def test_gather_targets_and_no_alloc_modes():
+    """The step with W parameter buffers as gather targets (56 B per owned
+    parameter at W = 8) and through zr_step_no_alloc report their lines."""
+    base = ["--config", "gpt2_124m_w8", "--no-companions", "--no-e2e", "--no-cpu-baseline",
+            "--steps", "20", "--warmup", "3"]
+    d = run_mode(*base, "--gather-targets")
+    assert d["config"]["gather_targets"] == 8 and d["config"]["bytes_per_owned_param"] == 56
+    assert d["value"] > 0 and d["roofline"]["traffic"] is None
+    d = run_mode(*base, "--no-alloc")
+    assert d["config"]["no_alloc"] is True and d["value"] > 0
