@@ -70,6 +70,13 @@ template <int CAP>
 __global__ void __launch_bounds__(kGatherThreads)
 zr_gather_kernel(const ShardPtrs<CAP> sp, const GatherPiece* __restrict__ pieces, int32_t first, int32_t n,
                  uint16_t* dst, int64_t dst_base) {
+    // Launched as a programmatic dependent of the previous kernel on the
+    // stream: scheduled while that kernel drains, it waits here until that
+    // kernel has completed and its writes are visible (it may be the step
+    // that wrote the shards, or the layer that read the slot about to be
+    // overwritten), then lets the next launch be scheduled.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
     for (int32_t k = blockIdx.x; k < n; k += gridDim.x) {
         const GatherPiece pc = pieces[first + k];
         copy_piece(sp.p[pc.owner] + pc.src, dst + (pc.dst - dst_base), pc.len);
@@ -82,8 +89,16 @@ cudaError_t launch_gather_cap(const GatherPiece* pieces, int32_t first, int32_t 
     ShardPtrs<CAP> sp;
     for (int w = 0; w < CAP; ++w)
         sp.p[w] = w < world_size ? static_cast<const uint16_t*>(shard_ptrs[w]) : nullptr;
-    zr_gather_kernel<CAP><<<ctas, kGatherThreads, 0, s>>>(sp, pieces, first, n, dst, dst_base);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+    cfg.blockDim = dim3(kGatherThreads);
+    cfg.stream = s;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, zr_gather_kernel<CAP>, sp, pieces, first, n, dst, dst_base);
 }
 
 }  // namespace
