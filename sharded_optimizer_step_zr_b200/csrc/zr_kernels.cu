@@ -374,6 +374,65 @@ __global__ void __launch_bounds__(kThreads) zr_clip_combine_kernel(const ClipArg
     clip_group_done(c, static_cast<int32_t>(blockIdx.x));
 }
 
+// The same sums for a plan of at most kSmallCombineGroups groups, in one CTA
+// of 128 threads per group: threads 128g .. 128g + 127 sum group g exactly as
+// fixed_sum128 does (a named barrier per group in place of the block-wide
+// one), the group totals meet in shared memory, and the first 128 threads
+// sum them in the same fixed order -- the same additions in the same order
+// as the grid, without the fence, the ticket and the second trip to L2.
+constexpr int kSmallCombineGroups = 8;
+
+__device__ __forceinline__ void group_bar(int g) {
+    asm volatile("bar.sync %0, %1;" :: "r"(g + 1), "r"(kThreads) : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads * kSmallCombineGroups) zr_clip_combine_small_kernel(const ClipArgs c) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+    __shared__ double warp_part[kSmallCombineGroups * (kThreads / 32)];
+    __shared__ double group_total[kSmallCombineGroups];
+    const int g = static_cast<int>(threadIdx.x) / kThreads;
+    const int t = static_cast<int>(threadIdx.x) % kThreads;
+    const int lane = t & 31, warp = t >> 5;
+    const int32_t n_groups = clip_groups(c.n_tiles);
+    // Group g's partials: thread t adds p[t], p[t + 128], ... (eight loads in
+    // flight), then the shuffle tree and the four warp totals in order.
+    const int32_t first = g * kClipGroupTiles;
+    const int32_t count = min(kClipGroupTiles, c.n_tiles - first);
+    double x = 0.0;
+    for (int32_t i0 = t; i0 < count; i0 += 8 * kThreads) {
+        double v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            v[k] = (i0 + k * kThreads < count) ? __ldcg(c.tile_partials + first + i0 + k * kThreads) : 0.0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (i0 + k * kThreads < count) x += v[k];
+    }
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1) x += __shfl_down_sync(0xFFFFFFFFu, x, d);
+    if (lane == 0) warp_part[g * (kThreads / 32) + warp] = x;
+    group_bar(g);
+    if (t == 0) {
+        double total = 0.0;
+        for (int w = 0; w < kThreads / 32; ++w) total += warp_part[g * (kThreads / 32) + w];
+        group_total[g] = total;
+    }
+    __syncthreads();
+    if (g != 0) return;
+    // The group totals, by threads 0..127 in the same fixed order.
+    double y = t < n_groups ? 0.0 + group_total[t] : 0.0;
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1) y += __shfl_down_sync(0xFFFFFFFFu, y, d);
+    if (lane == 0) warp_part[warp] = y;
+    group_bar(0);
+    if (t == 0) {
+        double own = 0.0;
+        for (int w = 0; w < kThreads / 32; ++w) own += warp_part[w];
+        clip_coefficient(c, own);
+    }
+}
+
 // Launch configuration for a programmatic dependent launch: the grid may be
 // scheduled while the previous kernel on the stream drains (the kernel's
 // first instruction, griddepcontrol.wait, holds it until that kernel has
@@ -453,7 +512,13 @@ int launch_tiles(Pass pass, const LaunchArgs& a, const void* const* grad_ptrs, b
 
 int launch_clip_combine(const ClipArgs& c, void* stream_v) {
     if (c.n_tiles <= 0) return cudaSuccess;
-    PdlLaunch l(static_cast<unsigned>(clip_groups(c.n_tiles)), static_cast<cudaStream_t>(stream_v));
+    const int32_t n_groups = clip_groups(c.n_tiles);
+    if (n_groups <= kSmallCombineGroups) {
+        PdlLaunch l(1u, static_cast<cudaStream_t>(stream_v));
+        l.cfg.blockDim = dim3(static_cast<unsigned>(kThreads * n_groups));
+        return cudaLaunchKernelEx(&l.cfg, zr_clip_combine_small_kernel, c);
+    }
+    PdlLaunch l(static_cast<unsigned>(n_groups), static_cast<cudaStream_t>(stream_v));
     return cudaLaunchKernelEx(&l.cfg, zr_clip_combine_kernel, c);
 }
 

@@ -327,6 +327,35 @@ def test_clip_all_ranks(W, mode):
         assert bf16_ulp_distance(u16(out_gpu), out_orc).max() <= 1
 
 
+def test_clip_combine_paths_agree():
+    """S_r of a plan of at most 8 groups of 1024 tiles (summed by one CTA) and
+    of a plan of more groups (a grid of CTAs) follow the same fixed order:
+    the same gradients, followed in tile order by 3907 tiles of zeros whose
+    partials are +0.0, give the same bits.  W = 1, flat; the extra tensor is
+    declared first, so it is packed last, in a bucket of its own."""
+    from sharded_optimizer_step_zr_b200.plan import ZrPlan
+    hp = (3e-4, 0.9, 0.999, 1e-8, 0.1, 1.0)
+    own = [(4_000_000,), (3_200_000,), (3_000_000,)]      # one 20.4 MB bucket: about 4980 tiles
+    extra = 3907 * 2048                                     # a multiple of the tile: same cuts after it
+    small = ZrPlan(own, 1, 0, 0, 25 << 20, *hp, device=DEV)
+    grid = ZrPlan([(extra,)] + own, 1, 0, 0, 25 << 20, *hp, device=DEV)
+    assert (small.n_buckets, grid.n_buckets) == (1, 2)
+    n = small.owned_numel
+    gen = torch.Generator(device=DEV).manual_seed(7)
+    g = (torch.randn(n, generator=gen, device=DEV) * 1e-2).to(torch.bfloat16)
+    g_grid = torch.cat([torch.zeros(extra, dtype=torch.bfloat16, device=DEV), g])
+    s_small = torch.zeros(1, dtype=torch.float64, device=DEV)
+    s_grid = torch.zeros(1, dtype=torch.float64, device=DEV)
+    small.grad_sumsq([g], s_small)
+    grid.grad_sumsq([g_grid], s_grid)
+    torch.cuda.synchronize()
+    assert s_small.item() == s_grid.item()
+    want = oracle.sumsq(oracle.reduce([u16(g)]))
+    assert abs(s_small.item() - want) <= 1e-12 * want
+    small.close()
+    grid.close()
+
+
 def test_unwritten_positions_untouched():
     """A rank writes exactly its own positions of the parameter buffer."""
     shapes = [(1000,), (333,), (4100,)]
