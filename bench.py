@@ -103,6 +103,11 @@ def parse():
                     help="process-group backend for N > 1 (gloo: tests of several processes on one GPU)")
     ap.add_argument("--same-gpu", action="store_true",
                     help="N > 1: every process on cuda:0 (a test on a one-GPU machine)")
+    ap.add_argument("--write-traffic-record", metavar="CSV",
+                    help="host only: turn an ncu --csv capture (dram__bytes_read.sum, dram__bytes_write.sum, "
+                         "gpu__time_duration.sum) of --small-case's launches of one step into the traffic "
+                         "record of --config under profiles/, scaled by owned parameters")
+    ap.add_argument("--small-case", default=None, help="workload the capture ran (default: --config)")
     args = ap.parse_args()
     if args.cpu_threads <= 0:
         args.cpu_threads = host_threads()
@@ -1358,8 +1363,68 @@ def plan_info(name):
     return info
 
 
+def _owned_params(name):
+    from sharded_optimizer_step_zr_b200.plan import ZrPlan
+    wl = workload(name)
+    plan = ZrPlan(wl.shapes, wl.world_size, wl.ranks[0], wl.mode, wl.bucket_cap_bytes, *wl.hp, bind=False)
+    n = plan.owned_numel
+    plan.close()
+    return n
+
+
+def write_traffic_record(csv_path, full_name, small_name):
+    """The record `recorded_traffic` reads: the DRAM bytes of the captured
+    launches of one step of `small_name` (an ncu --csv log of
+    dram__bytes_read.sum, dram__bytes_write.sum and gpu__time_duration.sum,
+    one row per launch and metric), per owned parameter, scaled to
+    `full_name`'s owned parameters, with the hash of the kernel source it
+    was taken on.  Host only."""
+    import csv
+    with open(csv_path) as f:
+        rows = list(csv.reader(line for line in f if not line.startswith("==")))
+    head = rows[0]
+    ki, mi, vi, ii = (head.index(k) for k in ("Kernel Name", "Metric Name", "Metric Value", "ID"))
+    metrics = {}
+    for r in rows[1:]:
+        metrics.setdefault((int(r[ii]), r[ki]), {})[r[mi]] = float(r[vi].replace(",", ""))
+    launches = []
+    for (_, name), m in sorted(metrics.items()):
+        short = name
+        for k in ("zr_tile_kernel", "zr_clip_combine_small_kernel", "zr_clip_combine_kernel"):
+            if k in name:
+                a = name.index(k)
+                short = name[a:name.index(">", a) + 1] if k == "zr_tile_kernel" else k
+                break
+        launches.append({"kernel": short, "dram_bytes_read": int(m["dram__bytes_read.sum"]),
+                         "dram_bytes_write": int(m["dram__bytes_write.sum"]),
+                         "gpu_time_duration_ns": int(m["gpu__time_duration.sum"])})
+    full = workload(full_name)
+    clip = full.max_grad_norm > 0
+    n_small, n_full = _owned_params(small_name), _owned_params(full_name)
+    total = sum(x["dram_bytes_read"] + x["dram_bytes_write"] for x in launches)
+    stem = f"zr_clip_step_{full_name}" if clip else f"zr_tile_kernel_{full_name}"
+    summary = "profiles/zr_clip_step_gpt_1p3b_w8_whole.md" if clip else f"profiles/zr_tile_kernel_{full_name}.md"
+    entry = {"kernel": " + ".join(x["kernel"] for x in launches), "launches_per_step": len(launches),
+             "small_case": {"workload": small_name, "owned_params": n_small, "per_launch": launches,
+                            "dram_bytes": total},
+             "bytes_per_owned_param": total / n_small,
+             "full_size": {"owned_params": n_full, "scaled_bytes_per_step": total / n_small * n_full,
+                           "algorithmic_bytes_per_step": n_full * bytes_per_owned_param(full.world_size, clip)},
+             "kernel_source_sha256_16": kernel_source_hash(), "summary": summary}
+    out = os.path.join(PROFILES, f"{stem}_traffic.json")
+    with open(out, "w") as f:
+        json.dump({full_name: entry}, f, indent=2)
+        f.write("\n")
+    return out, entry
+
+
 def main():
     args = parse()
+    if args.write_traffic_record:
+        out, entry = write_traffic_record(args.write_traffic_record, args.config, args.small_case or args.config)
+        print(json.dumps({"record": os.path.relpath(out, ROOT), "full_size": entry["full_size"],
+                          "bytes_per_owned_param": entry["bytes_per_owned_param"]}), flush=True)
+        return
     if args.plan_info:
         print(json.dumps(plan_info(args.config)), flush=True)
         return
