@@ -12,6 +12,7 @@ clipped workload the coefficient needs the global sum of squares over all
 over every rank's shard (inputs from the C twin of the generator).
 """
 import concurrent.futures as cf
+import dataclasses
 import os
 
 import numpy as np
@@ -67,12 +68,17 @@ def host_global_sumsq(oplan, wl, step, threads):
 
 
 SWEEP = {wl.name: wl for wl in synth.sweep_workloads()}
+# The Llama set at W = 2: rank 1 owns 3.37 G elements, so owned offsets pass
+# 2**31 (and byte offsets of the fp32 state 2**34); about 81 GB on the device.
+LARGE = {"llama_7b_w2": dataclasses.replace(synth.WORKLOADS["llama_7b_w64"], name="llama_7b_w2",
+                                            world_size=2, ranks=(1,))}
 
-# Configs 2-4 (and the last rank of config 4, whose offsets pass 2**32), and
+# Configs 2-4 (and the last rank of config 4, whose offsets pass 2**32; and
+# a shard of more than 2**31 elements), and
 # the 1.3B sweep at the 25 MB cap: three steps, each with fresh gradients,
 # so the checked m and v carry state from the earlier steps.
 THREE_STEP = ([("gpt2_124m_w8", None), ("llama_7b_w64", None), ("llama_7b_w64", 63),
-               ("gpt_1p3b_w8_whole_clip", None)] +
+               ("gpt_1p3b_w8_whole_clip", None), ("llama_7b_w2", None)] +
               [(f"sweep_1p3b_{m}_w{w}_cap25", None) for m in ("flat", "whole") for w in (2, 8, 32, 64)])
 # The rest of the sweep (caps 1, 5, 100 and 400 MB): one step each.
 ONE_STEP = [(f"sweep_1p3b_{m}_w{w}_cap{c}", None) for m in ("flat", "whole") for w in (2, 8, 32, 64)
@@ -82,7 +88,7 @@ ONE_STEP = [(f"sweep_1p3b_{m}_w{w}_cap{c}", None) for m in ("flat", "whole") for
 @pytest.mark.parametrize("name, rank, steps", [(n, r, 3) for n, r in THREE_STEP] +
                          [(n, r, 1) for n, r in ONE_STEP])
 def test_full_size_sampled(name, rank, steps):
-    wl = synth.WORKLOADS[name] if name in synth.WORKLOADS else SWEEP[name]
+    wl = synth.WORKLOADS.get(name) or SWEEP.get(name) or LARGE[name]
     rank = wl.ranks[0] if rank is None else rank
     W = wl.world_size
     clip = wl.max_grad_norm > 0
@@ -100,7 +106,7 @@ def test_full_size_sampled(name, rank, steps):
     oplan = oracle.Plan(wl.shapes, W, wl.mode, wl.bucket_cap_bytes)
     own = sample_owned(runs, n)
     glob = owned_to_global(runs, own)
-    assert np.array_equal(glob, oplan.owned_global_index(rank)[own])
+    assert np.array_equal(glob, owned_to_global(sorted(oplan.runs(rank)), own))
     tg = torch.from_numpy(glob)
     own_t = torch.from_numpy(own).to(DEV)
     p_ref = synth.master_f32(wl.seed, tg, n_valid=oplan.total_numel).numpy().copy()
