@@ -42,6 +42,24 @@ def test_only_zr_symbols_exported():
     assert syms and all(s.startswith("zr_") for s in syms), syms
 
 
+def test_import_without_the_library_fails_loudly(tmp_path):
+    """The binding has no fallback: a copy of the package without libzr.so
+    refuses to import, naming the missing file."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = os.path.join(ROOT, "sharded_optimizer_step_zr_b200")
+    dst = tmp_path / "sharded_optimizer_step_zr_b200"
+    dst.mkdir()
+    for f in os.listdir(pkg):
+        if f.endswith(".py"):
+            shutil.copy(os.path.join(pkg, f), dst / f)
+    r = subprocess.run([sys.executable, "-c", "import sharded_optimizer_step_zr_b200"], cwd=tmp_path,
+                       capture_output=True, text=True, env=dict(os.environ, PYTHONPATH=str(tmp_path)))
+    assert r.returncode != 0
+    assert "ImportError" in r.stderr and "libzr.so is missing" in r.stderr
+
+
 def test_status_strings():
     for s in range(7):
         assert zr.zr_status_string(s).startswith("ZR_")
