@@ -70,15 +70,24 @@ def host_global_sumsq(oplan, wl, step, threads):
 SWEEP = {wl.name: wl for wl in synth.sweep_workloads()}
 # The Llama set at W = 2: rank 1 owns 3.37 G elements, so owned offsets pass
 # 2**31 (and byte offsets of the fp32 state 2**34); about 81 GB on the device.
+# Replica counts that are not powers of two (a true division by W; three
+# full groups of 8 replicas, and one partial group), on the 1.3B set.
 LARGE = {"llama_7b_w2": dataclasses.replace(synth.WORKLOADS["llama_7b_w64"], name="llama_7b_w2",
-                                            world_size=2, ranks=(1,))}
+                                            world_size=2, ranks=(1,)),
+         "sweep_1p3b_flat_w24_cap25": dataclasses.replace(SWEEP["sweep_1p3b_flat_w32_cap25"],
+                                                          name="sweep_1p3b_flat_w24_cap25", world_size=24,
+                                                          ranks=(13,)),
+         "sweep_1p3b_whole_w6_cap25": dataclasses.replace(SWEEP["sweep_1p3b_whole_w8_cap25"],
+                                                          name="sweep_1p3b_whole_w6_cap25", world_size=6,
+                                                          ranks=(2,))}
 
 # Configs 2-4 (and the last rank of config 4, whose offsets pass 2**32; and
 # a shard of more than 2**31 elements), and
 # the 1.3B sweep at the 25 MB cap: three steps, each with fresh gradients,
 # so the checked m and v carry state from the earlier steps.
 THREE_STEP = ([("gpt2_124m_w8", None), ("llama_7b_w64", None), ("llama_7b_w64", 63),
-               ("gpt_1p3b_w8_whole_clip", None), ("llama_7b_w2", None)] +
+               ("gpt_1p3b_w8_whole_clip", None), ("llama_7b_w2", None),
+               ("sweep_1p3b_flat_w24_cap25", None), ("sweep_1p3b_whole_w6_cap25", None)] +
               [(f"sweep_1p3b_{m}_w{w}_cap25", None) for m in ("flat", "whole") for w in (2, 8, 32, 64)])
 # The rest of the sweep (caps 1, 5, 100 and 400 MB): one step each.
 ONE_STEP = [(f"sweep_1p3b_{m}_w{w}_cap{c}", None) for m in ("flat", "whole") for w in (2, 8, 32, 64)
