@@ -137,7 +137,21 @@ __device__ __forceinline__ void fold8(const GradPtrs<CAP>& gp, int W, int64_t of
 #pragma unroll
     for (int j = 1; j < G; ++j)
         if (j < W) add8(q[j], s);
-    if constexpr (CAP > G) {
+    if constexpr (CAP > G && CAP <= 2 * G) {
+        // At most one more group (W = 9 .. 16): its replica indices are
+        // compile-time constants, so the pointer array stays in the
+        // parameter bank (a runtime index made the compiler copy it to
+        // local memory, 128 bytes per thread) and the loads of both groups
+        // can be issued together.
+        if (W > G) {
+#pragma unroll
+            for (int j = 0; j < G; ++j)
+                if (G + j < W) q[j] = ld_grad16(gp.p[G + j] + off);
+#pragma unroll
+            for (int j = 0; j < G; ++j)
+                if (G + j < W) add8(q[j], s);
+        }
+    } else if constexpr (CAP > G) {
         for (int w0 = G; w0 < W; w0 += G) {
 #pragma unroll
             for (int j = 0; j < G; ++j)
