@@ -314,6 +314,21 @@ zr_status zr_grad_sumsq(const zr_plan* plan, const void* const* grad_ptrs, doubl
 zr_status zr_debug_reduce(const zr_plan* plan, const void* const* grad_ptrs, float* g_out,
                           zr_stream_t stream);
 
+/* Verification hook for the averaging of stage 1 (g = s / W, rounded to
+ * nearest even; for a power-of-two W the kernels multiply by 1/W instead of
+ * dividing, which is exact scaling).  Runs the kernels' averaging on every
+ * one of the 2^32 fp32 bit patterns s for each W in [w_first, w_last]
+ * (1 <= w_first <= w_last <= ZR_MAX_WORLD_SIZE) and compares the bits with
+ * IEEE division on the GPU; d_mismatches[W - w_first] (device,
+ * w_last - w_first + 1 uint64 counters, 8-byte aligned, zeroed by the call)
+ * receives the number of inputs whose results differ, NaN against NaN
+ * counting as equal.  Asynchronous on `stream`: one grid per W (about 10 ms
+ * each on a B200).  Errors: ZR_ERR_INVALID_ARG, ZR_ERR_ALIGNMENT,
+ * ZR_ERR_UNSUPPORTED (not compute capability 10.x), ZR_ERR_CUDA.  Needs no
+ * plan. */
+zr_status zr_debug_average_check(int32_t w_first, int32_t w_last, uint64_t* d_mismatches,
+                                 zr_stream_t stream);
+
 /* ---------------------------------------------------------------------
  * ZeRO across GPUs over peer memory (NVLink / NVSwitch), one process per GPU
  * ("CS336 lecture 8", ZeRO-1 sketch: reduce-scatter of the gradients, update

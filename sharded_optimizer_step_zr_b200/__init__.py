@@ -43,7 +43,7 @@ EXPORTED = [
     "zr_plan_workspace_bytes", "zr_plan_set_workspace", "zr_plan_set_adamw",
     "zr_plan_set_device_lr", "zr_plan_set_sumsq_partials", "zr_step", "zr_step_device_count",
     "zr_step_bucket", "zr_step_finish", "zr_step_host", "zr_grad_sumsq", "zr_bucket_sumsq",
-    "zr_debug_reduce", "zr_step_no_alloc", "zr_state_save", "zr_state_load", "zr_state_reshard",
+    "zr_debug_reduce", "zr_debug_average_check", "zr_step_no_alloc", "zr_state_save", "zr_state_load", "zr_state_reshard",
     "zr_state_export_params", "zr_plan_set_checked", "zr_plan_verify", "zr_plan_check_result",
     "zr_plan_set_param_layout", "zr_gather_params", "zr_plan_owner_offsets",
     "zr_plan_set_gather_targets", "zr_ipc_export", "zr_ipc_open", "zr_ipc_close", "zr_plan_destroy",
@@ -91,6 +91,7 @@ _lib.zr_step_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_grad_sumsq.argtypes = [_vp, _vp, _vp, _vp]
 _lib.zr_bucket_sumsq.argtypes = [_vp, _vp, _vp]
 _lib.zr_debug_reduce.argtypes = [_vp, _vp, _vp, _vp]
+_lib.zr_debug_average_check.argtypes = [ctypes.c_int32, ctypes.c_int32, _vp, _vp]
 _lib.zr_step_no_alloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_state_save.argtypes = [_vp, ctypes.c_char_p, _vp, _vp, _vp, _i64, _vp]
 _lib.zr_state_load.argtypes = [_vp, ctypes.c_char_p, _vp, _vp, _vp, _P(_i64), _vp]
@@ -257,6 +258,14 @@ def zr_step_host(plan: int, host_grads, dev_grads, master, m, v, param_out, host
 
 def zr_grad_sumsq(plan: int, grads, out, stream=None) -> None:
     _check(_lib.zr_grad_sumsq(plan, _ptr_array(grads), _addr(out), _stream(stream)), "zr_grad_sumsq")
+
+
+def zr_debug_average_check(w_first: int, w_last: int, mismatches, stream=None) -> None:
+    """Per W in [w_first, w_last]: inputs (of all 2^32 fp32 values) whose
+    averaged value differs from IEEE division, into mismatches (device
+    uint64 / int64 array of w_last - w_first + 1)."""
+    _check(_lib.zr_debug_average_check(int(w_first), int(w_last), _addr(mismatches), _stream(stream)),
+           "zr_debug_average_check")
 
 
 def zr_debug_reduce(plan: int, grads, g_out, stream=None) -> None:

@@ -34,10 +34,7 @@ zr::LaunchArgs base_args(const zr_plan* p) {
     zr::LaunchArgs a{};
     a.tiles = p->d_tiles;
     a.n_tiles = static_cast<int32_t>(p->tiles.size());
-    a.world_size = p->world_size;
-    const bool pow2 = (p->world_size & (p->world_size - 1)) == 0;
-    a.w_is_pow2 = pow2 ? 1 : 0;
-    a.inv_w = pow2 ? 1.0f / static_cast<float>(p->world_size) : 0.0f;
+    zr::set_world_size(a, p->world_size);
     a.n_targets = p->n_gather_targets;
     a.targets = p->d_gather_targets;
     return a;
@@ -620,6 +617,17 @@ zr_status zr_grad_sumsq(const zr_plan* p, const void* const* grad_ptrs, double* 
     int e = zr::launch_tiles(zr::Pass::kSumsq, a, grad_ptrs, false, false, s);
     if (e != cudaSuccess) return ZR_ERR_CUDA;
     return cuda_status(static_cast<cudaError_t>(zr::launch_clip_combine(clip_args(p, nullptr, d_out), s)));
+}
+
+zr_status zr_debug_average_check(int32_t w_first, int32_t w_last, uint64_t* d_mismatches, zr_stream_t stream) {
+    if (w_first < 1 || w_last < w_first || w_last > ZR_MAX_WORLD_SIZE || !d_mismatches) return ZR_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(d_mismatches) & 7u) != 0) return ZR_ERR_ALIGNMENT;
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ZR_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return ZR_ERR_CUDA;
+    if (major != 10) return ZR_ERR_UNSUPPORTED;
+    return cuda_status(static_cast<cudaError_t>(zr::launch_average_check(
+        w_first, w_last, reinterpret_cast<unsigned long long*>(d_mismatches), stream)));
 }
 
 zr_status zr_debug_reduce(const zr_plan* p, const void* const* grad_ptrs, float* g_out, zr_stream_t stream) {

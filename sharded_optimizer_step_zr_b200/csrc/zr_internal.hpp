@@ -119,7 +119,7 @@ struct LaunchArgs {
     int32_t n_tiles;
     int32_t world_size;
     int32_t w_is_pow2;
-    float inv_w;               // 1/W when W is a power of two (exact)
+    float inv_w;               // 1/W rounded to nearest (exact, and used, for powers of two)
     int32_t reverse;           // CTA b takes tile n_tiles - 1 - b (see the clip pass 2)
     int32_t n_targets;         // 0: bf16 results to param_out; else to each of targets[0..n)
     uint16_t* const* targets;  // device array of parameter buffers (every rank's, for the
@@ -143,6 +143,19 @@ int launch_device_scalars(int64_t* d_step, const zr_adamw& hp, const float* d_lr
 // S_r and the coefficient from the per-tile partials of pass 1: one
 // 128-thread CTA per group of tiles, the last to finish sums the groups.
 int launch_clip_combine(const ClipArgs& c, void* stream);
+
+// W's scalars in the launch arguments: the count, whether it is a power of
+// two, and 1/W rounded to nearest (IEEE single division on the host).
+inline void set_world_size(LaunchArgs& a, int32_t W) {
+    a.world_size = W;
+    a.w_is_pow2 = (W & (W - 1)) == 0 ? 1 : 0;
+    a.inv_w = 1.0f / static_cast<float>(W);
+}
+
+// For every W in [w_first, w_last]: how many of the 2^32 fp32 values s
+// the step's averaging (s / W) maps to other bits than IEEE division does;
+// mismatches[W - w_first] receives the count (a verification hook).
+int launch_average_check(int32_t w_first, int32_t w_last, unsigned long long* mismatches, void* stream);
 // ZeRO-3 gather: copy pieces [first, first + n) from the W shards to dst,
 // where dst holds the global range starting at dst_base, on at most
 // max_ctas CTAs (<= 0: one per piece).  shard_ptrs: host

@@ -84,7 +84,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ float average(float s, const LaunchArgs& a) {
     // Division by a power of two is exact scaling: multiplying by 1/W gives
-    // the same correctly rounded value as the division.
+    // the same correctly rounded value as the division (zr_debug_average_check
+    // compares the two on every fp32 input).
     return a.w_is_pow2 ? __fmul_rn(s, a.inv_w) : __fdiv_rn(s, static_cast<float>(a.world_size));
 }
 
@@ -447,6 +448,23 @@ __global__ void __launch_bounds__(kThreads * kSmallCombineGroups) zr_clip_combin
     }
 }
 
+// Every fp32 bit pattern s through average() for one W, against IEEE
+// division: the count of results whose bits differ (NaN against NaN counts
+// as equal).
+__global__ void __launch_bounds__(kThreads) zr_average_check_kernel(const LaunchArgs a,
+                                                                   unsigned long long* mismatches) {
+    const float w = static_cast<float>(a.world_size);
+    unsigned long long bad = 0;
+    const uint64_t stride = static_cast<uint64_t>(gridDim.x) * kThreads;
+    for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * kThreads + threadIdx.x; i < (1ull << 32); i += stride) {
+        const float s = __uint_as_float(static_cast<uint32_t>(i));
+        const float got = average(s, a);
+        const float want = __fdiv_rn(s, w);
+        if (__float_as_uint(got) != __float_as_uint(want) && !(got != got && want != want)) ++bad;
+    }
+    if (bad) atomicAdd(mismatches, bad);
+}
+
 // Launch configuration for a programmatic dependent launch: the grid may be
 // scheduled while the previous kernel on the stream drains (the kernel's
 // first instruction, griddepcontrol.wait, holds it until that kernel has
@@ -534,6 +552,21 @@ int launch_clip_combine(const ClipArgs& c, void* stream_v) {
     }
     PdlLaunch l(static_cast<unsigned>(n_groups), static_cast<cudaStream_t>(stream_v));
     return cudaLaunchKernelEx(&l.cfg, zr_clip_combine_kernel, c);
+}
+
+int launch_average_check(int32_t w_first, int32_t w_last, unsigned long long* mismatches, void* stream_v) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream_v);
+    const int n = w_last - w_first + 1;
+    cudaError_t e = cudaMemsetAsync(mismatches, 0, sizeof(unsigned long long) * n, s);
+    if (e != cudaSuccess) return e;
+    for (int32_t W = w_first; W <= w_last; ++W) {
+        LaunchArgs a{};
+        set_world_size(a, W);
+        zr_average_check_kernel<<<148 * 32, kThreads, 0, s>>>(a, mismatches + (W - w_first));
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace zr

@@ -128,10 +128,7 @@ extern "C" zr_status zr_step_no_alloc(const zr_plan* p, const void* const* grad_
     zr::LaunchArgs a{};
     a.tiles = d_tiles;
     a.n_tiles = static_cast<int32_t>(p->tiles.size());
-    a.world_size = p->world_size;
-    const bool pow2 = (p->world_size & (p->world_size - 1)) == 0;
-    a.w_is_pow2 = pow2 ? 1 : 0;
-    a.inv_w = pow2 ? 1.0f / static_cast<float>(p->world_size) : 0.0f;
+    zr::set_world_size(a, p->world_size);
     a.master = master;
     a.m = m;
     a.v = v;

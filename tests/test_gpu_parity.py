@@ -327,6 +327,19 @@ def test_clip_all_ranks(W, mode):
         assert bf16_ulp_distance(u16(out_gpu), out_orc).max() <= 1
 
 
+def test_average_matches_ieee_division_for_every_input():
+    """Stage 1's averaging (s / W: a multiply by 1/W for powers of two, a
+    division otherwise) gives the bits of IEEE division for every one of the
+    2^32 fp32 values s -- subnormal quotients included -- and every W the
+    library accepts."""
+    from sharded_optimizer_step_zr_b200 import ZR_MAX_WORLD_SIZE, zr_debug_average_check
+    bad = torch.full((ZR_MAX_WORLD_SIZE,), -1, dtype=torch.int64, device=DEV)
+    zr_debug_average_check(1, ZR_MAX_WORLD_SIZE, bad)
+    torch.cuda.synchronize()
+    bad = bad.cpu().numpy()
+    assert (bad == 0).all(), {w + 1: int(b) for w, b in enumerate(bad) if b}
+
+
 def test_clip_combine_paths_agree():
     """S_r of a plan of at most 8 groups of 1024 tiles (summed by one CTA) and
     of a plan of more groups (a grid of CTAs) follow the same fixed order:
