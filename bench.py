@@ -108,6 +108,9 @@ def parse():
                          "gpu__time_duration.sum) of --small-case's launches of one step into the traffic "
                          "record of --config under profiles/, scaled by owned parameters")
     ap.add_argument("--small-case", default=None, help="workload the capture ran (default: --config)")
+    ap.add_argument("--sweep-w", default=None, metavar="W,W,...",
+                    help="with --sweep: instead of the 40 sweep points, the 1.3B set flat, 25 MB buckets, "
+                         "rank 0, at each of these replica counts (1 - 512)")
     args = ap.parse_args()
     if args.cpu_threads <= 0:
         args.cpu_threads = host_threads()
@@ -857,7 +860,8 @@ def run_zr(args):
 def run_sweep(args):
     """Every point of the 1.3B sweep (bucket cap {1,5,25,100,400} MB x W
     {2,8,32,64} x {flat, whole-tensor}); rank 0, plus the most-loaded rank
-    for whole-tensor points.  Prints one JSON record per point."""
+    for whole-tensor points -- or, with --sweep-w, the flat 25 MB point at
+    each listed W.  Prints one JSON record per point."""
     import torch
     import synth
     from sharded_optimizer_step_zr_b200.plan import ZrPlan
@@ -865,7 +869,11 @@ def run_sweep(args):
     dev = torch.device("cuda", 0)
     stream = torch.cuda.current_stream()
     peak, peak_kind = measured_peak()
-    for wl in synth.sweep_workloads():
+    points = synth.sweep_workloads()
+    if args.sweep_w:
+        points = [synth.Workload(f"sweep_1p3b_flat_w{w}_cap25", "gpt_1p3b", w, (0,), 0, 25, 1e-3, 0.01)
+                  for w in (int(x) for x in args.sweep_w.split(","))]
+    for wl in points:
         probe = ZrPlan(wl.shapes, wl.world_size, 0, wl.mode, wl.bucket_cap_bytes, *wl.hp, bind=False)
         loads = {}
         for s in probe.segments():
