@@ -79,7 +79,14 @@ LARGE = {"llama_7b_w2": dataclasses.replace(synth.WORKLOADS["llama_7b_w64"], nam
                                                           ranks=(13,)),
          "sweep_1p3b_whole_w6_cap25": dataclasses.replace(SWEEP["sweep_1p3b_whole_w8_cap25"],
                                                           name="sweep_1p3b_whole_w6_cap25", world_size=6,
-                                                          ranks=(2,))}
+                                                          ranks=(2,)),
+         # the widest replica counts (up to the library's limit), last rank
+         "sweep_1p3b_flat_w512_cap25": dataclasses.replace(SWEEP["sweep_1p3b_flat_w64_cap25"],
+                                                           name="sweep_1p3b_flat_w512_cap25", world_size=512,
+                                                           ranks=(511,)),
+         "sweep_1p3b_flat_w96_cap25": dataclasses.replace(SWEEP["sweep_1p3b_flat_w64_cap25"],
+                                                          name="sweep_1p3b_flat_w96_cap25", world_size=96,
+                                                          ranks=(50,))}
 
 # Configs 2-4 (and the last rank of config 4, whose offsets pass 2**32; and
 # a shard of more than 2**31 elements), and
@@ -87,7 +94,8 @@ LARGE = {"llama_7b_w2": dataclasses.replace(synth.WORKLOADS["llama_7b_w64"], nam
 # so the checked m and v carry state from the earlier steps.
 THREE_STEP = ([("gpt2_124m_w8", None), ("llama_7b_w64", None), ("llama_7b_w64", 63),
                ("gpt_1p3b_w8_whole_clip", None), ("llama_7b_w2", None),
-               ("sweep_1p3b_flat_w24_cap25", None), ("sweep_1p3b_whole_w6_cap25", None)] +
+               ("sweep_1p3b_flat_w24_cap25", None), ("sweep_1p3b_whole_w6_cap25", None),
+               ("sweep_1p3b_flat_w512_cap25", None), ("sweep_1p3b_flat_w96_cap25", None)] +
               [(f"sweep_1p3b_{m}_w{w}_cap25", None) for m in ("flat", "whole") for w in (2, 8, 32, 64)])
 # The rest of the sweep (caps 1, 5, 100 and 400 MB): one step each.
 ONE_STEP = [(f"sweep_1p3b_{m}_w{w}_cap{c}", None) for m in ("flat", "whole") for w in (2, 8, 32, 64)
