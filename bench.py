@@ -711,7 +711,7 @@ def measure_peer(args, ctx):
     every process)."""
     import torch
     import synth
-    from sharded_optimizer_step_zr_b200.peer import PeerZero
+    from sharded_optimizer_step_zr_b200.peer import PeerFailure, PeerZero
     from sharded_optimizer_step_zr_b200.plan import ZrPlan
 
     wl = workload(args.config)
@@ -719,7 +719,12 @@ def measure_peer(args, ctx):
     shapes = synth.PARAM_SETS[set_name]()
     W, rank, dev = ctx.world, ctx.grank, ctx.dev
     hp = wl.hp[:5] + (0.0,)
-    pz = PeerZero(ctx.dist.group.WORLD, shapes, 0, wl.bucket_cap_bytes, *hp, device=dev, stage=2)
+    try:
+        pz = PeerZero(ctx.dist.group.WORLD, shapes, 0, wl.bucket_cap_bytes, *hp, device=dev, stage=2)
+    except PeerFailure as e:
+        # every rank gets it together (the set-up agrees before anyone steps):
+        # the line keeps the independent-shard measurements
+        return {"mode": "peer", "W": W, "param_set": set_name, "unavailable": str(e)}
     n = pz.plan.owned_numel
     N = pz.plan.total_numel
     segs = pz.plan.segments()

@@ -86,26 +86,52 @@ class PeerZero:
         everyone = [None] * self.world_size
         dist.all_gather_object(everyone, zr_ipc_export(self._shared), group=group)
         self._opened = []
-        grad_bases, second_bases = [], []
-        for w, handle in enumerate(everyone):
-            base = self._shared.data_ptr() if w == self.rank else zr_ipc_open(handle)
-            if w != self.rank:
-                self._opened.append(base)
-            grad_bases.append(base)
-            second_bases.append(base + 2 * half)
-        start = 2 * self.offsets[self.rank]                 # bytes: bf16 elements
-        self.grad_ptrs = None if grad_slot_elems else [b + start for b in grad_bases]
-        # with slots: every replica's slot j starts at byte grad_slot_bases[w][j]
-        self.grad_slot_bases = [[b, b + 2 * slot] for b in grad_bases] if grad_slot_elems else None
-        if stage == 3:
-            self.param_shard = self._shared[half:half + self.plan.owned_numel]
-            self.shard_ptrs = second_bases
-            self.plan.set_param_layout(ZR_PARAMS_OWNED)
-        else:
-            self.param_buffer = self._shared[half:]
-            zr_plan_set_gather_targets(self.plan.handle, second_bases)
-        self._segments = self.plan.segments()
-        dist.barrier(group)
+        error = None
+        try:
+            grad_bases, second_bases = [], []
+            for w, handle in enumerate(everyone):
+                base = self._shared.data_ptr() if w == self.rank else zr_ipc_open(handle)
+                if w != self.rank:
+                    self._opened.append(base)
+                grad_bases.append(base)
+                second_bases.append(base + 2 * half)
+            start = 2 * self.offsets[self.rank]                 # bytes: bf16 elements
+            self.grad_ptrs = None if grad_slot_elems else [b + start for b in grad_bases]
+            # with slots: every replica's slot j starts at byte grad_slot_bases[w][j]
+            self.grad_slot_bases = [[b, b + 2 * slot] for b in grad_bases] if grad_slot_elems else None
+            if stage == 3:
+                self.param_shard = self._shared[half:half + self.plan.owned_numel]
+                self.shard_ptrs = second_bases
+                self.plan.set_param_layout(ZR_PARAMS_OWNED)
+            else:
+                self.param_buffer = self._shared[half:]
+                zr_plan_set_gather_targets(self.plan.handle, second_bases)
+            self._segments = self.plan.segments()
+        except Exception as e:      # e.g. a peer's buffer that cannot be mapped
+            error = e
+        self._agree_set_up(error)
+
+    def _agree_set_up(self, error):
+        """Every rank learns whether every rank mapped its peers' buffers (one
+        all-reduce in place of the set-up's closing barrier).  If any rank
+        failed, every rank unmaps what it opened and raises PeerFailure, so
+        no rank is left waiting for another and none steps."""
+        import torch
+        dist, group = self.dist, self.group
+        dev = self.device if dist.get_backend(group) == "nccl" else torch.device("cpu")
+        flag = torch.tensor([0 if error is None else 1], dtype=torch.int32, device=dev)
+        try:
+            dist.all_reduce(flag, op=dist.ReduceOp.MAX, group=group)
+        except Exception as e:
+            raise PeerFailure(f"set-up: a peer did not arrive ({type(e).__name__}: {e})") from e
+        if int(flag.item()) == 0:
+            return
+        for addr in self._opened:
+            zr_ipc_close(addr)
+        self._opened = []
+        self.plan.close()
+        where = f"this rank ({type(error).__name__}: {error})" if error is not None else "another rank"
+        raise PeerFailure(f"set-up: {where} could not map the peers' buffers") from error
 
     def grad_pieces(self, tensor_index):
         """[(offset in the tensor, view of the owner-major buffer)] of tensor

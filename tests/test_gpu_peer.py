@@ -355,3 +355,49 @@ def test_zero3_module_two_processes(partition, max_norm):
     for r in results:
         assert r[1] is True, r
     assert all(p.exitcode == 0 for p in procs)
+
+
+def _failing_set_up_main(rank, world, port, q):
+    """Rank 1 cannot map its peer's buffer (the IPC call replaced by one that
+    fails, on the host); both ranks must leave the set-up with PeerFailure
+    and keep a working process group."""
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    import torch
+    import torch.distributed as dist
+    import sharded_optimizer_step_zr_b200.peer as peer
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        if rank == 1:
+            def refuse(handle):
+                raise RuntimeError("zr_ipc_open: mapping refused")
+            peer.zr_ipc_open = refuse
+        try:
+            peer.PeerZero(dist.group.WORLD, [(300, 7), (1001,)], 0, 4096)
+            outcome = "constructed"
+        except peer.PeerFailure as e:
+            outcome = str(e)
+        dist.barrier()                       # the group still works after the failure
+        q.put((rank, outcome))
+    except Exception as e:                   # noqa: BLE001 -- reported to the test
+        q.put((rank, f"error {type(e).__name__}: {e}"))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_set_up_failure_on_one_rank_reaches_every_rank():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _port()
+    procs = [ctx.Process(target=_failing_set_up_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = dict(q.get(timeout=240) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+    assert "this rank" in results[1] and "mapping refused" in results[1], results
+    assert "another rank" in results[0], results
