@@ -472,6 +472,18 @@ class ProcessContext:
             else:
                 self.dist.barrier()
 
+    def all_ok(self, ok):
+        """True on every process when `ok` holds on every process (one
+        all-reduce; the local value for one process): a step that failed on
+        one rank is skipped by all of them, with no rank left waiting."""
+        if self.dist is None:
+            return bool(ok)
+        import torch
+        d = self.dev if self.backend == "nccl" else torch.device("cpu")
+        flag = torch.tensor([1 if ok else 0], dtype=torch.int32, device=d)
+        self.dist.all_reduce(flag, op=self.dist.ReduceOp.MIN)
+        return bool(flag.item())
+
     def reduce(self, elapsed_ms, owned_done):
         """(max of elapsed_ms, sum of owned_done) over the processes."""
         if self.dist is None:
@@ -623,9 +635,19 @@ def measure_local(args, ctx, wl, with_e2e, with_cpu):
 
     # end to end through zr_step_host: pinned host gradients in, result out
     e2e = None
+    pinned = None
     if with_e2e and not args.gather_targets:
-        host_grads = [g.cpu().pin_memory() for g in grads]
-        host_out = torch.empty(plan.padded_numel, dtype=torch.bfloat16).pin_memory()
+        try:
+            host_grads = [g.cpu().pin_memory() for g in grads]
+            host_out = torch.empty(plan.padded_numel, dtype=torch.bfloat16).pin_memory()
+        except (RuntimeError, MemoryError) as e:     # pinned host memory is a host resource
+            host_grads = host_out = None
+            pinned = f"{type(e).__name__}: {e}"
+        if not ctx.all_ok(pinned is None):
+            e2e = {"unavailable": f"pinned host buffers could not be allocated on every process"
+                                  f"{' (here: ' + pinned + ')' if pinned else ''}",
+                   "h2d_bytes_per_step": 2 * W * n, "d2h_bytes_per_step": 2 * n}
+    if with_e2e and not args.gather_targets and e2e is None:
         for _ in range(3):
             step_no += 1
             plan.step_host(host_grads, grads, master, m, v, param_out, host_out, step_no, stream)

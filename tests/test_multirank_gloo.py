@@ -178,7 +178,9 @@ def _bench_ctx_worker(rank, world, port, result_q):
         moved = bench.peer_bytes(ctx.world, n)
         ctx.barrier()
         ms, owned = ctx.reduce(5.0 * (rank + 1), n)
-        result_q.put((rank, ctx.grank, ctx.world, n, padded, moved, ms, owned))
+        # a step that failed on one process is skipped by every process
+        agreed = (ctx.all_ok(True), ctx.all_ok(rank != 1), ctx.all_ok(rank != 0))
+        result_q.put((rank, ctx.grank, ctx.world, n, padded, moved, ms, owned, agreed))
     finally:
         ctx.close()
 
@@ -187,7 +189,8 @@ def test_bench_process_context_and_peer_accounting():
     """bench.py's N > 1 plumbing over a real gloo group on the CPU: each
     process's rank, the peer step's owned slices covering the padded set
     (flat, W = 2), the bytes each rank moves over peers, and the max / sum
-    reduction of the timings."""
+    reduction of the timings, and the agreement on a step that failed on
+    one process."""
     world = 2
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
@@ -208,3 +211,4 @@ def test_bench_process_context_and_peer_accounting():
     assert res[0][5] == {"peer_loads": 2 * n0, "peer_stores": 2 * n0, "local_hbm": 28 * n0}
     for r in range(world):
         assert res[r][6] == 10.0 and res[r][7] == float(padded)
+        assert res[r][8] == (True, False, False)
